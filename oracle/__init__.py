@@ -1,0 +1,225 @@
+"""TEST INFRASTRUCTURE ONLY — the CPU oracle for the attention forward pass and
+for the FP8 (e4m3) rotate-and-quantise step.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package. The CUDA
+library never does, and this package imports nothing from the library.
+
+Pieces, each citing the passage it follows:
+
+* :func:`attention` — exact attention in fp64, row by row, in plain C
+  (``attn_oracle.c``). Definition: "Flash Attention" glossary page, first two
+  paragraphs (same result as standard attention; standard attention forms the
+  N x N matrix).
+* :func:`attention_naive` — a second, independently written fp64 routine that
+  materialises the whole N x N score and probability matrices, i.e. the
+  "standard attention" of "FlashAttention-3 (PT)", section "O problema do
+  mecanismo de atenção". Used to cross-check :func:`attention` on tiny inputs.
+* :func:`sylvester_hadamard`, :func:`rotation_matrix`, :func:`rotate` — the
+  orthogonal transform of "FlashAttention-3 (PT)", section "Inovações técnicas",
+  subsection 3 ("Baixa precisão (FP8)"), steps 1 and 4: Q and K multiplied by a
+  random orthogonal (Hadamard) matrix, which leaves Q Kᵀ unchanged.
+* :func:`e4m3_decode`, :func:`e4m3_encode` — the 8-bit e4m3 format (OCP 8-bit
+  floating point, E4M3: bias 7, no infinities, one NaN pattern per sign, largest
+  finite 448), encoded with round-to-nearest-even and saturation.
+* :func:`quantize_per_tensor` — step 3 of the same subsection ("quantização para
+  FP8") with one scale per tensor: descale = amax/448 after rotation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "attn_oracle.c"
+_LIB_PATH = _HERE / "liboracle.so"
+_lib = None
+
+E4M3_MAX = 448.0
+
+
+def build(force: bool = False) -> Path:
+    """Compile ``attn_oracle.c`` into ``liboracle.so`` next to it (gcc, -O2, IEEE math)."""
+    if force or not _LIB_PATH.exists() or _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB_PATH.with_suffix(".so.tmp")
+        subprocess.run(
+            ["gcc", "-std=c99", "-O2", "-fPIC", "-shared", "-pthread", "-o", str(tmp), str(_SRC), "-lm"],
+            check=True,
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(str(_LIB_PATH))
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_attn_rows.argtypes = [
+            dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp, ctypes.c_int,
+        ]
+        lib.oracle_attn_rows.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def _as_f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a torch tensor: widen exactly on the host
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def attention(q, k, v, causal: bool, scale: float, rows=None, threads: int | None = None):
+    """Exact attention of ``[B, H, N, d]`` inputs in fp64.
+
+    ``rows``: optional flat row ids ``(b*H + h)*N + i``; if given, only those rows
+    are computed and the result has shape ``[len(rows), d]`` / ``[len(rows)]``,
+    otherwise ``[B, H, N, d]`` / ``[B, H, N]``. Returns ``(O, LSE)`` with the
+    natural-log LSE.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if q.ndim != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    B, H, N, d = q.shape
+    lib = _load()
+    dp = ctypes.POINTER(ctypes.c_double)
+    if rows is None:
+        nrows = B * H * N
+        rows_arr = None
+        rows_ptr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows = rows_arr.size
+        rows_ptr = rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    o = np.zeros((nrows, d), dtype=np.float64)
+    lse = np.zeros((nrows,), dtype=np.float64)
+    rc = lib.oracle_attn_rows(
+        q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp), B, H, N, d, int(bool(causal)),
+        float(scale), rows_ptr, nrows, o.ctypes.data_as(dp), lse.ctypes.data_as(dp),
+        int(threads or default_threads()),
+    )
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_rows failed with code {rc}")
+    if rows is None:
+        return o.reshape(B, H, N, d), lse.reshape(B, H, N)
+    return o, lse
+
+
+def attention_naive(q, k, v, causal: bool, scale: float, return_probs: bool = False):
+    """Standard attention: materialise S = scale*Q Kᵀ (N x N per head), mask,
+    softmax along keys, then P V. fp64 numpy; for small N only."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    N = q.shape[-2]
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    if causal:
+        future = np.triu(np.ones((N, N), dtype=bool), k=1)  # key j > query i
+        s = np.where(future, -np.inf, s)
+    row_max = s.max(axis=-1, keepdims=True)
+    w = np.exp(s - row_max)
+    denom = w.sum(axis=-1, keepdims=True)
+    p = w / denom
+    o = np.einsum("bhij,bhjd->bhid", p, v)
+    lse = (row_max + np.log(denom))[..., 0]
+    if return_probs:
+        return o, lse, p
+    return o, lse
+
+
+# ----------------------------------------------------------------- rotation --
+def sylvester_hadamard(d: int) -> np.ndarray:
+    """Unnormalised Sylvester Hadamard matrix H_d (d a power of two):
+    H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]."""
+    if d < 1 or d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = np.ones((1, 1), dtype=np.float64)
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def rotation_matrix(d: int, signs=None) -> np.ndarray:
+    """M = D H_d / sqrt(d), D = diag(signs) (identity if ``signs`` is None).
+    Orthogonal: M Mᵀ = I. Applied to row vectors, x' = x M."""
+    h = sylvester_hadamard(d) / np.sqrt(d)
+    if signs is None:
+        return h
+    s = _as_f64(signs).reshape(d)
+    return s[:, None] * h
+
+
+def rotate(x, signs=None) -> np.ndarray:
+    """x M along the last axis, in fp64."""
+    x = _as_f64(x)
+    return x @ rotation_matrix(x.shape[-1], signs)
+
+
+# -------------------------------------------------------------------- e4m3 --
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 code (uint8) as fp64; 0x7F / 0xFF decode to NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)))
+    out = sign * mag
+    return np.where((c & 0x7F) == 0x7F, np.nan, out)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest e4m3 code to each finite fp64 value, ties to even, magnitudes
+    above 448 saturated to 448. Negative values that round to zero give -0 (0x80)."""
+    x = _as_f64(x)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("e4m3_encode takes finite values only")
+    neg = np.signbit(x)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    # Spacing of representable values around a: 2^(e-3) with e = floor(log2 a),
+    # clamped to the subnormal spacing 2^-9 below the smallest normal 2^-6.
+    _, ex = np.frexp(a)  # a = f * 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    val = np.rint(a / quantum) * quantum  # np.rint rounds half to even
+    # val is a representable magnitude (possibly the next binade's first value).
+    _, vex = np.frexp(val)
+    ve = vex - 1
+    normal = val >= 2.0**-6
+    e_field = np.where(normal, ve + 7, 0)
+    m_field = np.where(
+        normal,
+        np.rint(val / np.ldexp(1.0, ve.astype(np.int64)) * 8.0 - 8.0),
+        np.rint(val / 2.0**-9),
+    )
+    code = (e_field.astype(np.int64) << 3) | m_field.astype(np.int64)
+    code = code | np.where(neg, 0x80, 0)
+    return code.astype(np.uint8)
+
+
+def quantize_per_tensor(x, rotate_qk: bool, signs=None, return_scaled: bool = False):
+    """Rotate (optionally) then quantise a whole tensor to e4m3 with one scale.
+
+    x' = x M (if ``rotate_qk``), amax = max |x'|, descale = amax / 448 (1 if
+    amax = 0), codes = e4m3_encode(x' * 448 / amax). Returns ``(codes, descale)``
+    and, with ``return_scaled``, also the unrounded ``x' * 448 / amax``.
+    """
+    xr = rotate(x, signs) if rotate_qk else _as_f64(x)
+    amax = float(np.max(np.abs(xr))) if xr.size else 0.0
+    if amax == 0.0:
+        scaled = np.zeros_like(xr)
+        descale = 1.0
+    else:
+        scaled = xr * (E4M3_MAX / amax)
+        descale = amax / E4M3_MAX
+    codes = e4m3_encode(scaled)
+    if return_scaled:
+        return codes, descale, scaled
+    return codes, descale
