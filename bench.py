@@ -1,0 +1,383 @@
+"""Benchmark of the fused attention forward on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input of
+the B=4, H=16, N=2048, d=128 workload (Q, K, V ~ N(0,1) bf16, scale 1/sqrt(128)):
+  1. BF16 forward, non-causal;   2. BF16 forward, causal;
+  3. Hadamard rotate + e4m3 quantise of Q and of K;   4. e4m3-QK forward, non-causal.
+Metric: attention TFLOPS = sum of 4*B*H*N^2*d (halved when causal) over the
+three forward passes / step time. L2 (126 MB) is flushed between steps by
+writing a 512 MB buffer outside the timed events, since the inputs (100 MB)
+would otherwise stay resident.
+
+``--impl reference`` times the CPU oracle instead (rank 0 only), on a bounded
+row sample of the same workload per step.
+
+Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
+torch.distributed.run, one rank per GPU, each rank its own batch: weak scaling,
+no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+from io_aware_exact_17_b200 import inputs as fa_inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (4·B·H·N²·d, ½ if causal) and % of B200 BF16/FP8 peak"
+B, H, N, D = 4, 16, 2048, 128
+SEED = 1001
+WORKLOAD = f"b{B}h{H}n{N}d{D}: bf16 fwd non-causal + bf16 fwd causal + rotate/quantise Q,K + e4m3-QK fwd non-causal"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_fwd(causal: bool) -> float:
+    f = 4.0 * B * H * N * N * D
+    return f / 2 if causal else f
+
+
+STEP_FLOPS = flops_fwd(False) + flops_fwd(True) + flops_fwd(False)
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+        except Exception:
+            pass
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------- distributed --
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (identity for one rank)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        # nvidia-smi numbers GPUs physically; address ours by UUID instead.
+        try:
+            uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(gpu_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- GPU step --
+class Step:
+    """All buffers of one step, allocated once; run() enqueues the step's kernels
+    on the current stream, bracketing each kernel group with CUDA events."""
+
+    def __init__(self, seed: int):
+        import io_aware_exact_17_b200 as fa
+
+        self.fa = fa
+        q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
+        self.signs = fa_inputs.hadamard_signs(D, seed).cuda()
+        self.q_h, self.k_h, self.v_h = (t.pin_memory() for t in (q, k, v))
+        self.q, self.k, self.v = (t.cuda() for t in (q, k, v))
+        shp = (B, H, N, D)
+        self.o = [torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+        self.lse = [torch.empty((B, H, N), dtype=torch.float32, device="cuda") for _ in range(3)]
+        self.q8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
+        self.k8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
+        self.desc = torch.empty(2, dtype=torch.float32, device="cuda")
+        self.o_h = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+        self.lse_h = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(3)]
+        self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 7  # 3 attention kernels + 2 x (amax, quantise)
+
+    def flush_l2(self):
+        self.flush_buf.zero_()
+
+    def run(self, ev=None):
+        fa = self.fa
+        if ev is not None:
+            ev[0].record()
+        fa.fwd(self.q, self.k, self.v, causal=False, out=self.o[0], lse=self.lse[0])
+        if ev is not None:
+            ev[1].record()
+        fa.fwd(self.q, self.k, self.v, causal=True, out=self.o[1], lse=self.lse[1])
+        if ev is not None:
+            ev[2].record()
+        fa.hadamard_quant(self.q, rotate=True, signs=self.signs, out=self.q8, descale=self.desc[0:1])
+        fa.hadamard_quant(self.k, rotate=True, signs=self.signs, out=self.k8, descale=self.desc[1:2])
+        if ev is not None:
+            ev[3].record()
+        fa.fwd(self.q8, self.k8, self.v, causal=False, qk_descale=self.desc, out=self.o[2], lse=self.lse[2])
+        if ev is not None:
+            ev[4].record()
+
+    def run_e2e(self):
+        """The step through the same public calls with host buffers: pinned
+        host -> device copies of Q, K, V, the step, device -> host copies of
+        every O and LSE."""
+        self.q.copy_(self.q_h, non_blocking=True)
+        self.k.copy_(self.k_h, non_blocking=True)
+        self.v.copy_(self.v_h, non_blocking=True)
+        self.run()
+        for i in range(3):
+            self.o_h[i].copy_(self.o[i], non_blocking=True)
+            self.lse_h[i].copy_(self.lse[i], non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.q_h, self.k_h, self.v_h))
+
+    @property
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.o_h + self.lse_h)
+
+
+def time_steps(step: Step, steps: int, warmup: int, world: int):
+    for _ in range(warmup):
+        step.flush_l2()
+        step.run()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step.flush_l2()
+        step.run(evs[i])
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)]
+    return per  # ms: [bf16 nc, bf16 causal, quant Q+K, fp8 nc] per step
+
+
+def time_e2e(step: Step, steps: int, warmup: int, world: int):
+    for _ in range(warmup):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    total = 0.0
+    for _ in range(steps):
+        step.flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step.run_e2e()
+        e1.record()
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    dist_barrier(world)
+    return total / steps
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_sample(target_s: float, seed: int):
+    """Time the oracle (as it stands) on a row sample of the three attention
+    passes of the step, sized for about ``target_s`` seconds. Returns
+    (flops, seconds, threads, rows_per_pass)."""
+    import numpy as np
+
+    import oracle
+
+    q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(seed)
+
+    def run(rows_n):
+        rows = rng.integers(0, B * H * N, rows_n)
+        fl = 0.0
+        t0 = time.perf_counter()
+        for causal in (False, True, False):
+            oracle.attention(qd, kd, vd, causal, D ** -0.5, rows=rows, threads=threads)
+            i = rows % N
+            fl += float(np.sum(4.0 * D * (i + 1))) if causal else 4.0 * N * D * rows_n
+        return fl, time.perf_counter() - t0
+
+    probe_rows = max(threads * 4, 64)
+    fl, dt = run(probe_rows)
+    rows_n = int(min(B * H * N, max(probe_rows, probe_rows * target_s / max(dt, 1e-3))))
+    fl, dt = run(rows_n)
+    return fl, dt, threads, rows_n
+
+
+# ------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        if rank == 0:
+            warm = [oracle_sample(2.0, SEED + 100 + i) for i in range(args.warmup)]
+            del warm
+            runs = [oracle_sample(args.cpu_seconds / 2, SEED + i) for i in range(args.steps)]
+            fl = sum(r[0] for r in runs)
+            sec = sum(r[1] for r in runs)
+            val = fl / sec / 1e12
+            line = {
+                "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1))",
+                "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "l2": "n/a (CPU)"},
+                "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": runs[0][2], "kind": "oracle",
+                                 "sample": f"{runs[0][3]} random query rows per attention pass per step, "
+                                           "3 passes (non-causal, causal, non-causal), exact fp64"},
+                "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            }
+            print(json.dumps(line), flush=True)
+        dist_done(world)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    step = Step(SEED + rank)
+    with ClockSampler(local) as clk:
+        per = time_steps(step, args.steps, args.warmup, world)
+    e2e_ms = time_e2e(step, max(3, args.steps // 4), 3, world)
+    step_ms = [sum(p) for p in per]
+    ms_local = statistics.mean(step_ms)
+    ms = dist_max(ms_local, world)
+    e2e_ms = dist_max(e2e_ms, world)
+    comp = [statistics.mean(p[j] for p in per) for j in range(4)]
+    comp = [dist_max(c, world) for c in comp]
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+
+    if rank == 0:
+        value = world * STEP_FLOPS / (ms * 1e-3) / 1e12
+        nc_ms = comp[0]
+        achieved = flops_fwd(False) / (nc_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+            "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (512 MB write outside the timed events)"},
+            "breakdown_ms": {"bf16_noncausal": comp[0], "bf16_causal": comp[1], "rotate_quant_qk": comp[2],
+                             "e4m3qk_noncausal": comp[3]},
+            "breakdown_tflops": {"bf16_noncausal": flops_fwd(False) / comp[0] / 1e9,
+                                 "bf16_causal": flops_fwd(True) / comp[1] / 1e9,
+                                 "e4m3qk_noncausal": flops_fwd(False) / comp[3] / 1e9},
+            "roofline": {"kernel": "attn_fwd_kernel<128,2,nc,bf16>", "bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "peak_source": f"{peak_src} cuBLAS bf16 (burst)"},
+            "e2e": {"value": world * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"]},
+        }
+        if not args.no_cpu_baseline and world == 1:
+            fl, sec, cores, rows_n = oracle_sample(args.cpu_seconds, SEED)
+            line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                    "sample": f"{rows_n} random query rows x 3 attention passes of the workload, "
+                                              f"exact fp64, {sec:.1f} s"}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

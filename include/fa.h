@@ -1,0 +1,117 @@
+/*
+ * fa.h — C ABI of libfa.so: fused exact-attention forward on B200 (sm_100a),
+ * BF16 and FP8-e4m3 (for Q Kᵀ), and the Hadamard rotate-and-quantise step that
+ * prepares FP8 queries and keys.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" must point to memory of the CUDA device that is
+ *    current on the calling thread; the caller allocates and owns every buffer.
+ *    The library allocates no device memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *    enqueued on it; nothing synchronises the host.
+ *  - Argument errors are returned before anything is enqueued. A failed launch
+ *    returns FA_ERR_CUDA. A device-side failure (a bounded wait that ran out)
+ *    is recorded on the device and read with fa_device_status().
+ *  - Tensors are dense and row-major ("contiguous"), with the layouts stated.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, size < 1, bad scale, workspace too small */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension / dtype combination not built */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer is not aligned as required */
+  FA_ERR_CUDA = 4,        /* a CUDA call or a launch failed */
+  FA_ERR_TIMEOUT = 5      /* (device status only) a bounded wait inside a kernel ran out */
+} fa_status;
+
+typedef enum {
+  FA_BF16 = 0, /* Q and K are bf16 */
+  FA_E4M3 = 1  /* Q and K are e4m3 codes (one byte each) with per-tensor descales */
+} fa_dtype;
+
+/*
+ * fa_fwd — exact attention forward with per-row log-sum-exp.
+ *
+ * Defined by: "Flash Attention" glossary page, paragraphs 1-2 (the output equals
+ * standard attention softmax(scale Q Kᵀ) V; the N x N matrix is never written to
+ * HBM, tiles are processed on chip with an online, numerically stable softmax),
+ * and "FlashAttention-3 (PT)", section "FlashAttention e FlashAttention-2"
+ * (tiling; matmul, softmax and matmul fused in one kernel). For every batch b,
+ * head h and query row i:
+ *   O[b,h,i,:] = sum_j w_ij V[b,h,j,:],  w_ij = exp(z_ij) / sum_j' exp(z_ij'),
+ *   z_ij = scale * Q[b,h,i,:] . K[b,h,j,:],   LSE[b,h,i] = ln sum_j exp(z_ij),
+ * with j over 0..N-1, or over 0..i when `causal` != 0 (square mask, top-left).
+ *
+ * q, k    device, [B][H][N][d]; bf16 when qk_dtype = FA_BF16, e4m3 codes when
+ *         FA_E4M3 (then Q = dq * decode(q), K = dk * decode(k)). 16-byte aligned.
+ * v       device, bf16 [B][H][N][d], 16-byte aligned.
+ * o       device, bf16 [B][H][N][d] output (round to nearest even), 16-byte aligned.
+ * lse     device, fp32 [B][H][N] output (natural log), 4-byte aligned; may be NULL.
+ * B, H, N >= 1; d in {64, 128, 256} for FA_BF16, {128, 256} for FA_E4M3.
+ * scale   finite and > 0 (usually 1/sqrt(d)).
+ * descale_qk  device, two fp32 {dq, dk} for FA_E4M3 (as written by
+ *         fa_hadamard_quant); ignored (may be NULL) for FA_BF16.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                 int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, void* stream);
+
+/* Bytes of device workspace fa_hadamard_quant needs (a 4-byte amax word, padded). */
+#define FA_QUANT_WORKSPACE_BYTES 256
+
+/*
+ * fa_hadamard_quant — rotate (optionally) and quantise one tensor to e4m3 with a
+ * single scale.
+ *
+ * Defined by: "FlashAttention-3 (PT)", section "Inovações técnicas", subsection 3
+ * ("Baixa precisão (FP8)"), steps 1-4: queries and keys are multiplied by a random
+ * orthogonal (Hadamard) matrix, which spreads outlier coordinates, then quantised
+ * to FP8; Q Kᵀ is unchanged by the rotation. Per row r:
+ *   x'[r,:] = x[r,:] diag(signs) H_d / sqrt(d)   (H_d: Sylvester Hadamard)  if rotate,
+ *   x'[r,:] = x[r,:]                                                       otherwise;
+ *   amax = max |x'| over the whole tensor;  descale = amax / 448 (1 if amax = 0);
+ *   out[r,c] = e4m3(x'[r,c] * 448 / amax), round to nearest even, saturating.
+ *
+ * x           device, bf16 [rows][d], 16-byte aligned (e.g. [B][H][N][d], rows = B*H*N);
+ *             may be NULL when rows = 0.
+ * out         device, e4m3 codes [rows][d], 16-byte aligned; may be NULL when rows = 0.
+ * descale_out device, one fp32 (written last, by the second kernel).
+ * rows >= 0;  d in {64, 128, 256}.
+ * rotate      0 = quantise only, 1 = rotate first.
+ * signs       device, d fp32 values +-1 (16-byte aligned), or NULL for no sign flips.
+ * workspace   device scratch of >= FA_QUANT_WORKSPACE_BYTES bytes, 16-byte aligned,
+ *             owned by the caller; its contents are overwritten. Calls that overlap on
+ *             the GPU must not share one workspace.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_t rows, int d, int rotate,
+                            const float* signs, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(fa_status s);
+
+/*
+ * fa_device_status — read and clear the device-side status of the current
+ * device. Synchronises the device first. *code receives FA_OK or FA_ERR_TIMEOUT,
+ * *site an internal wait-site number and *block the CTA index that recorded it;
+ * any output pointer may be NULL. Returns FA_ERR_CUDA if the read itself failed.
+ */
+fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
+
+/* ABI version of this header: 1. */
+int fa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

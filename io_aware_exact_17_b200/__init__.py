@@ -1,0 +1,17 @@
+"""Fused exact-attention forward for B200 (sm_100a): BF16 and FP8-e4m3 kernels,
+and the Hadamard rotate-and-quantise step of the FP8 path.
+
+The compute lives in ``libfa.so`` (CUDA, built from ``csrc/``); this package is
+its Python binding. Importing the package does not load the library; the first
+call does, and fails loudly if the library or a GPU is missing.
+"""
+from .binding import (  # noqa: F401
+    FaError,
+    device_status,
+    fwd,
+    hadamard_quant,
+    library_path,
+    load_library,
+)
+
+__all__ = ["fwd", "hadamard_quant", "device_status", "load_library", "library_path", "FaError"]

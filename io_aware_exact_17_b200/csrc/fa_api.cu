@@ -1,0 +1,177 @@
+// fa_api.cu — the C ABI declared in include/fa.h: argument checks, TMA tensor
+// maps, and the launches of the attention and quantisation kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/fa.h"
+#include "attn_fwd.cuh"
+#include "quant.cuh"
+#include "tmap.h"
+
+namespace {
+
+using fa::FwdCfg;
+using fa::FwdParams;
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+bool set_smem_once(K kernel, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (*done_mask & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  *done_mask |= bit;
+  return true;
+}
+
+template <int D, int NQ, bool CAUSAL, bool QK_FP8>
+fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                     float scale, const float* descale_qk, cudaStream_t stream) {
+  using C = FwdCfg<D, NQ, QK_FP8>;
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV;
+  const CUtensorMapDataType qk_type = QK_FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!fa::make_tmap_3d(&tmQ, q, qk_type, C::EQK, D, N, BH, 128 / C::EQK, C::BM) ||
+      !fa::make_tmap_3d(&tmK, k, qk_type, C::EQK, D, N, BH, 128 / C::EQK, C::BN) ||
+      !fa::make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, C::BN))
+    return FA_ERR_CUDA;
+  auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8>;
+  static unsigned long long smem_done = 0;
+  if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
+  FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.descale_qk = descale_qk;
+  p.N = N;
+  p.n_qb = (N + NQ * C::BM - 1) / (NQ * C::BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = static_cast<long long>(p.n_qb) * BH;
+  kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t rows, int rotate, const float* signs,
+                       unsigned int* amax, cudaStream_t stream) {
+  using QC = fa::QuantCfg<D>;
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  const int64_t steps = (rows + QC::ROWS_PER_STEP - 1) / QC::ROWS_PER_STEP;  // warp-steps of work
+  const int64_t warps_per_block = fa::kQuantThreads / 32;
+  int64_t blocks = (steps + warps_per_block - 1) / warps_per_block;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident blocks of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  uint8_t* ob = static_cast<uint8_t*>(out);
+  if (rotate) {
+    fa::quant_amax_kernel<D, true><<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, rows, signs, amax);
+    fa::quant_apply_kernel<D, true>
+        <<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, ob, rows, signs, amax, descale_out);
+  } else {
+    fa::quant_amax_kernel<D, false><<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, rows, nullptr, amax);
+    fa::quant_apply_kernel<D, false>
+        <<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, ob, rows, nullptr, amax, descale_out);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (qk_dtype != FA_BF16 && qk_dtype != FA_E4M3) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (qk_dtype == FA_E4M3 && d == 64) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return FA_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  if (qk_dtype == FA_E4M3) {
+    if (descale_qk == nullptr) return FA_ERR_INVALID_ARG;
+    if (!aligned(descale_qk, 4)) return FA_ERR_ALIGNMENT;
+  }
+  const int rows_per_cta = d == 256 ? 128 : 256;
+  const long long n_qb = (static_cast<long long>(N) + rows_per_cta - 1) / rows_per_cta;
+  if (n_qb * B * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool c = causal != 0;
+  if (qk_dtype == FA_BF16) {
+    switch (d) {
+      case 64: return c ? launch_fwd<64, 2, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
+                        : launch_fwd<64, 2, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
+      case 128: return c ? launch_fwd<128, 2, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
+                         : launch_fwd<128, 2, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
+      default: return c ? launch_fwd<256, 1, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
+                        : launch_fwd<256, 1, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
+    }
+  }
+  switch (d) {
+    case 128: return c ? launch_fwd<128, 2, true, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s)
+                       : launch_fwd<128, 2, false, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s);
+    default: return c ? launch_fwd<256, 1, true, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s)
+                      : launch_fwd<256, 1, false, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s);
+  }
+}
+
+fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_t rows, int d, int rotate,
+                            const float* signs, void* workspace, size_t workspace_bytes, void* stream) {
+  if (descale_out == nullptr || workspace == nullptr) return FA_ERR_INVALID_ARG;
+  if (rows < 0 || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || out == nullptr)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < FA_QUANT_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (rows > (static_cast<int64_t>(1) << 40)) return FA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(descale_out, 4))
+    return FA_ERR_ALIGNMENT;
+  if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
+  const float* sg = rotate ? signs : nullptr;
+  unsigned int* amax = static_cast<unsigned int*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_quant<64>(x, out, descale_out, rows, rotate, sg, amax, s);
+    case 128: return launch_quant<128>(x, out, descale_out, rows, rotate, sg, amax, s);
+    default: return launch_quant<256>(x, out, descale_out, rows, rotate, sg, amax, s);
+  }
+}
+
+const char* fa_status_string(fa_status st) {
+  switch (st) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension or dtype";
+    case FA_ERR_ALIGNMENT: return "misaligned pointer";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+  }
+  return "unknown status";
+}
+
+fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  fa::DevStatus h;
+  if (cudaMemcpyFromSymbol(&h, fa::g_fa_status, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  const fa::DevStatus zero = {0, 0, 0, 0};
+  if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  if (code) *code = static_cast<int>(h.code);
+  if (site) *site = h.site;
+  if (block) *block = h.block;
+  return FA_OK;
+}
+
+int fa_abi_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,28 @@
+"""Small shared pieces of the GPU parity tests (comparison and tolerances)."""
+import numpy as np
+import torch
+
+# Tolerances of the forward pass against the fp64 oracle (N(0,1) inputs):
+# BF16 O max-abs 1e-2 and LSE max-abs 1e-3; FP8 relative RMSE 5e-2.
+BF16_O_ATOL = 1e-2
+BF16_LSE_ATOL = 1e-3
+FP8_REL_RMSE = 5e-2
+
+
+def bf16_out_tol(o_ref: np.ndarray) -> np.ndarray:
+    """Element tolerance for inputs outside the N(0,1), scale 1/sqrt(d) regime:
+    the 1e-2 bound plus the bf16 half-ulp of the exact output (2^-8 |O|), since
+    O is returned rounded to bf16 and large-logit rows can have |O| near max|V|."""
+    return BF16_O_ATOL + 2.0**-8 * np.abs(o_ref)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def rel_rmse(a: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.linalg.norm(a - ref) / np.linalg.norm(ref))
+
+
+def max_abs(a: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.max(np.abs(a - ref))) if a.size else 0.0
