@@ -237,7 +237,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
     const int kmax = CAUSAL ? min(qrow, p.N - 1) : p.N - 1;  // last visible key of this row
     float m_ref = -INFINITY;  // reference max, scaled log2 units
-    float l = 0.f;
+    float l_exact = 0.f;      // sum of the fp32 weights: gives the LSE
+    float l_round = 0.f;      // sum of the bf16-rounded weights P uses: normalises O
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
@@ -255,16 +256,51 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int c = 0; c < 128; ++c)
           if (kbase + c > kmax) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(s[0]);
+      // Row max: four independent chains of 3-input max.
+      float a0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
+      float a1 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
+      float a2 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
+      float a3 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-      const float mx_s = mx * s_log2;
+      for (int c = 8; c < 128; c += 8) {
+        a0 = fmax3(a0, __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
+        a1 = fmax3(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        a2 = fmax3(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        a3 = fmax3(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+      }
+      const float mx_s = fmax3(a0, a1, fmaxf(a2, a3)) * s_log2;
       const bool grow = mx_s > m_ref + 8.0f;
       const float m_new = grow ? mx_s : m_ref;
       const float alpha = ex2_approx(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
+      m_ref = m_new;
+      // p = 2^(x*s - m): one packed FMA per pair, then the SFU exp2; P packs to bf16.
+      const uint64_t s2 = f2_pack(s_log2, s_log2);
+      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc_e[2] = {0ull, 0ull}, acc_r[2] = {0ull, 0ull};
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        float t0, t1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), s2, nm2), t0, t1);
+        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+        const uint32_t pk = pack_bf16x2(p0, p1);
+        const int a = (c >> 1) & 1;
+        acc_e[a] = f2_add(acc_e[a], f2_pack(p0, p1));
+        acc_r[a] = f2_add(acc_r[a], f2_pack(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
+        s[c >> 1] = pk;
+      }
+      tmem_st32(tS + 0, &s[0]);
+      tmem_st32(tS + 32, &s[32]);
+      float e0, e1, e2, e3, r0, r1, r2, r3;
+      f2_unpack(acc_e[0], e0, e1);
+      f2_unpack(acc_e[1], e2, e3);
+      f2_unpack(acc_r[0], r0, r1);
+      f2_unpack(acc_r[1], r2, r3);
+      l_exact = l_exact * alpha + ((e0 + e1) + (e2 + e3));
+      l_round = l_round * alpha + ((r0 + r1) + (r2 + r3));
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // Rescale this warp's O rows in TMEM (PV of tile j-1 has completed: the
-        // commit that signalled S_t for tile j also covers it).
+        // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
+        // completed: the commit that signalled S_t for tile j also covers it, and
+        // PV of tile j is issued only after this warpgroup arrives below.
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t ov[32];
@@ -275,32 +311,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tmem_st32(tO + c0, ov);
         }
       }
-      l *= alpha;
-      m_ref = m_new;
-      const float neg_m = -m_ref;
-      // l sums the bf16-rounded weights the PV product actually uses, so the
-      // weights of a row sum to exactly one in the final O / l.
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), s_log2, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), s_log2, neg_m));
-        const uint32_t pk = pack_bf16x2(p0, p1);
-        sum4[(c >> 1) & 3] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xFFFF0000u);
-        s[c >> 1] = pk;
-      }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      tmem_st32(tS + 0, &s[0]);
-      tmem_st32(tS + 32, &s[32]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_p[t]);
-      l += sum;
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = 1.0f / l_round;
       const bool in_range = qrow < p.N;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? qrow : 0)) * D;
 #pragma unroll 1
@@ -319,7 +337,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       if (in_range && p.lse != nullptr)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     }
   }
 
