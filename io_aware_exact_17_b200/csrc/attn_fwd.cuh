@@ -17,13 +17,15 @@
 //      warp 4*NQ       : tcgen05.mma issuer (one elected thread), TMEM owner;
 //      warp 4*NQ+1     : TMA producer (Q once; K_j, V_j through a ring of
 //                        shared-memory slots, prefetched ahead: section 2);
-//  * S_t = Q_t K_jᵀ accumulates in TMEM (128 fp32 columns); softmax reads it,
-//    writes P_t = exp2(..) as bf16 over the same columns, and the MMA warp
-//    issues O_t += P_t V_j with P_t taken straight from TMEM;
+//      warps 4*NQ+2,3  : idle (they complete the last warpgroup for setmaxnreg);
+//  * S_t = Q_t K_jᵀ accumulates in TMEM (128 fp32 columns); softmax reads it
+//    in four 32-column chunks, each load overlapping the previous chunk's exps,
+//    writes P_t = exp2(..) as bf16 pairs over the first 64 columns, and the MMA
+//    warp issues O_t += P_t V_j with P_t taken straight from TMEM;
 //  * online softmax in base 2 with the scale folded into one FMA; the running
 //    reference max is moved only when a row's max grows by more than 2^8, so
 //    the O rescale (a TMEM read-modify-write) is rare. The final O / l and the
-//    LSE use the same reference, so the result is exact, not approximated.
+//    LSE use the same reference, so the result is exact, not approximated;
 //  * the QK product can take e4m3 Q and K (the FP8 path with Hadamard-rotated
 //    inputs: section "Inovações técnicas", 3); P and V stay bf16.
 #pragma once
@@ -35,6 +37,13 @@
 namespace fa {
 
 __device__ DevStatus g_fa_status;  // first device-side error of any launch
+
+#ifndef FA_REG_SOFTMAX
+#define FA_REG_SOFTMAX 208
+#endif
+#ifndef FA_REG_OTHER
+#define FA_REG_OTHER 88
+#endif
 
 template <int D, int NQ, bool QK_FP8>
 struct FwdCfg {
@@ -50,11 +59,21 @@ struct FwdCfg {
   static constexpr int RING_BUDGET = 200 * 1024 - NQ * Q_TILE;
   static constexpr int NSLOT = (RING_BUDGET / SLOT) > 6 ? 6 : (RING_BUDGET / SLOT);
   static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + NSLOT * SLOT;
-  static constexpr int MMA_WARP = 4 * NQ;
-  static constexpr int TMA_WARP = 4 * NQ + 1;
-  static constexpr int THREADS = (4 * NQ + 2) * 32;
+  static constexpr int SOFTMAX_WARPS = 4 * NQ;
+  static constexpr int MMA_WARP = SOFTMAX_WARPS;
+  static constexpr int TMA_WARP = SOFTMAX_WARPS + 1;
+  static constexpr int THREADS = (SOFTMAX_WARPS + 4) * 32;  // whole warpgroups
+  // NQ = 2 (384 threads) launches at 168 registers per thread; setmaxnreg then
+  // moves registers from the last warpgroup to the two softmax warpgroups.
+  static constexpr bool SPLIT_REGS = NQ == 2;
+  static constexpr int REG_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
+  static constexpr int REG_SOFTMAX = FA_REG_SOFTMAX;  // per softmax thread after setmaxnreg.inc
+  static constexpr int REG_OTHER = FA_REG_OTHER;      // per thread of the last warpgroup after .dec
+  static_assert(!SPLIT_REGS || SOFTMAX_WARPS * 32 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * REG_LAUNCH,
+                "register split exceeds the block's launch allocation");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL(int t) { return static_cast<uint32_t>(t) * 128u; }
+  static constexpr uint32_t P_COL(int t) { return S_COL(t); }  // 64 columns of bf16 pairs over S
   static constexpr uint32_t O_COL(int t) { return static_cast<uint32_t>(NQ) * 128u + static_cast<uint32_t>(t * D); }
   static_assert(D == 64 || D == 128 || D == 256, "head dim");
   static_assert(QK_CHUNKS >= 1, "an e4m3 row must fill a 128-byte swizzle row");
@@ -78,10 +97,108 @@ struct FwdParams {
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return;
   const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return;
-    if ((it & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) return;
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+}
+
+#ifndef FA_EXP_POLY_EVERY
+#define FA_EXP_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FA_EXP_POLY_EVERY;  // 1 pair in kPolyEvery uses the polynomial (0: none)
+
+// Exponentials of one 32-key chunk of a row of S: p = 2^(x*s - m), packed to
+// bf16 pairs into pk[0..15]; accumulates the fp32 weights and the rounded ones
+// into the packed-pair sums and (WITH_MAX) the raw-score max into mx[0..3].
+// With EMU (a tile with no masked key) one pair in kPolyEvery goes to the
+// FMA-pipe polynomial.
+template <bool EMU, bool WITH_MAX>
+__device__ __forceinline__ void exp_chunk32(const uint32_t* s, uint32_t* pk, uint64_t s2, uint64_t nm2,
+                                            uint64_t* acc_e, uint64_t* acc_r, float* mx) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    float t0, t1, p0, p1;
+    if (WITH_MAX) mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), s2, nm2), t0, t1);
+    if (EMU && kPolyEvery > 0 && ((c >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+      exp2_poly_x2(t0, t1, p0, p1);
+    } else {
+      p0 = ex2_approx(t0);
+      p1 = ex2_approx(t1);
+    }
+    const uint32_t q = pack_bf16x2(p0, p1);
+    const int a = (c >> 1) & 1;
+    acc_e[a] = f2_add(acc_e[a], f2_pack(p0, p1));
+    acc_r[a] = f2_add(acc_r[a], f2_pack(__uint_as_float(q << 16), __uint_as_float(q & 0xFFFF0000u)));
+    pk[c >> 1] = q;
   }
+}
+
+__device__ __forceinline__ void mask_chunk32(uint32_t* s, int kbase, int kmax) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    if (kbase + c > kmax) s[c] = __float_as_uint(-INFINITY);
+}
+
+// One row of S (128 keys, from TMEM at tS) through the exponentials: the four
+// 32-column loads are software-pipelined with the exps of the previous chunk
+// (tcgen05.wait::ld waits for all earlier loads, so chunk c+1 is issued before
+// chunk c is computed). P is packed into pk[0..63]. Returns the fp32 and rounded
+// weight sums and, with WITH_MAX, the max of the raw scores.
+template <bool EMU, bool WITH_MAX>
+__device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, uint32_t* pk, float s_log2, float m_ref,
+                                            int kbase, int kmax, bool masked, float& sum_e, float& sum_r,
+                                            float& raw_max) {
+  const uint64_t s2 = f2_pack(s_log2, s_log2);
+  const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+  uint64_t acc_e[2] = {0ull, 0ull}, acc_r[2] = {0ull, 0ull};
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  tmem_ld32(tS + 0, &s[0]);
+  tmem_wait_ld_dep32(&s[0]);
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    if (ch < 3) tmem_ld32(tS + 32 * (ch + 1), &s[32 * (ch + 1)]);
+    if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
+    exp_chunk32<EMU, WITH_MAX>(&s[32 * ch], &pk[16 * ch], s2, nm2, acc_e, acc_r, mx);
+    if (ch < 3) tmem_wait_ld_dep32(&s[32 * (ch + 1)]);
+  }
+  float e0, e1, e2, e3, r0, r1, r2, r3;
+  f2_unpack(acc_e[0], e0, e1);
+  f2_unpack(acc_e[1], e2, e3);
+  f2_unpack(acc_r[0], r0, r1);
+  f2_unpack(acc_r[1], r2, r3);
+  sum_e = (e0 + e1) + (e2 + e3);
+  sum_r = (r0 + r1) + (r2 + r3);
+  if (WITH_MAX) raw_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// `masked` must be warp-uniform: both paths issue tcgen05.ld.
+template <bool WITH_MAX>
+__device__ __forceinline__ void softmax_row_dispatch(uint32_t tS, uint32_t* s, uint32_t* pk, float s_log2,
+                                                     float m_ref, int kbase, int kmax, bool masked, float& se,
+                                                     float& sr, float& mx) {
+  if (masked)
+    softmax_row<false, WITH_MAX>(tS, s, pk, s_log2, m_ref, kbase, kmax, true, se, sr, mx);
+  else
+    softmax_row<true, WITH_MAX>(tS, s, pk, s_log2, m_ref, kbase, kmax, false, se, sr, mx);
+}
+
+// Raw-score max of one row of S (first tile only, before any reference exists).
+__device__ __forceinline__ float row_max_tmem(uint32_t tS, uint32_t* s, int kbase, int kmax, bool masked) {
+  float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    tmem_ld32(tS + 32 * ch, &s[32 * ch]);
+    tmem_wait_ld_dep32(&s[32 * ch]);
+    if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
+#pragma unroll
+    for (int c = 0; c < 32; c += 8) {
+      a[0] = fmax3(a[0], __uint_as_float(s[32 * ch + c + 0]), __uint_as_float(s[32 * ch + c + 1]));
+      a[1] = fmax3(a[1], __uint_as_float(s[32 * ch + c + 2]), __uint_as_float(s[32 * ch + c + 3]));
+      a[2] = fmax3(a[2], __uint_as_float(s[32 * ch + c + 4]), __uint_as_float(s[32 * ch + c + 5]));
+      a[3] = fmax3(a[3], __uint_as_float(s[32 * ch + c + 6]), __uint_as_float(s[32 * ch + c + 7]));
+    }
+  }
+  return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
 }
 
 template <int D, int NQ, bool CAUSAL, bool QK_FP8>
@@ -119,7 +236,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(&bar_drain, 1);
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&bar_s[t], 1);
-      mbar_init(&bar_p[t], 128);
+      mbar_init(&bar_p[t], 4);  // one arrival per softmax warp of the tile
       mbar_init(&bar_o[t], 1);
     }
     fence_mbar_init();
@@ -134,17 +251,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tbase = tmem_slot;
   DevStatus* st = &g_fa_status;
 
-  if (warp == C::TMA_WARP) {
-    // ------------------------------------------------------------ producer --
-    if (lane == 0) {
+  if (warp >= C::SOFTMAX_WARPS) {
+    // Last warpgroup: MMA issuer, TMA producer, two idle warps. It gives
+    // registers back so the softmax warpgroups can take them.
+    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_OTHER));
+    if (warp == C::TMA_WARP && lane == 0) {
+      // ---------------------------------------------------------- producer --
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bar_q, NQ * C::Q_TILE);
       for (int t = 0; t < NQ; ++t)
         for (int c = 0; c < C::QK_CHUNKS; ++c)
-          tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK),
-                      q0 + t * C::BM, bh);
+          tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK), q0 + t * C::BM,
+                      bh);
       int pos = 0;
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -169,10 +289,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_drain(&bar_q, 0);
       for (int q = pos - C::NSLOT; q < pos; ++q)
         if (q >= 0) mbar_drain(&bar_full[q % C::NSLOT], (q / C::NSLOT) & 1);
-    }
-  } else if (warp == C::MMA_WARP) {
-    // ---------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    } else if (warp == C::MMA_WARP && lane == 0) {
+      // -------------------------------------------------------- MMA issuer --
       constexpr uint32_t idesc_qk = idesc_make(QK_FP8 ? 0u : 1u, 128, C::BN, false);
       constexpr uint32_t idesc_pv = idesc_make(1u, 128, D, true);
       const uint32_t ring = smem_u32(sRing);
@@ -187,7 +305,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
         for (int t = 0; t < NQ && ok; ++t) {
           if (j > 0) {
-            ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23);
+            // The single issuer polls: its wake-up is on the critical path.
+            ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, false);
             if (!ok) break;
             tc_fence_after();
             // O_t += P_t V_{j-1}: A = P_t from TMEM (bf16 pairs), B = V tile (MN-major).
@@ -195,7 +314,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int kk = 0; kk < C::BN / 16; ++kk) {
               const uint64_t bdesc = sdesc_sw128(vaddr + kk * 16 * 128, C::BN * 128, 1024);
-              mma_bf16_ts(tbase + C::O_COL(t), tbase + C::S_COL(t) + kk * 8, bdesc, idesc_pv,
+              mma_bf16_ts(tbase + C::O_COL(t), tbase + C::P_COL(t) + kk * 8, bdesc, idesc_pv,
                           (j > 1 || kk > 0) ? 1u : 0u);
             }
             if (j == n_kv) mma_commit(&bar_o[t]);
@@ -226,13 +345,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_drain(&bar_drain, 0);
     }
   } else {
-    // ------------------------------------------------------------- softmax --
+    // ----------------------------------------------------------- softmax --
+    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
     const int t = static_cast<int>(warp >> 2);
     const uint32_t lane_base = (warp & 3u) * 32u;
-    const int r = static_cast<int>(lane_base + lane);
+    const int r = static_cast<int>(lane_base + lane);  // row within the tile = TMEM lane
     const int qrow = q0 + t * C::BM + r;
-    const uint32_t tS = tbase + (lane_base << 16) + C::S_COL(t);
-    const uint32_t tO = tbase + (lane_base << 16) + C::O_COL(t);
+    const uint32_t row_addr = tbase + (lane_base << 16);
+    const uint32_t tS = row_addr + C::S_COL(t);
+    const uint32_t tP = row_addr + C::P_COL(t);
+    const uint32_t tO = row_addr + C::O_COL(t);
     float s_log2 = p.scale_log2;
     if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
     const int kmax = CAUSAL ? min(qrow, p.N - 1) : p.N - 1;  // last visible key of this row
@@ -244,76 +366,51 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
       if (!ok) break;
       tc_fence_after();
-      uint32_t s[128];
-      tmem_ld32(tS + 0, &s[0]);
-      tmem_ld32(tS + 32, &s[32]);
-      tmem_ld32(tS + 64, &s[64]);
-      tmem_ld32(tS + 96, &s[96]);
-      tmem_wait_ld();
+      uint32_t s[128], pk[64];
       const int kbase = j * C::BN;
-      if (kbase + C::BN - 1 > kmax) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kbase + c > kmax) s[c] = __float_as_uint(-INFINITY);
-      }
-      // Row max: four independent chains of 3-input max.
-      float a0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
-      float a1 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
-      float a2 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
-      float a3 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
-#pragma unroll
-      for (int c = 8; c < 128; c += 8) {
-        a0 = fmax3(a0, __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
-        a1 = fmax3(a1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-        a2 = fmax3(a2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-        a3 = fmax3(a3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-      }
-      const float mx_s = fmax3(a0, a1, fmaxf(a2, a3)) * s_log2;
-      const bool grow = mx_s > m_ref + 8.0f;
-      const float m_new = grow ? mx_s : m_ref;
-      const float alpha = ex2_approx(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
-      m_ref = m_new;
-      // p = 2^(x*s - m): one packed FMA per pair, then the SFU exp2; P packs to bf16.
-      const uint64_t s2 = f2_pack(s_log2, s_log2);
-      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
-      uint64_t acc_e[2] = {0ull, 0ull}, acc_r[2] = {0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        float t0, t1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), s2, nm2), t0, t1);
-        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-        const uint32_t pk = pack_bf16x2(p0, p1);
-        const int a = (c >> 1) & 1;
-        acc_e[a] = f2_add(acc_e[a], f2_pack(p0, p1));
-        acc_r[a] = f2_add(acc_r[a], f2_pack(__uint_as_float(pk << 16), __uint_as_float(pk & 0xFFFF0000u)));
-        s[c >> 1] = pk;
-      }
-      tmem_st32(tS + 0, &s[0]);
-      tmem_st32(tS + 32, &s[32]);
-      float e0, e1, e2, e3, r0, r1, r2, r3;
-      f2_unpack(acc_e[0], e0, e1);
-      f2_unpack(acc_e[1], e2, e3);
-      f2_unpack(acc_r[0], r0, r1);
-      f2_unpack(acc_r[1], r2, r3);
-      l_exact = l_exact * alpha + ((e0 + e1) + (e2 + e3));
-      l_round = l_round * alpha + ((r0 + r1) + (r2 + r3));
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
-        // completed: the commit that signalled S_t for tile j also covers it, and
-        // PV of tile j is issued only after this warpgroup arrives below.
+      // Some key of this tile is not visible to some row of this warp. Warp-uniform:
+      // it selects code paths that issue tcgen05.ld, which all 32 lanes must
+      // execute together (a lane-divergent .sync.aligned instruction deadlocks).
+      const bool masked = __any_sync(0xffffffffu, kbase + C::BN - 1 > kmax);
+      float sum_e, sum_r, alpha = 1.0f, mx = 0.f;
+      if (j == 0) {
+        m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;  // finite: key 0 is visible
+        softmax_row_dispatch<false>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+      } else {
+        // Exponentials against the current reference, taking the row's max on the
+        // way; only if some row's max grew by more than 2^8 (rare after the first
+        // tiles) is the row redone against the new reference. S is still intact:
+        // P is written only below.
+        softmax_row_dispatch<true>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        const float mx_s = mx * s_log2;
+        const bool grow = mx_s > m_ref + 8.0f;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float m_new = grow ? mx_s : m_ref;
+          alpha = ex2_approx(m_ref - m_new);  // 1 for rows that did not grow
+          m_ref = m_new;
+          softmax_row_dispatch<false>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+          // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
+          // completed (the commit that signalled S_t for tile j also covers it),
+          // and PV of tile j is issued only after this warpgroup arrives below.
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO + c0, ov);
-          tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c0, ov);
+            tmem_wait_ld_dep32(ov);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tO + c0, ov);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tO + c0, ov);
+          }
         }
       }
+      tmem_st32(tP + 0, &pk[0]);
+      tmem_st32(tP + 32, &pk[32]);
+      l_exact = l_exact * alpha + sum_e;
+      l_round = l_round * alpha + sum_r;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_p[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p[t]);  // one arrival per warp
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
     if (ok) {
@@ -325,15 +422,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
         tmem_ld32(tO + c0, ov);
-        tmem_wait_ld();
-        uint32_t pk[16];
+        tmem_wait_ld_dep32(ov);
+        uint32_t q[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+          q[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
         if (in_range) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
         }
       }
       if (in_range && p.lse != nullptr)

@@ -45,6 +45,19 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8>;
   static unsigned long long smem_done = 0;
   if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
+  if constexpr (C::SPLIT_REGS) {
+    // The kernel moves registers between warpgroups with setmaxnreg; that only
+    // completes if the block was launched with the register count the split was
+    // sized for. Refuse to launch otherwise (an .inc that can never be satisfied
+    // would wait forever).
+    static int checked = 0;  // 0 = not yet, 1 = ok, 2 = bad
+    if (checked == 0) {
+      cudaFuncAttributes fa_attr;
+      if (cudaFuncGetAttributes(&fa_attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+      checked = fa_attr.numRegs >= C::REG_LAUNCH ? 1 : 2;
+    }
+    if (checked != 1) return FA_ERR_UNSUPPORTED;
+  }
   FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;

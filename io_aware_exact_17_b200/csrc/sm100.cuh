@@ -66,25 +66,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps
+// in hardware (issuing nothing) until the phase completes or hint_ns pass, so
+// waiting warps leave the issue slots to the warps sharing their SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete. Returns false if
 // the CTA is already aborting or the wait ran past kWaitLimitNs; in the latter
 // case the first such event in the grid is recorded in *st.
+// With `sleep` false the thread polls (lowest wake-up latency, for the single
+// MMA-issuing thread on the critical path); otherwise it sleeps between polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          DevStatus* st, uint32_t site) {
+                                          DevStatus* st, uint32_t site, bool sleep = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        if (st != nullptr && atomicCAS(&st->code, 0u, 5u /*FA_ERR_TIMEOUT*/) == 0u) {
-          st->site = site;
-          st->block = blockIdx.x;
-        }
-        return false;
+  for (;;) {
+    if (sleep ? mbar_try_wait_sleep(bar, parity, 20000u) : mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      if (st != nullptr && atomicCAS(&st->code, 0u, 5u /*FA_ERR_TIMEOUT*/) == 0u) {
+        st->site = site;
+        st->block = blockIdx.x;
       }
+      return false;
     }
   }
 }
@@ -122,6 +137,18 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for prior tcgen05.ld and tie 32 destination registers to the wait, so the
+// compiler cannot move their first use above it (the loads write them asynchronously).
+__device__ __forceinline__ void tmem_wait_ld_dep32(uint32_t* r) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // TMEM address: lane in bits [31:16], column in bits [15:0]. A warp may touch
@@ -249,6 +276,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// bf16 round-to-nearest-even of two non-negative finite floats on the integer
+// pipe (no conversion instruction): returns the packed pair and, in r0/r1, the
+// rounded values as fp32 bit patterns.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi, uint32_t& r0, uint32_t& r1) {
+  const uint32_t u0 = __float_as_uint(lo), u1 = __float_as_uint(hi);
+  r0 = (u0 + 0x7FFFu + ((u0 >> 16) & 1u)) & 0xFFFF0000u;
+  r1 = (u1 + 0x7FFFu + ((u1 >> 16) & 1u)) & 0xFFFF0000u;
+  return __byte_perm(r0, r1, 0x7632);
+}
 // Two floats -> two e4m3 codes (round-to-nearest-even, saturating to +-448), lo in bits [7:0].
 __device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
   uint16_t r;
@@ -279,6 +315,32 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x on the FMA pipe, for two lanes at once: x = n + f with n = round(x) and
+// |f| <= 1/2 (Cody-Waite split via the 1.5*2^23 rounding constant), 2^f from a
+// degree-3 polynomial fitted for minimax relative error on [-1/2, 1/2]
+// (max relative error 7.5e-5 after fp32 evaluation), and 2^n added to the
+// exponent field. x is clamped below at -126, so the result is never zero:
+// callers use it only where no key is masked.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f, c2 = 0.24261054396629333f,
+                  c3 = 0.05517132207751274f;
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));            // low bits hold round(x)
+  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));          // round(x) as float
+  const uint64_t f = f2_add(x, n ^ 0x8000000080000000ull);          // x - round(x)
+  uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
+  p = f2_fma(p, f, f2_pack(c1, c1));
+  p = f2_fma(p, f, f2_pack(c0, c0));
+  float t0, t1, p0, p1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(p, p0, p1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
