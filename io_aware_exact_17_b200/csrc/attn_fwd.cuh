@@ -106,6 +106,14 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 #endif
 constexpr int kPolyEvery = FA_EXP_POLY_EVERY;  // 1 pair in kPolyEvery uses the polynomial (0: none)
 
+#ifndef FA_MMA_WAIT_SLEEP_NS
+#define FA_MMA_WAIT_SLEEP_NS 0
+#endif
+// Suspend hint of the MMA issuer's wait for P (0: poll). Its wake-up latency is
+// on the critical path, but a polling warp also takes issue slots from the two
+// softmax warps on its sub-partition.
+constexpr uint32_t kMmaWaitSleepNs = FA_MMA_WAIT_SLEEP_NS;
+
 // Exponentials of one 32-key chunk of a row of S: p = 2^(x*s - m), packed to
 // bf16 pairs into pk[0..15]; accumulates the fp32 weights and the rounded ones
 // into the packed-pair sums and (WITH_MAX) the raw-score max into mx[0..3].
@@ -306,7 +314,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int t = 0; t < NQ && ok; ++t) {
           if (j > 0) {
             // The single issuer polls: its wake-up is on the critical path.
-            ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, false);
+            ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, kMmaWaitSleepNs);
             if (!ok) break;
             tc_fence_after();
             // O_t += P_t V_{j-1}: A = P_t from TMEM (bf16 pairs), B = V tile (MN-major).

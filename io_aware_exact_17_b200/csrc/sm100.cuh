@@ -84,14 +84,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // Wait for the phase of `bar` with the given parity to complete. Returns false if
 // the CTA is already aborting or the wait ran past kWaitLimitNs; in the latter
 // case the first such event in the grid is recorded in *st.
-// With `sleep` false the thread polls (lowest wake-up latency, for the single
-// MMA-issuing thread on the critical path); otherwise it sleeps between polls.
+// `sleep_ns` is the suspend-time hint of each poll: 0 polls without sleeping
+// (lowest wake-up latency), larger values leave more issue slots to the warps
+// sharing the sub-partition.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          DevStatus* st, uint32_t site, bool sleep = true) {
+                                          DevStatus* st, uint32_t site, uint32_t sleep_ns = 20000u) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
-    if (sleep ? mbar_try_wait_sleep(bar, parity, 20000u) : mbar_try_wait(bar, parity)) return true;
+    if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
