@@ -96,6 +96,35 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_t rows, int d, int rotate,
                             const float* signs, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_hadamard_quant_noalloc — fa_hadamard_quant for callers that cannot allocate
+ * device memory, for up to 64 tensors of one shape (e.g. Q and K) per call.
+ *
+ * No counterpart in the pages: this is a service entry point of this library.
+ * Some callers cannot call cudaMalloc or hand over a workspace: code that owns
+ * no device allocator (a plugin inside an application that manages all device
+ * memory itself), or code that must not trigger the implicit device-wide
+ * synchronisation an allocation can cause. This entry point needs no workspace:
+ * the scratch (one 4-byte amax word per tensor) is a 256-byte array inside the
+ * library, allocated when the library is loaded and held by every device that
+ * loads it until the process exits. Results are identical to calling
+ * fa_hadamard_quant once per tensor.
+ *
+ * xs, outs   host arrays of `ntensors` device pointers: bf16 inputs [rows][d] and
+ *            e4m3 outputs [rows][d], each 16-byte aligned (may be NULL if rows = 0).
+ * descales   device, ntensors fp32 (descale of tensor i at descales[i]).
+ * ntensors   1..64; more is rejected with FA_ERR_INVALID_ARG (the array holds 64 words).
+ * rows, d, rotate, signs: as for fa_hadamard_quant, shared by all tensors.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up per device, with that device current); make that first call before any
+ * stream capture. Every call zeroes and reuses the same array, so calls that
+ * overlap on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_hadamard_quant_noalloc(const void* const* xs, void* const* outs, float* descales, int ntensors,
+                                    int64_t rows, int d, int rotate, const float* signs, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fa_status_string(fa_status s);
 

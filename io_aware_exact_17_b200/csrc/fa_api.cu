@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/fa.h"
 #include "attn_fwd.cuh"
@@ -159,6 +160,77 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
     case 128: return launch_quant<128>(x, out, descale_out, rows, rotate, sg, amax, s);
     default: return launch_quant<256>(x, out, descale_out, rows, rotate, sg, amax, s);
   }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free quantisation (fa_hadamard_quant_noalloc).
+//
+// The scratch of the quantiser (one amax word per tensor) lives in this
+// file-scope device array instead of a caller workspace. Every device that
+// loads the library holds it until the process exits. In host code the name
+// g_noalloc_scratch is only a host-side stand-in, never a device address: the
+// kernels get the address cudaGetSymbolAddress returns, looked up once per
+// device with that device current.
+namespace {
+
+constexpr int kNoallocScratchBytes = 256;
+constexpr int kNoallocMaxTensors = kNoallocScratchBytes / static_cast<int>(sizeof(unsigned int));  // 64
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoallocMaxTensors];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned int* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on first use).
+fa_status noalloc_scratch(unsigned int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_hadamard_quant_noalloc(const void* const* xs, void* const* outs, float* descales, int ntensors,
+                                    int64_t rows, int d, int rotate, const float* signs, void* stream) {
+  if (xs == nullptr || outs == nullptr || descales == nullptr) return FA_ERR_INVALID_ARG;
+  if (ntensors < 1 || ntensors > kNoallocMaxTensors) return FA_ERR_INVALID_ARG;  // scratch holds 64 words
+  if (rows < 0 || rows > (static_cast<int64_t>(1) << 40) || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned(descales, 4)) return FA_ERR_ALIGNMENT;
+  if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
+  for (int i = 0; i < ntensors; ++i) {
+    if (rows > 0 && (xs[i] == nullptr || outs[i] == nullptr)) return FA_ERR_INVALID_ARG;
+    if (!aligned(xs[i], 16) || !aligned(outs[i], 16)) return FA_ERR_ALIGNMENT;
+  }
+  unsigned int* scratch = nullptr;
+  const fa_status sst = noalloc_scratch(&scratch);
+  if (sst != FA_OK) return sst;
+  const float* sg = rotate ? signs : nullptr;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < ntensors; ++i) {
+    // Word i of the array is tensor i's amax; launch_quant zeroes it first on
+    // this stream, so what an earlier call left there does not matter.
+    fa_status r;
+    switch (d) {
+      case 64: r = launch_quant<64>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
+      case 128: r = launch_quant<128>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
+      default: r = launch_quant<256>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
+    }
+    if (r != FA_OK) return r;
+  }
+  return FA_OK;
 }
 
 const char* fa_status_string(fa_status st) {
