@@ -42,6 +42,29 @@ SEED = 1001
 WORKLOAD = f"b{B}h{H}n{N}d{D}: bf16 fwd non-causal + bf16 fwd causal + rotate/quantise Q,K + e4m3-QK fwd non-causal"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# bf16 non-causal attention kernel on this workload, from one ncu capture, and
+# the SHA-256 of the kernel's sources at that capture. When the sources differ
+# the figure no longer describes the kernel and `traffic` is reported as null.
+KERNEL_SOURCES = ("io_aware_exact_17_b200/csrc/attn_fwd.cuh", "io_aware_exact_17_b200/csrc/sm100.cuh")
+NCU_TRAFFIC_BYTES = None
+NCU_TRAFFIC_SHA256 = None
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    if NCU_TRAFFIC_BYTES is None or NCU_TRAFFIC_SHA256 != kernel_sources_sha256():
+        return None
+    return NCU_TRAFFIC_BYTES
+
 
 def flops_fwd(causal: bool) -> float:
     f = 4.0 * B * H * N * N * D
@@ -184,7 +207,7 @@ class Step:
         self.o_h = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
         self.lse_h = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(3)]
         self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-        self.launches_per_step = 7  # 3 attention kernels + 2 x (amax, quantise)
+        self.launches_per_step = 5  # 3 attention kernels + 2 one-launch quantisations
 
     def flush_l2(self):
         self.flush_buf.zero_()
@@ -228,21 +251,47 @@ class Step:
         return sum(t.numel() * t.element_size() for t in self.o_h + self.lse_h)
 
 
-def time_steps(step: Step, steps: int, warmup: int, world: int):
+def capture_step(step: Step):
+    """The step's kernels captured once as a CUDA graph, so a timed step carries
+    no host launch overhead (the quantiser kernels are ~10 us each)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        step.run()  # every lazy set-up (attributes, occupancy) done before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            step.run()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_steps(step: Step, graph, steps: int, warmup: int, world: int):
+    """K timed steps (graph replays, L2 flushed between them outside the events),
+    then K eager steps with events around each kernel group for the breakdown."""
     for _ in range(warmup):
         step.flush_l2()
-        step.run()
+        graph.replay()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     dist_barrier(world)
     torch.cuda.synchronize()
     for i in range(steps):
         step.flush_l2()
-        step.run(evs[i])
+        ev[i][0].record()
+        graph.replay()
+        ev[i][1].record()
     torch.cuda.synchronize()
     dist_barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        step.flush_l2()
+        step.run(evs[i])
+    torch.cuda.synchronize()
     per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)]
-    return per  # ms: [bf16 nc, bf16 causal, quant Q+K, fp8 nc] per step
+    return step_ms, per  # per: ms [bf16 nc, bf16 causal, quant Q+K, fp8 nc] per eager step
 
 
 def time_e2e(step: Step, steps: int, warmup: int, world: int):
@@ -333,10 +382,10 @@ def main():
         raise SystemExit("bench.py needs a CUDA device for --impl ours")
     torch.cuda.set_device(local)
     step = Step(SEED + rank)
+    graph = capture_step(step)
     with ClockSampler(local) as clk:
-        per = time_steps(step, args.steps, args.warmup, world)
+        step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
     e2e_ms = time_e2e(step, max(3, args.steps // 4), 3, world)
-    step_ms = [sum(p) for p in per]
     ms_local = statistics.mean(step_ms)
     ms = dist_max(ms_local, world)
     e2e_ms = dist_max(e2e_ms, world)
@@ -355,6 +404,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
             "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (512 MB write outside the timed events)"},
+            "timing": "value: CUDA-graph replay of the step; breakdown: eager calls, events per kernel group",
             "breakdown_ms": {"bf16_noncausal": comp[0], "bf16_causal": comp[1], "rotate_quant_qk": comp[2],
                              "e4m3qk_noncausal": comp[3]},
             "breakdown_tflops": {"bf16_noncausal": flops_fwd(False) / comp[0] / 1e9,
@@ -362,7 +412,8 @@ def main():
                                  "e4m3qk_noncausal": flops_fwd(False) / comp[3] / 1e9},
             "roofline": {"kernel": "attn_fwd_kernel<128,2,nc,bf16>", "bound": "tensor", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": measured_traffic(),
+                         "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "peak_source": f"{peak_src} cuBLAS bf16 (burst)"},
             "e2e": {"value": world * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                     "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},

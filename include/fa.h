@@ -65,7 +65,7 @@ typedef enum {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
                  int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, void* stream);
 
-/* Bytes of device workspace fa_hadamard_quant needs (a 4-byte amax word, padded). */
+/* Bytes of device workspace fa_hadamard_quant needs (the amax word and a grid-barrier counter, padded). */
 #define FA_QUANT_WORKSPACE_BYTES 256
 
 /*

@@ -36,8 +36,6 @@
 
 namespace fa {
 
-__device__ DevStatus g_fa_status;  // first device-side error of any launch
-
 #ifndef FA_REG_SOFTMAX
 #define FA_REG_SOFTMAX 208
 #endif
@@ -150,10 +148,12 @@ __device__ __forceinline__ void mask_chunk32(uint32_t* s, int kbase, int kmax) {
 // One row of S (128 keys, from TMEM at tS) through the exponentials: the four
 // 32-column loads are software-pipelined with the exps of the previous chunk
 // (tcgen05.wait::ld waits for all earlier loads, so chunk c+1 is issued before
-// chunk c is computed). P is packed into pk[0..63]. Returns the fp32 and rounded
+// chunk c is computed). P is packed in place: chunk c's 16 bf16 pairs go to
+// s[16c .. 16c+15], scores already consumed (chunk c/2's) and never the target of
+// a pending load, so only 128 registers are live. Returns the fp32 and rounded
 // weight sums and, with WITH_MAX, the max of the raw scores.
 template <bool EMU, bool WITH_MAX>
-__device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, uint32_t* pk, float s_log2, float m_ref,
+__device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
                                             int kbase, int kmax, bool masked, float& sum_e, float& sum_r,
                                             float& raw_max) {
   const uint64_t s2 = f2_pack(s_log2, s_log2);
@@ -166,7 +166,7 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, uint32_t* 
   for (int ch = 0; ch < 4; ++ch) {
     if (ch < 3) tmem_ld32(tS + 32 * (ch + 1), &s[32 * (ch + 1)]);
     if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
-    exp_chunk32<EMU, WITH_MAX>(&s[32 * ch], &pk[16 * ch], s2, nm2, acc_e, acc_r, mx);
+    exp_chunk32<EMU, WITH_MAX>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
     if (ch < 3) tmem_wait_ld_dep32(&s[32 * (ch + 1)]);
   }
   float e0, e1, e2, e3, r0, r1, r2, r3;
@@ -181,13 +181,13 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, uint32_t* 
 
 // `masked` must be warp-uniform: both paths issue tcgen05.ld.
 template <bool WITH_MAX>
-__device__ __forceinline__ void softmax_row_dispatch(uint32_t tS, uint32_t* s, uint32_t* pk, float s_log2,
-                                                     float m_ref, int kbase, int kmax, bool masked, float& se,
-                                                     float& sr, float& mx) {
+__device__ __forceinline__ void softmax_row_dispatch(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
+                                                     int kbase, int kmax, bool masked, float& se, float& sr,
+                                                     float& mx) {
   if (masked)
-    softmax_row<false, WITH_MAX>(tS, s, pk, s_log2, m_ref, kbase, kmax, true, se, sr, mx);
+    softmax_row<false, WITH_MAX>(tS, s, s_log2, m_ref, kbase, kmax, true, se, sr, mx);
   else
-    softmax_row<true, WITH_MAX>(tS, s, pk, s_log2, m_ref, kbase, kmax, false, se, sr, mx);
+    softmax_row<true, WITH_MAX>(tS, s, s_log2, m_ref, kbase, kmax, false, se, sr, mx);
 }
 
 // Raw-score max of one row of S (first tile only, before any reference exists).
@@ -374,7 +374,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
       if (!ok) break;
       tc_fence_after();
-      uint32_t s[128], pk[64];
+      uint32_t s[128];
       const int kbase = j * C::BN;
       // Some key of this tile is not visible to some row of this warp. Warp-uniform:
       // it selects code paths that issue tcgen05.ld, which all 32 lanes must
@@ -383,20 +383,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float sum_e, sum_r, alpha = 1.0f, mx = 0.f;
       if (j == 0) {
         m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;  // finite: key 0 is visible
-        softmax_row_dispatch<false>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
       } else {
         // Exponentials against the current reference, taking the row's max on the
         // way; only if some row's max grew by more than 2^8 (rare after the first
         // tiles) is the row redone against the new reference. S is still intact:
         // P is written only below.
-        softmax_row_dispatch<true>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        softmax_row_dispatch<true>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
         const float mx_s = mx * s_log2;
         const bool grow = mx_s > m_ref + 8.0f;
         if (__any_sync(0xffffffffu, grow)) {
           const float m_new = grow ? mx_s : m_ref;
           alpha = ex2_approx(m_ref - m_new);  // 1 for rows that did not grow
           m_ref = m_new;
-          softmax_row_dispatch<false>(tS, s, pk, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+          softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
           // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
           // completed (the commit that signalled S_t for tile j also covers it),
           // and PV of tile j is issued only after this warpgroup arrives below.
@@ -411,8 +411,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      tmem_st32(tP + 0, &pk[0]);
-      tmem_st32(tP + 32, &pk[32]);
+      tmem_st32(tP + 0, &s[0]);
+      tmem_st32(tP + 32, &s[32]);
       l_exact = l_exact * alpha + sum_e;
       l_round = l_round * alpha + sum_r;
       tmem_wait_st();

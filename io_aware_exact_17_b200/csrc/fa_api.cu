@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -99,6 +100,42 @@ fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t row
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Both quantisation passes in one cooperative launch (quant_fused_kernel): the
+// workspace holds the amax word and the grid barrier's counter, zeroed here.
+template <int D>
+fa_status launch_quant_fused(const void* x, void* out, float* descale_out, int64_t rows, int rotate,
+                             const float* signs, unsigned int* ws, cudaStream_t stream) {
+  using FC = fa::FusedCfg<D>;
+  if (cudaMemsetAsync(ws, 0, 2 * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  auto kernel = rotate ? fa::quant_fused_kernel<D, true> : fa::quant_fused_kernel<D, false>;
+  // Co-resident blocks per SM and SM count, looked up once per device (this is
+  // host time in front of a ~10 us kernel).
+  static int cached_per_sm[2][64] = {};
+  static int cached_sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
+  int& per_sm = cached_per_sm[rotate ? 1 : 0][dev];
+  int& sms = cached_sms[dev];
+  if (sms == 0 && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (per_sm == 0 &&
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, fa::kFusedThreads, 0) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (per_sm < 1 || sms < 1) return FA_ERR_CUDA;
+  const int64_t steps = (rows + FC::RPW - 1) / FC::RPW;  // warp-steps of work
+  int64_t blocks = (steps + fa::kFusedThreads / 32 - 1) / (fa::kFusedThreads / 32);
+  const int64_t cap = static_cast<int64_t>(per_sm) * sms;  // all blocks co-resident
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  uint8_t* ob = static_cast<uint8_t*>(out);
+  void* args[] = {&xb, &ob, &rows, &signs, &ws, &descale_out};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(static_cast<unsigned>(blocks)),
+                                  dim3(fa::kFusedThreads), args, 0, stream) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -118,7 +155,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (descale_qk == nullptr) return FA_ERR_INVALID_ARG;
     if (!aligned(descale_qk, 4)) return FA_ERR_ALIGNMENT;
   }
-  const int rows_per_cta = d == 256 ? 128 : 256;
+  const int rows_per_cta = 128;  // the smallest query block of any kernel
   const long long n_qb = (static_cast<long long>(N) + rows_per_cta - 1) / rows_per_cta;
   if (n_qb * B * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -156,9 +193,9 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
   unsigned int* amax = static_cast<unsigned int*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_quant<64>(x, out, descale_out, rows, rotate, sg, amax, s);
-    case 128: return launch_quant<128>(x, out, descale_out, rows, rotate, sg, amax, s);
-    default: return launch_quant<256>(x, out, descale_out, rows, rotate, sg, amax, s);
+    case 64: return launch_quant_fused<64>(x, out, descale_out, rows, rotate, sg, amax, s);
+    case 128: return launch_quant_fused<128>(x, out, descale_out, rows, rotate, sg, amax, s);
+    default: return launch_quant_fused<256>(x, out, descale_out, rows, rotate, sg, amax, s);
   }
 }
 

@@ -12,9 +12,11 @@
 //
 // Two streaming passes over the bf16 input, both HBM/L2-bound:
 //   pass 1: rotate, reduce |x'| to one block max, atomicMax into a scratch word;
-//   pass 2: rotate again, scale, convert, store 8 codes (8 bytes) per thread.
+//   pass 2: rotate again, scale, convert, store the codes.
 // A tensor of up to ~60 MB stays in the 126 MB L2 between the passes, so the
-// second read mostly hits L2.
+// second read mostly hits L2. quant_fused_kernel runs both passes in one
+// cooperative launch; quant_amax_kernel + quant_apply_kernel are the two-launch
+// form (used where the scratch is the library's own static array).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -159,6 +161,193 @@ quant_apply_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
       uint32_t hi = static_cast<uint32_t>(pack_e4m3x2(v[u][4] * scale, v[u][5] * scale)) |
                     (static_cast<uint32_t>(pack_e4m3x2(v[u][6] * scale, v[u][7] * scale)) << 16);
       if (row < rows) *reinterpret_cast<uint2*>(out + row * D + 8 * lr) = make_uint2(lo, hi);
+    }
+  }
+}
+
+}  // namespace fa
+
+namespace fa {
+
+// ---------------------------------------------------------------------------
+// One-launch variant: both passes in one cooperative kernel with a grid-wide
+// barrier between them (all blocks are co-resident, which the cooperative
+// launch guarantees), 32 elements per thread (fewer cross-lane butterfly
+// stages), and the second pass re-reading the tensor while it is still in L2.
+// The butterfly stages run in the same order (index bits 0, 1, 2, ...) with
+// the same operands as hadamard_rotate, so the codes are bit-identical to the
+// two-kernel path.
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = 256;
+
+template <int D>
+struct FusedCfg {
+  static constexpr int E = 32;          // elements per thread (four 16-byte chunks)
+  static constexpr int L = D / E;       // threads per row
+  static constexpr int RPW = 32 / L;    // rows per warp per step
+  static_assert(D == 64 || D == 128 || D == 256, "head dim");
+};
+
+// Thread lr of a row holds the four 16-byte chunks lr, lr+L, lr+2L, lr+3L (8
+// elements each) of the row: v[8*q + i] is element 8*(lr + L*q) + i. A warp's
+// load instruction q then covers L consecutive chunks of each of its rows.
+template <int D>
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* row, int lr, float (&v)[32]) {
+  constexpr int L = D / 32;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + lr + L * q);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// In place: (v * signs) H_D / sqrt(D) for the elements this thread holds (the
+// layout of load_bf16x32). Butterflies run over index bits 0, 1, 2 (inside a
+// chunk), then the log2(L) bits of the chunk's lane (warp shuffles), then the two
+// bits of q (inside the thread): the same stage order as hadamard_rotate.
+// Every lane of the warp must call.
+template <int D>
+__device__ __forceinline__ void hadamard_rotate32(float (&v)[32], int lr, const float* signs) {
+  constexpr int L = D / 32;
+  if (signs != nullptr) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q)));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q) + 4));
+      v[8 * q + 0] *= s0.x; v[8 * q + 1] *= s0.y; v[8 * q + 2] *= s0.z; v[8 * q + 3] *= s0.w;
+      v[8 * q + 4] *= s1.x; v[8 * q + 5] *= s1.y; v[8 * q + 6] *= s1.z; v[8 * q + 7] *= s1.w;
+    }
+  }
+  // index bits 0..2
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+  // index bits 3 .. 2+log2(L): across the L lanes of the row
+#pragma unroll
+  for (int m = 1; m < L; m <<= 1) {
+    // lower lane: v + other; upper lane: other - v; both as one fma with +-1
+    // (exact: the same single rounding as the add or subtract).
+    const float sgn = (lr & m) != 0 ? -1.0f : 1.0f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[e], m);
+      v[e] = fmaf(v[e], sgn, other);
+    }
+  }
+  // the two bits of q
+#pragma unroll
+  for (int h = 8; h < 32; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+  constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] *= inv_sqrt_d;
+}
+
+// ws[0]: amax bits, ws[1]: arrival counter of the grid barrier; both zero at launch.
+template <int D, bool ROT>
+__global__ void __launch_bounds__(kFusedThreads)
+quant_fused_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ out, int64_t rows,
+                   const float* __restrict__ signs, unsigned int* ws, float* descale_out) {
+  DevStatus* st = &g_fa_status;
+  using C = FusedCfg<D>;
+  const int lane = threadIdx.x & 31;
+  const int lr = lane % C::L, sub = lane / C::L;
+  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * kFusedThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kFusedThreads) >> 5;
+  // pass 1: amax of the rotated tensor
+  float m = 0.f;
+  for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
+    const int64_t row = w * C::RPW + sub;
+    float v[32];
+    if (row < rows) {
+      load_bf16x32<D>(x + row * D, lr, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    }
+    if (ROT) hadamard_rotate32<D>(v, lr, signs);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(v[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float warp_max[kFusedThreads / 32];
+  __shared__ unsigned int amax_sh;
+  if (lane == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = warp_max[0];
+#pragma unroll
+    for (int i = 1; i < kFusedThreads / 32; ++i) b = fmaxf(b, warp_max[i]);
+    atomicMax(&ws[0], __float_as_uint(b));
+    // Grid-wide barrier: every block is resident (cooperative launch). The wait
+    // is bounded; if it runs out the status word records it and the block goes on.
+    __threadfence();
+    atomicAdd(&ws[1], 1u);
+    const unsigned long long t0 = globaltimer_ns();
+    unsigned int arrived;
+    for (;;) {
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + 1) : "memory");
+      if (arrived >= gridDim.x) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (atomicCAS(&st->code, 0u, 5u) == 0u) {
+          st->site = 60;
+          st->block = blockIdx.x;
+        }
+        break;
+      }
+      __nanosleep(64);
+    }
+    unsigned int a;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(ws) : "memory");
+    amax_sh = a;
+  }
+  __syncthreads();
+  // pass 2: quantise (the tensor is re-read, mostly from L2)
+  const float amax = __uint_as_float(amax_sh);
+  const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *descale_out = amax > 0.f ? amax / 448.0f : 1.0f;
+  for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
+    const int64_t row = w * C::RPW + sub;
+    float v[32];
+    if (row < rows) {
+      load_bf16x32<D>(x + row * D, lr, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    }
+    if (ROT) hadamard_rotate32<D>(v, lr, signs);
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      q[i] = static_cast<uint32_t>(pack_e4m3x2(v[4 * i] * scale, v[4 * i + 1] * scale)) |
+             (static_cast<uint32_t>(pack_e4m3x2(v[4 * i + 2] * scale, v[4 * i + 3] * scale)) << 16);
+    if (row < rows) {
+      // chunk c of the row (8 codes, 8 bytes) goes to out[row*D + 8c]
+      uint2* dst = reinterpret_cast<uint2*>(out + row * D);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
     }
   }
 }

@@ -26,6 +26,8 @@ struct DevStatus {
   unsigned int pad;
 };
 
+__device__ DevStatus g_fa_status;  // first device-side error of any launch of this library
+
 // 1 s: no legitimate wait inside one CTA comes near this (the longest kernels
 // run for milliseconds), so hitting it means a lost arrival, not slowness.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
