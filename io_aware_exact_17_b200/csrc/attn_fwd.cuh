@@ -231,8 +231,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   int qb = blockIdx.x % p.n_qb;
   if (CAUSAL) qb = p.n_qb - 1 - qb;
   const int q0 = qb * NQ * C::BM;
-  const int kv_end = CAUSAL ? min(p.N, q0 + NQ * C::BM) : p.N;
-  const int n_kv = (kv_end + C::BN - 1) / C::BN;
+  // KV tiles a query tile needs: all of them, or (causal) up to its last row.
+  // The CTA streams n_kv = the last tile's count; an earlier causal tile stops sooner
+  // (n_kv_t), so it never spends a step on a key tile that is entirely in its future.
+  auto n_kv_of = [&](int t) {
+    const int end = CAUSAL ? min(p.N, q0 + (t + 1) * C::BM) : p.N;
+    return (end + C::BN - 1) / C::BN;
+  };
+  const int n_kv = n_kv_of(NQ - 1);
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -312,7 +318,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < NQ && ok; ++t) {
-          if (j > 0) {
+          const int n_kv_t = n_kv_of(t);
+          if (j > 0 && j - 1 < n_kv_t) {
             // The single issuer polls: its wake-up is on the critical path.
             ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, kMmaWaitSleepNs);
             if (!ok) break;
@@ -325,9 +332,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               mma_bf16_ts(tbase + C::O_COL(t), tbase + C::P_COL(t) + kk * 8, bdesc, idesc_pv,
                           (j > 1 || kk > 0) ? 1u : 0u);
             }
-            if (j == n_kv) mma_commit(&bar_o[t]);
+            if (j == n_kv_t) mma_commit(&bar_o[t]);
           }
-          if (j < n_kv) {
+          if (j < n_kv_t) {
             // S_t = Q_t K_jᵀ, both K-major, 32 bytes of the reduction dim per MMA.
             const uint32_t kaddr = ring + kslot * C::SLOT;
             const uint32_t qt = qaddr + t * C::Q_TILE;
@@ -370,7 +377,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float l_exact = 0.f;      // sum of the fp32 weights: gives the LSE
     float l_round = 0.f;      // sum of the bf16-rounded weights P uses: normalises O
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
+    const int n_kv_t = n_kv_of(t);
+    for (int j = 0; j < n_kv_t; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
       if (!ok) break;
       tc_fence_after();
