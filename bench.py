@@ -47,8 +47,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the SHA-256 of the kernel's sources at that capture. When the sources differ
 # the figure no longer describes the kernel and `traffic` is reported as null.
 KERNEL_SOURCES = ("io_aware_exact_17_b200/csrc/attn_fwd.cuh", "io_aware_exact_17_b200/csrc/sm100.cuh")
-NCU_TRAFFIC_BYTES = None
-NCU_TRAFFIC_SHA256 = None
+NCU_TRAFFIC_BYTES = 113745920  # 100.837120 MB read + 12.908800 MB written
+NCU_TRAFFIC_SHA256 = "6d072f683a539f1e75dff09f2f28ceafb119541020228db82c0ecd319d0ca483"
 
 
 def kernel_sources_sha256() -> str:
