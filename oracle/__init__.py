@@ -11,10 +11,19 @@ Pieces, each citing the passage it follows:
   (``attn_oracle.c``). Definition: "Flash Attention" glossary page, first two
   paragraphs (same result as standard attention; standard attention forms the
   N x N matrix).
+  Queries may be fewer than keys (the queries are then the last positions of
+  the sequence, for the causal mask), and a key range restricts the softmax to
+  one block of keys: the partial result the glossary page's online softmax
+  accumulates (second paragraph).
 * :func:`attention_naive` — a second, independently written fp64 routine that
   materialises the whole N x N score and probability matrices, i.e. the
   "standard attention" of "FlashAttention-3 (PT)", section "O problema do
   mecanismo de atenção". Used to cross-check :func:`attention` on tiny inputs.
+* :func:`lse_merge` — combines results over disjoint key blocks into the
+  result over their union, from their LSEs: the online-softmax rescale of the
+  glossary page (second paragraph) applied to whole partial results, as
+  splitting the keys over several processors needs (same page, fourth
+  paragraph, ring attention over several devices).
 * :func:`sylvester_hadamard`, :func:`rotation_matrix`, :func:`rotate` — the
   orthogonal transform of "FlashAttention-3 (PT)", section "Inovações técnicas",
   subsection 3 ("Baixa precisão (FP8)"), steps 1 and 4: Q and K multiplied by a
@@ -65,6 +74,12 @@ def _load():
             ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp, ctypes.c_int,
         ]
         lib.oracle_attn_rows.restype = ctypes.c_int
+        lib.oracle_attn_range_rows.argtypes = [
+            dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp,
+            ctypes.c_int,
+        ]
+        lib.oracle_attn_range_rows.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -79,22 +94,28 @@ def _as_f64(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
 
 
-def attention(q, k, v, causal: bool, scale: float, rows=None, threads: int | None = None):
-    """Exact attention of ``[B, H, N, d]`` inputs in fp64.
+def attention(q, k, v, causal: bool, scale: float, rows=None, threads: int | None = None, key_range=None):
+    """Exact attention in fp64 of ``q`` ``[B, H, Nq, d]`` over ``k``, ``v``
+    ``[B, H, Nk, d]``.
 
-    ``rows``: optional flat row ids ``(b*H + h)*N + i``; if given, only those rows
-    are computed and the result has shape ``[len(rows), d]`` / ``[len(rows)]``,
-    otherwise ``[B, H, N, d]`` / ``[B, H, N]``. Returns ``(O, LSE)`` with the
-    natural-log LSE.
+    ``causal``: key j is visible to query i iff j <= i + (Nk - Nq) (the queries
+    are the last Nq positions; for Nq = Nk, j <= i). ``key_range=(lo, hi)``:
+    only keys lo <= j < hi take part (default: all); rows left with no key get
+    O = 0 and LSE = -inf. ``rows``: optional flat row ids ``(b*H + h)*Nq + i``;
+    if given, only those rows are computed and the result has shape
+    ``[len(rows), d]`` / ``[len(rows)]``, otherwise ``[B, H, Nq, d]`` /
+    ``[B, H, Nq]``. Returns ``(O, LSE)`` with the natural-log LSE.
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
-    if q.ndim != 4 or q.shape != k.shape or q.shape != v.shape:
-        raise ValueError("q, k, v must share one [B, H, N, d] shape")
-    B, H, N, d = q.shape
+    if q.ndim != 4 or k.shape != v.shape or k.ndim != 4 or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be [B, H, Nq, d] and k, v one [B, H, Nk, d] shape")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    lo, hi = (0, Nk) if key_range is None else (int(key_range[0]), int(key_range[1]))
     lib = _load()
     dp = ctypes.POINTER(ctypes.c_double)
     if rows is None:
-        nrows = B * H * N
+        nrows = B * H * Nq
         rows_arr = None
         rows_ptr = None
     else:
@@ -103,35 +124,67 @@ def attention(q, k, v, causal: bool, scale: float, rows=None, threads: int | Non
         rows_ptr = rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
     o = np.zeros((nrows, d), dtype=np.float64)
     lse = np.zeros((nrows,), dtype=np.float64)
-    rc = lib.oracle_attn_rows(
-        q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp), B, H, N, d, int(bool(causal)),
-        float(scale), rows_ptr, nrows, o.ctypes.data_as(dp), lse.ctypes.data_as(dp),
+    rc = lib.oracle_attn_range_rows(
+        q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp), B, H, Nq, Nk, d, int(bool(causal)),
+        float(scale), lo, hi, rows_ptr, nrows, o.ctypes.data_as(dp), lse.ctypes.data_as(dp),
         int(threads or default_threads()),
     )
     if rc != 0:
-        raise RuntimeError(f"oracle_attn_rows failed with code {rc}")
+        raise RuntimeError(f"oracle_attn_range_rows failed with code {rc}")
     if rows is None:
-        return o.reshape(B, H, N, d), lse.reshape(B, H, N)
+        return o.reshape(B, H, Nq, d), lse.reshape(B, H, Nq)
     return o, lse
 
 
-def attention_naive(q, k, v, causal: bool, scale: float, return_probs: bool = False):
-    """Standard attention: materialise S = scale*Q Kᵀ (N x N per head), mask,
-    softmax along keys, then P V. fp64 numpy; for small N only."""
+def attention_naive(q, k, v, causal: bool, scale: float, return_probs: bool = False, key_range=None):
+    """Standard attention: materialise S = scale*Q Kᵀ (Nq x Nk per head), mask,
+    softmax along keys, then P V. fp64 numpy; for small sizes only.
+
+    Masked scores are -inf: keys j > i + (Nk - Nq) when causal, and keys outside
+    ``key_range = (lo, hi)``. A row with every key masked has P = 0, O = 0 and
+    LSE = -inf."""
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
-    N = q.shape[-2]
+    Nq, Nk = q.shape[-2], k.shape[-2]
     s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    hidden = np.zeros((Nq, Nk), dtype=bool)
     if causal:
-        future = np.triu(np.ones((N, N), dtype=bool), k=1)  # key j > query i
-        s = np.where(future, -np.inf, s)
+        hidden |= j > i + (Nk - Nq)
+    if key_range is not None:
+        hidden |= (j < key_range[0]) | (j >= key_range[1])
+    s = np.where(hidden, -np.inf, s)
     row_max = s.max(axis=-1, keepdims=True)
-    w = np.exp(s - row_max)
+    empty = np.isneginf(row_max)
+    w = np.where(empty, 0.0, np.exp(s - np.where(empty, 0.0, row_max)))
     denom = w.sum(axis=-1, keepdims=True)
-    p = w / denom
+    p = w / np.where(empty, 1.0, denom)
     o = np.einsum("bhij,bhjd->bhid", p, v)
-    lse = (row_max + np.log(denom))[..., 0]
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, row_max + np.log(denom))[..., 0]
     if return_probs:
         return o, lse, p
+    return o, lse
+
+
+def lse_merge(o_parts, lse_parts):
+    """Result over the union of disjoint key blocks from the results over each.
+
+    ``o_parts`` ``[S, ..., d]`` and ``lse_parts`` ``[S, ...]`` hold, for each
+    block s, the normalised output O_s and the natural-log LSE_s (-inf for a row
+    that saw no key of block s). With M = max_s LSE_s and w_s = exp(LSE_s - M):
+    LSE = M + ln(sum_s w_s) and O = sum_s w_s O_s / sum_s w_s, since
+    exp(LSE_s) is the softmax denominator of block s. Rows with no key in any
+    block get O = 0 and LSE = -inf. fp64."""
+    o_parts = _as_f64(o_parts)
+    lse_parts = _as_f64(lse_parts)
+    m = lse_parts.max(axis=0)
+    empty = np.isneginf(m)
+    w = np.where(empty[None], 0.0, np.exp(lse_parts - np.where(empty, 0.0, m)[None]))
+    total = w.sum(axis=0)
+    o = (w[..., None] * o_parts).sum(axis=0) / np.where(empty, 1.0, total)[..., None]
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, total)))
     return o, lse
 
 

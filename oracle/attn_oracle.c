@@ -11,19 +11,28 @@
  *   - "FlashAttention-3 (PT)", section "O problema do mecanismo de atenção": the
  *     self-attention that is quadratic in sequence length.
  *
- * For one query row i of head (b, h):
- *   allowed(i) = { j : 0 <= j < N and (not causal or j <= i) }
+ * For one query row i of head (b, h), with Nq query rows and Nk keys per head:
+ *   allowed(i) = { j : lo <= j < min(Nk, hi) and (not causal or j <= i + Nk - Nq) }
  *   z_j  = scale * sum_c q[i][c] * k[j][c]                    (fp64)
  *   m    = max_{j in allowed} z_j
  *   l    = sum_{j in allowed} exp(z_j - m)
  *   O[c] = sum_{j in allowed} exp(z_j - m) * v[j][c] / l
  *   LSE  = m + ln(l)                                           (natural log)
- * The causal rule (key j visible iff j <= i, top-left aligned square mask) and
- * the natural-log LSE are readings: the pages state neither.
+ * The causal rule and the natural-log LSE are readings: the pages state neither.
+ * Key j is visible to query i iff j <= i + (Nk - Nq): the queries are the last Nq
+ * positions of the key sequence. For Nq = Nk this is the square, top-left
+ * aligned mask j <= i.
  *
- * Layout: q, k, v are contiguous [B][H][N][d] fp64; o is [rows][d] and lse is
- * [rows], where the row list holds flat ids r = (b*H + h)*N + i (NULL = every row
- * in order). Work is split over rows across `nthreads` POSIX threads.
+ * The key range [lo, hi) restricts attention to a slice of the keys: the
+ * partial result over one block of keys that the online softmax of the
+ * "Flash Attention" glossary page (second paragraph) accumulates, here produced
+ * on its own. A row with no allowed key gets O = 0 and LSE = -inf (the empty
+ * sum). lo = 0, hi = Nk is ordinary attention.
+ *
+ * Layout: q is contiguous [B][H][Nq][d] fp64, k and v [B][H][Nk][d]; o is
+ * [rows][d] and lse is [rows], where the row list holds flat ids
+ * r = (b*H + h)*Nq + i (NULL = every row in order). Work is split over rows
+ * across `nthreads` POSIX threads.
  */
 #include <math.h>
 #include <pthread.h>
@@ -32,7 +41,7 @@
 
 typedef struct {
   const double *q, *k, *v;
-  int N, d, causal;
+  int Nq, Nk, d, causal, lo, hi;
   double scale;
   const int64_t* rows;
   int64_t row_begin, row_end;
@@ -41,16 +50,25 @@ typedef struct {
 } oracle_job;
 
 static void attend_one_row(const oracle_job* jb, int64_t out_idx, int64_t flat, double* z) {
-  const int N = jb->N, d = jb->d;
-  const int64_t bh = flat / N;
-  const int i = (int)(flat % N);
+  const int Nq = jb->Nq, Nk = jb->Nk, d = jb->d;
+  const int64_t bh = flat / Nq;
+  const int i = (int)(flat % Nq);
   const double* qi = jb->q + flat * d;
-  const double* kh = jb->k + bh * (int64_t)N * d;
-  const double* vh = jb->v + bh * (int64_t)N * d;
-  const int last = jb->causal ? i : N - 1; /* allowed keys are 0..last */
+  const double* kh = jb->k + bh * (int64_t)Nk * d;
+  const double* vh = jb->v + bh * (int64_t)Nk * d;
+  /* allowed keys are first..last */
+  const int first = jb->lo;
+  int last = (jb->hi < Nk ? jb->hi : Nk) - 1;
+  if (jb->causal && i + (Nk - Nq) < last) last = i + (Nk - Nq);
+  double* oi = jb->o + out_idx * d;
+  if (last < first) {
+    for (int c = 0; c < d; ++c) oi[c] = 0.0;
+    jb->lse[out_idx] = -INFINITY;
+    return;
+  }
 
   double m = -INFINITY;
-  for (int j = 0; j <= last; ++j) {
+  for (int j = first; j <= last; ++j) {
     const double* kj = kh + (int64_t)j * d;
     double dot = 0.0;
     for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
@@ -58,13 +76,12 @@ static void attend_one_row(const oracle_job* jb, int64_t out_idx, int64_t flat, 
     if (z[j] > m) m = z[j];
   }
   double l = 0.0;
-  for (int j = 0; j <= last; ++j) {
+  for (int j = first; j <= last; ++j) {
     z[j] = exp(z[j] - m); /* z now holds the unnormalised weights */
     l += z[j];
   }
-  double* oi = jb->o + out_idx * d;
   for (int c = 0; c < d; ++c) oi[c] = 0.0;
-  for (int j = 0; j <= last; ++j) {
+  for (int j = first; j <= last; ++j) {
     const double* vj = vh + (int64_t)j * d;
     for (int c = 0; c < d; ++c) oi[c] += z[j] * vj[c];
   }
@@ -74,7 +91,7 @@ static void attend_one_row(const oracle_job* jb, int64_t out_idx, int64_t flat, 
 
 static void* run_job(void* arg) {
   oracle_job* jb = (oracle_job*)arg;
-  double* z = (double*)malloc(sizeof(double) * (size_t)jb->N);
+  double* z = (double*)malloc(sizeof(double) * (size_t)jb->Nk);
   if (z == NULL) {
     jb->status = 1;
     return NULL;
@@ -89,11 +106,11 @@ static void* run_job(void* arg) {
 }
 
 /* Returns 0 on success, 1 on bad arguments, 2 on allocation/thread failure. */
-int oracle_attn_rows(const double* q, const double* k, const double* v, int B, int H, int N, int d,
-                     int causal, double scale, const int64_t* rows, int64_t nrows, double* o, double* lse,
-                     int nthreads) {
-  if (B < 1 || H < 1 || N < 1 || d < 1 || !q || !k || !v || !o || !lse) return 1;
-  const int64_t total = (int64_t)B * H * N;
+int oracle_attn_range_rows(const double* q, const double* k, const double* v, int B, int H, int Nq, int Nk,
+                           int d, int causal, double scale, int lo, int hi, const int64_t* rows, int64_t nrows,
+                           double* o, double* lse, int nthreads) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || d < 1 || lo < 0 || hi < lo || !q || !k || !v || !o || !lse) return 1;
+  const int64_t total = (int64_t)B * H * Nq;
   if (rows == NULL) nrows = total;
   for (int64_t r = 0; rows && r < nrows; ++r)
     if (rows[r] < 0 || rows[r] >= total) return 1;
@@ -112,7 +129,8 @@ int oracle_attn_rows(const double* q, const double* k, const double* v, int B, i
   for (int t = 0; t < nthreads; ++t) {
     oracle_job* jb = &jobs[t];
     jb->q = q; jb->k = k; jb->v = v;
-    jb->N = N; jb->d = d; jb->causal = causal; jb->scale = scale;
+    jb->Nq = Nq; jb->Nk = Nk; jb->d = d; jb->causal = causal; jb->scale = scale;
+    jb->lo = lo; jb->hi = hi;
     jb->rows = rows;
     jb->row_begin = nrows * t / nthreads;
     jb->row_end = nrows * (t + 1) / nthreads;
@@ -131,4 +149,11 @@ int oracle_attn_rows(const double* q, const double* k, const double* v, int B, i
   free(jobs);
   free(tids);
   return rc;
+}
+
+/* Square attention (Nq = Nk = N) over every key. */
+int oracle_attn_rows(const double* q, const double* k, const double* v, int B, int H, int N, int d,
+                     int causal, double scale, const int64_t* rows, int64_t nrows, double* o, double* lse,
+                     int nthreads) {
+  return oracle_attn_range_rows(q, k, v, B, H, N, N, d, causal, scale, 0, N, rows, nrows, o, lse, nthreads);
 }

@@ -26,3 +26,16 @@ def rel_rmse(a: np.ndarray, ref: np.ndarray) -> float:
 
 def max_abs(a: np.ndarray, ref: np.ndarray) -> float:
     return float(np.max(np.abs(a - ref))) if a.size else 0.0
+
+
+def record(case: str, **values) -> None:
+    """Append one JSON line {case, values...} to the file named by the
+    FA_PARITY_LOG environment variable, if set: the measured errors of a GPU
+    parity run, kept for reporting. Does nothing otherwise."""
+    import json
+    import os
+
+    path = os.environ.get("FA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, **{k: float(v) for k, v in values.items()}}) + "\n")

@@ -12,7 +12,7 @@ import torch
 import oracle
 import io_aware_exact_17_b200 as fa
 from io_aware_exact_17_b200 import inputs
-from helpers import BF16_LSE_ATOL, BF16_O_ATOL, FP8_REL_RMSE, max_abs, rel_rmse, to_np
+from helpers import BF16_LSE_ATOL, BF16_O_ATOL, FP8_REL_RMSE, max_abs, record, rel_rmse, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -112,6 +112,8 @@ def test_fp8_config_rel_rmse_sampled():
     for rotate in (False, True):
         o, *_ = _fp8_attention(q, k, v, False, rotate, inputs.hadamard_signs(d, 1003) if rotate else None)
         err = rel_rmse(to_np(o).reshape(-1, d)[rows], o_ref)
+        record(f"e4m3 QK B{B} H{H} N{N} d{d} N(0,1) {'rotated' if rotate else 'unrotated'} (sampled rows)",
+               rel_rmse=err)
         assert err <= FP8_REL_RMSE, (rotate, err)
 
 
@@ -125,6 +127,8 @@ def test_fp8_outliers_rotation_strictly_better():
     for rotate in (False, True):
         o, *_ = _fp8_attention(q1, k1, v, False, rotate, inputs.hadamard_signs(d, 1003) if rotate else None)
         err[rotate] = rel_rmse(to_np(o).reshape(-1, d)[rows], o_ref)
+    record(f"e4m3 QK B{B} H{H} N{N} d{d} outliers (sampled rows)", rel_rmse_rotated=err[True],
+           rel_rmse_unrotated=err[False])
     assert err[True] < err[False], err
 
 

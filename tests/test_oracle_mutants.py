@@ -1,9 +1,10 @@
-"""The pins in test_oracle.py must be able to fail. Each case here plants one
+"""The oracle's pins must be able to fail. Each case here plants one
 plausible mistake in a private copy of the oracle's C source (a dropped scale,
 a dropped mask, an off-by-one key range, a wrong operand index, a transposed
 value operand, a dropped normalisation, an LSE without the max, an unshifted
-exponent), builds it, and checks that at least one pin rejects it. Nothing
-here touches the real oracle library.
+exponent, a causal mask that ignores the query offset, a key range whose start
+or end is ignored, an empty row with a finite LSE), builds it, and checks that
+at least one pin rejects it. Nothing here touches the real oracle library.
 """
 import ctypes
 import json
@@ -21,8 +22,12 @@ GOLDEN = json.loads((ROOT / "tests" / "golden" / "attention_closed_form.json").r
 
 MUTANTS = {
     "dropped_scale": ("z[j] = jb->scale * dot;", "z[j] = dot;"),
-    "dropped_mask": ("jb->causal ? i : N - 1", "N - 1"),
-    "off_by_one_keys": ("const int last = jb->causal ? i : N - 1;", "const int last = jb->causal ? i - (i > 0) : N - 2 + (N == 1);"),
+    "dropped_mask": ("if (jb->causal && i + (Nk - Nq) < last) last = i + (Nk - Nq);", ""),
+    "off_by_one_keys": ("int last = (jb->hi < Nk ? jb->hi : Nk) - 1;", "int last = (jb->hi < Nk ? jb->hi : Nk) - 2 + (Nk == 1);"),
+    "causal_offset_ignored": ("i + (Nk - Nq) < last) last = i + (Nk - Nq);", "i < last) last = i;"),
+    "range_start_ignored": ("const int first = jb->lo;", "const int first = 0;"),
+    "range_end_ignored": ("int last = (jb->hi < Nk ? jb->hi : Nk) - 1;", "int last = Nk - 1;"),
+    "empty_row_not_empty": ("jb->lse[out_idx] = -INFINITY;", "jb->lse[out_idx] = 0.0;"),
     "wrong_k_index": ("dot += qi[c] * kj[c];", "dot += qi[c] * kj[0];"),
     "transposed_v": ("oi[c] += z[j] * vj[c];", "oi[c] += z[j] * vj[d - 1 - c];"),
     "no_normalisation": ("oi[c] /= l;", "oi[c] /= 1.0;"),
@@ -42,6 +47,10 @@ def _build(tmp_path, name, src):
     lib.oracle_attn_rows.argtypes = [dp, dp, dp] + [ctypes.c_int] * 5 + [
         ctypes.c_double, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp, ctypes.c_int]
     lib.oracle_attn_rows.restype = ctypes.c_int
+    lib.oracle_attn_range_rows.argtypes = [dp, dp, dp] + [ctypes.c_int] * 6 + [
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp,
+        ctypes.c_int]
+    lib.oracle_attn_range_rows.restype = ctypes.c_int
     return lib
 
 
@@ -57,6 +66,28 @@ def _run(lib, q, k, v, causal, scale):
                                   lse.ctypes.data_as(dp), 1)
     assert rc == 0
     return o.reshape(B, H, N, d), lse.reshape(B, H, N)
+
+
+def _run_range(lib, q, k, v, causal, scale, lo, hi):
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    dp = ctypes.POINTER(ctypes.c_double)
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    o = np.zeros((B * H * Nq, d))
+    lse = np.zeros(B * H * Nq)
+    with np.errstate(all="ignore"):
+        rc = lib.oracle_attn_range_rows(q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp), B, H, Nq,
+                                        Nk, d, int(causal), scale, lo, hi, None, B * H * Nq, o.ctypes.data_as(dp),
+                                        lse.ctypes.data_as(dp), 1)
+    assert rc == 0
+    return o.reshape(B, H, Nq, d), lse.reshape(B, H, Nq)
+
+
+def _same(o, lse, o2, lse2) -> bool:
+    with np.errstate(all="ignore"):
+        return bool(np.allclose(o, o2, rtol=0, atol=1e-12) and np.array_equal(np.isneginf(lse), np.isneginf(lse2))
+                    and np.allclose(np.where(np.isinf(lse), 0, lse), np.where(np.isinf(lse2), 0, lse2), rtol=0,
+                                    atol=1e-12))
 
 
 def _pins_pass(lib) -> bool:
@@ -85,6 +116,14 @@ def _pins_pass(lib) -> bool:
     v = rng.standard_normal((1, 1, N, d))
     o, _ = _run(lib, q, k, v, False, 1.0)
     ok &= np.allclose(o[0, 0], np.broadcast_to(v[0, 0, 5], (N, d)), rtol=0, atol=1e-12)
+    # fewer queries than keys, and key ranges, against the materialised routine
+    q = rng.standard_normal((1, 2, 5, 8))
+    k, v = rng.standard_normal((1, 2, 19, 8)), rng.standard_normal((1, 2, 19, 8))
+    for causal in (False, True):
+        for lo, hi in ((0, 19), (3, 11), (15, 19)):
+            o, lse = _run_range(lib, q, k, v, causal, 0.45, lo, hi)
+            o2, lse2 = oracle.attention_naive(q, k, v, causal, 0.45, key_range=(lo, hi))
+            ok &= _same(o, lse, o2, lse2)
     return bool(ok)
 
 
