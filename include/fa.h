@@ -65,6 +65,80 @@ typedef enum {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
                  int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, void* stream);
 
+/*
+ * fa_fwd_splitkv — attention of Nq queries over Nk keys per head (decode- and
+ * chunk-shaped problems: few queries, long key sequences), with the keys split
+ * into n_split blocks that separate CTAs process in parallel, then merged.
+ *
+ * Defined by: the same output as fa_fwd (standard attention; "Flash Attention"
+ * glossary page, paragraphs 1-2), for a query block that is the last Nq
+ * positions of the key sequence. The split follows the glossary page's second
+ * paragraph: the online softmax accumulates results over blocks of keys; here
+ * the blocks are computed at once and combined by their LSEs (fa_lse_merge).
+ * FlashDecoding++ ("FlashAttention-3 (PT)", references) is the pages' title for
+ * this decode setting; the pages give no algorithm for it. For query row i:
+ *   key j is visible iff j < Nk and (causal == 0 or j <= i + (Nk - Nq)).
+ *
+ * q       device, [B][H][Nq][d] (bf16, or e4m3 codes for FA_E4M3), 16-byte aligned.
+ * k, v    device, [B][H][Nk][d] (k: bf16 or e4m3 codes; v: bf16), 16-byte aligned.
+ * o       device, bf16 [B][H][Nq][d] output; lse fp32 [B][H][Nq] (natural log) or NULL.
+ * B, H, Nq, Nk >= 1; causal requires Nq <= Nk. d, scale, qk_dtype, descale_qk: as fa_fwd.
+ * n_split 1 = no split (no workspace; the same kernel as fa_fwd); >= 2 = that many
+ *         blocks of ceil(ceil(Nk/128)/n_split) key tiles of 128 keys (the last ones
+ *         may be empty); 0 = fa_fwd_splitkv_splits(B, H, Nq, Nk, d).
+ * workspace  device, >= fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split)
+ *         bytes, 256-byte aligned, owned by the caller (may be NULL if that is 0);
+ *         overwritten. Calls that overlap on the GPU must not share it.
+ * Errors: FA_ERR_INVALID_ARG (also: workspace missing or too small),
+ *         FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                         int Nk, int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk,
+                         int n_split, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of fa_fwd_splitkv for these sizes (n_split = 0: the automatic
+ * count on the current device); 0 when no workspace is needed or on bad sizes. */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split);
+
+/* The split count fa_fwd_splitkv uses for n_split = 0 on the current device: the
+ * count that gives the fewest key-tile steps on the busiest SM (one CTA per SM),
+ * at least 1. */
+int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d);
+
+/*
+ * fa_fwd_partial — the per-block results of fa_fwd_splitkv, without the merge:
+ * for block s (keys of tiles s*T .. s*T+T-1, T = ceil(ceil(Nk/128)/n_split)), the
+ * output normalised over that block's visible keys and its LSE. Blocks computed
+ * by separate calls (for example over key chunks that arrive one at a time from
+ * other devices, as in ring attention: "Flash Attention" glossary page, fourth
+ * paragraph) combine with fa_lse_merge.
+ *
+ * o_part    device, fp32 [n_split][B][H][Nq][d], 16-byte aligned.
+ * lse_part  device, fp32 [n_split][B][H][Nq] (natural log), 4-byte aligned. A row
+ *           with no visible key in a block gets O = 0 and LSE = -inf there.
+ * Other arguments as fa_fwd_splitkv (n_split >= 1).
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int H,
+                         int Nq, int Nk, int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk,
+                         int n_split, void* stream);
+
+/*
+ * fa_lse_merge — combine results over disjoint blocks of keys into the result over
+ * their union. With M = max_s LSE_s and w_s = exp(LSE_s - M) per row:
+ *   O = sum_s w_s O_s / sum_s w_s  (bf16, round to nearest even),
+ *   LSE = M + ln sum_s w_s;        rows with every LSE_s = -inf get O = 0, LSE = -inf.
+ * Defined by: "Flash Attention" glossary page, second paragraph (the online
+ * softmax's rescale of partial results), applied to whole partial results.
+ *
+ * o_part    device, fp32 [n_part][rows][d], 16-byte aligned; lse_part fp32 [n_part][rows].
+ * o         device, bf16 [rows][d], 16-byte aligned; lse fp32 [rows] or NULL.
+ * n_part >= 1; rows >= 1; d in {64, 128, 256}.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
+                       float* lse, void* stream);
+
 /* Bytes of device workspace fa_hadamard_quant needs (the amax word and a grid-barrier counter, padded). */
 #define FA_QUANT_WORKSPACE_BYTES 256
 
@@ -136,7 +210,7 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
 
-/* ABI version of this header: 1. */
+/* ABI version of this header: 2 (1 plus the split-key, partial and merge calls). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

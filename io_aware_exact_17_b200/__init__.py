@@ -1,5 +1,7 @@
 """Fused exact-attention forward for B200 (sm_100a): BF16 and FP8-e4m3 kernels,
-and the Hadamard rotate-and-quantise step of the FP8 path.
+the Hadamard rotate-and-quantise step of the FP8 path, and attention of few
+queries over long key sequences with the keys split across CTAs and merged by
+their LSEs.
 
 The compute lives in ``libfa.so`` (CUDA, built from ``csrc/``); this package is
 its Python binding. Importing the package does not load the library; the first
@@ -9,9 +11,14 @@ from .binding import (  # noqa: F401
     FaError,
     device_status,
     fwd,
+    fwd_partial,
+    fwd_splitkv,
     hadamard_quant,
     library_path,
     load_library,
+    lse_merge,
+    splitkv_splits,
 )
 
-__all__ = ["fwd", "hadamard_quant", "device_status", "load_library", "library_path", "FaError"]
+__all__ = ["fwd", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant", "device_status",
+           "load_library", "library_path", "FaError"]

@@ -59,6 +59,16 @@ def load_library():
         lib.fa_device_status.restype = i
         lib.fa_abi_version.argtypes = []
         lib.fa_abi_version.restype = i
+        lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
+        lib.fa_fwd_splitkv.restype = i
+        lib.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        lib.fa_fwd_splitkv_workspace_bytes.restype = sz
+        lib.fa_fwd_splitkv_splits.argtypes = [i, i, i, i, i]
+        lib.fa_fwd_splitkv_splits.restype = i
+        lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp]
+        lib.fa_fwd_partial.restype = i
+        lib.fa_lse_merge.argtypes = [vp, vp, i, i64, i, vp, vp, vp]
+        lib.fa_lse_merge.restype = i
         _lib = lib
         return lib
 
@@ -118,6 +128,110 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
                         int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
                         _ptr(qk_descale.contiguous()) if fp8 else None, _stream(q.device))
     _check(rc, "fa_fwd")
+    return out, (lse if return_lse else None)
+
+
+def _qkv_kinds(q, k, v, qk_descale):
+    """Shapes and dtypes of q [B, H, Nq, d] against k, v [B, H, Nk, d]; returns
+    (B, H, Nq, Nk, d, fp8)."""
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise FaError("q must be [B, H, Nq, d] and k, v one [B, H, Nk, d] shape")
+    fp8 = q.dtype in E4M3_DTYPES
+    if fp8 != (k.dtype in E4M3_DTYPES) or (not fp8 and (q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16)):
+        raise FaError("q and k must both be bf16 or both e4m3")
+    if v.dtype != torch.bfloat16:
+        raise FaError("v must be bf16")
+    if fp8 and (qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2):
+        raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk]")
+    B, H, Nq, d = q.shape
+    return B, H, Nq, k.shape[2], d, fp8
+
+
+def splitkv_splits(B: int, H: int, Nq: int, Nk: int, d: int, device=None) -> int:
+    """The split count ``fwd_splitkv`` picks for ``n_split=0`` on ``device``."""
+    lib = load_library()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(lib.fa_fwd_splitkv_splits(B, H, Nq, Nk, d))
+
+
+def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=None, n_split: int = 0,
+                out=None, lse=None, workspace=None, return_lse: bool = True):
+    """Attention of ``q`` ``[B, H, Nq, d]`` over ``k``, ``v`` ``[B, H, Nk, d]``
+    through ``fa_fwd_splitkv``: the keys are split into ``n_split`` blocks (0 =
+    automatic) processed in parallel and merged by their LSEs. With ``causal``,
+    query i is position ``Nk - Nq + i`` (Nq <= Nk). Returns ``(O, LSE)`` as
+    :func:`fwd`. ``workspace``: optional uint8 CUDA tensor of at least
+    ``fa_fwd_splitkv_workspace_bytes`` bytes (allocated here if not given)."""
+    _require_cuda(q, k, v)
+    lib = load_library()
+    B, H, Nq, Nk, d, fp8 = _qkv_kinds(q, k, v, qk_descale)
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(q.device):
+        if n_split == 0:
+            n_split = int(lib.fa_fwd_splitkv_splits(B, H, Nq, Nk, d))
+        need = int(lib.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, int(n_split)))
+        if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        rc = lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, Nq,
+                                Nk, d, int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
+                                _ptr(qk_descale.contiguous()) if fp8 else None, int(n_split),
+                                _ptr(workspace) if need > 0 else None, ws_bytes, _stream(q.device))
+    _check(rc, "fa_fwd_splitkv")
+    return out, (lse if return_lse else None)
+
+
+def fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=None, n_split: int = 1,
+                o_part=None, lse_part=None):
+    """Per-block attention results through ``fa_fwd_partial``: for each of the
+    ``n_split`` blocks of keys, fp32 ``O_s`` ``[n_split, B, H, Nq, d]``
+    (normalised over the block) and ``LSE_s`` ``[n_split, B, H, Nq]`` (natural
+    log; -inf and O = 0 where a row sees no key of the block)."""
+    _require_cuda(q, k, v)
+    lib = load_library()
+    B, H, Nq, Nk, d, fp8 = _qkv_kinds(q, k, v, qk_descale)
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if o_part is None:
+        o_part = torch.empty((n_split, B, H, Nq, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((n_split, B, H, Nq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(q.device):
+        rc = lib.fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, Nq, Nk, d,
+                                int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
+                                _ptr(qk_descale.contiguous()) if fp8 else None, int(n_split), _stream(q.device))
+    _check(rc, "fa_fwd_partial")
+    return o_part, lse_part
+
+
+def lse_merge(o_part, lse_part, out=None, lse=None, return_lse: bool = True):
+    """Merge per-block results ``o_part`` ``[S, ..., d]`` (fp32) and ``lse_part``
+    ``[S, ...]`` through ``fa_lse_merge`` into bf16 ``O`` ``[..., d]`` and fp32
+    ``LSE`` ``[...]``."""
+    _require_cuda(o_part, lse_part)
+    lib = load_library()
+    if o_part.dtype != torch.float32 or lse_part.dtype != torch.float32:
+        raise FaError("o_part and lse_part must be fp32")
+    if o_part.dim() < 2 or tuple(o_part.shape[:-1]) != tuple(lse_part.shape):
+        raise FaError("o_part must be [S, ..., d] and lse_part [S, ...]")
+    n_part, d = o_part.shape[0], o_part.shape[-1]
+    rows = lse_part[0].numel()
+    o_part, lse_part = o_part.contiguous(), lse_part.contiguous()
+    if out is None:
+        out = torch.empty(tuple(o_part.shape[1:]), dtype=torch.bfloat16, device=o_part.device)
+    if return_lse and lse is None:
+        lse = torch.empty(tuple(lse_part.shape[1:]), dtype=torch.float32, device=o_part.device)
+    with torch.cuda.device(o_part.device):
+        rc = lib.fa_lse_merge(_ptr(o_part), _ptr(lse_part), n_part, rows, d, _ptr(out),
+                              _ptr(lse) if return_lse else None, _stream(o_part.device))
+    _check(rc, "fa_lse_merge")
     return out, (lse if return_lse else None)
 
 

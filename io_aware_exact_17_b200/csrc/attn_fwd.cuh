@@ -69,7 +69,8 @@ struct FwdCfg {
   static constexpr int REG_OTHER = FA_REG_OTHER;      // per thread of the last warpgroup after .dec
   static_assert(!SPLIT_REGS || SOFTMAX_WARPS * 32 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * REG_LAUNCH,
                 "register split exceeds the block's launch allocation");
-  static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns: S (128 fp32 per tile) then O (D per tile), allocated as a power of two.
+  static constexpr uint32_t TMEM_COLS = NQ * (128 + D) <= 256 ? 256u : 512u;
   static constexpr uint32_t S_COL(int t) { return static_cast<uint32_t>(t) * 128u; }
   static constexpr uint32_t P_COL(int t) { return S_COL(t); }  // 64 columns of bf16 pairs over S
   static constexpr uint32_t O_COL(int t) { return static_cast<uint32_t>(NQ) * 128u + static_cast<uint32_t>(t * D); }
@@ -78,15 +79,22 @@ struct FwdCfg {
   static_assert(NSLOT >= 2, "ring needs two slots");
   static_assert(NQ * 128 + NQ * D <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-  static_assert(SMEM_BYTES > 114 * 1024, "one CTA per SM (TMEM is allocated whole)");
+  // Two co-resident CTAs must not both want all 512 TMEM columns.
+  static_assert(SMEM_BYTES > 114 * 1024 || TMEM_COLS <= 256, "TMEM of co-resident CTAs");
 };
 
 struct FwdParams {
-  __nv_bfloat16* o;          // [BH][N][D]
-  float* lse;                // [BH][N], may be null
+  __nv_bfloat16* o;          // [BH][Nq][D]; null in partial mode
+  float* lse;                // [BH][Nq], may be null
+  float* o_part;             // partial mode: [n_split][BH][Nq][D] fp32, O of the split's keys; else null
+  float* lse_part;           // partial mode: [n_split][BH][Nq], -inf where a row sees no key of the split
   const float* descale_qk;   // e4m3 path: {dq, dk}; else null
-  int N;
+  int BH;                    // batch * heads
+  int Nq, Nk;                // query rows and keys per head
+  int causal_off;            // Nk - Nq: key j is visible to query i iff j <= i + causal_off (causal)
   int n_qb;                  // query blocks (NQ*128 rows) per head
+  int n_split;               // key splits per head (1: all keys)
+  int split_tiles;           // key tiles per split
   float scale_log2;          // scale * log2(e)
 };
 
@@ -226,19 +234,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   const uint32_t warp = warp_id(), lane = lane_id();
 
-  // Work item: head bh, query block qb (heaviest causal blocks of a head first).
-  const int bh = blockIdx.x / p.n_qb;
+  // Work item: head bh, key split sp, query block qb (heaviest causal blocks of
+  // a head first).
+  const int bh = blockIdx.x / (p.n_qb * p.n_split);
+  const int sp = (blockIdx.x / p.n_qb) % p.n_split;
   int qb = blockIdx.x % p.n_qb;
   if (CAUSAL) qb = p.n_qb - 1 - qb;
   const int q0 = qb * NQ * C::BM;
-  // KV tiles a query tile needs: all of them, or (causal) up to its last row.
-  // The CTA streams n_kv = the last tile's count; an earlier causal tile stops sooner
-  // (n_kv_t), so it never spends a step on a key tile that is entirely in its future.
+  // Key tiles of this split: kt0 .. kt0 + split_tiles - 1 (clipped to Nk). Query
+  // tile t steps through n_kv_of(t) of them: none if it has no row (past Nq),
+  // else up to the tile holding its last visible key, so a causal tile never
+  // spends a step on keys entirely in its future. The CTA streams the most any
+  // tile needs.
+  const int kt0 = sp * p.split_tiles;
   auto n_kv_of = [&](int t) {
-    const int end = CAUSAL ? min(p.N, q0 + (t + 1) * C::BM) : p.N;
-    return (end + C::BN - 1) / C::BN;
+    const int row0 = q0 + t * C::BM;
+    if (row0 >= p.Nq) return 0;
+    const int end = CAUSAL ? min(p.Nk, min(p.Nq, row0 + C::BM) + p.causal_off) : p.Nk;  // keys [0, end)
+    const int tiles = min((end + C::BN - 1) / C::BN, kt0 + p.split_tiles);
+    return max(0, tiles - kt0);
   };
-  const int n_kv = n_kv_of(NQ - 1);
+  const int n_kv0 = n_kv_of(0);
+  const int n_kv1 = NQ > 1 ? n_kv_of(NQ - 1) : n_kv0;
+  const int n_kv = max(n_kv0, n_kv1);
+  auto n_kv_at = [&](int t) { return t == 0 ? n_kv0 : n_kv1; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -291,11 +310,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (kind == 0) {
             mbar_arrive_expect_tx(&bar_full[slot], C::K_TILE);
             for (int c = 0; c < C::QK_CHUNKS; ++c)
-              tma_load_3d(dst + c * (C::BN * 128), &tmK, &bar_full[slot], c * (128 / C::EQK), j * C::BN, bh);
+              tma_load_3d(dst + c * (C::BN * 128), &tmK, &bar_full[slot], c * (128 / C::EQK), (kt0 + j) * C::BN,
+                          bh);
           } else {
             mbar_arrive_expect_tx(&bar_full[slot], C::V_TILE);
             for (int c = 0; c < C::V_CHUNKS; ++c)
-              tma_load_3d(dst + c * (C::BN * 128), &tmV, &bar_full[slot], c * 64, j * C::BN, bh);
+              tma_load_3d(dst + c * (C::BN * 128), &tmV, &bar_full[slot], c * 64, (kt0 + j) * C::BN, bh);
           }
         }
       }
@@ -318,7 +338,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < NQ && ok; ++t) {
-          const int n_kv_t = n_kv_of(t);
+          const int n_kv_t = n_kv_at(t);
           if (j > 0 && j - 1 < n_kv_t) {
             // The single issuer polls: its wake-up is on the critical path.
             ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, kMmaWaitSleepNs);
@@ -372,32 +392,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tO = row_addr + C::O_COL(t);
     float s_log2 = p.scale_log2;
     if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
-    const int kmax = CAUSAL ? min(qrow, p.N - 1) : p.N - 1;  // last visible key of this row
+    // Last visible key of this row, counted from the split's first key (so the
+    // loop below works in split-relative key indices).
+    const int kmax = (CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1) - kt0 * C::BN;
     float m_ref = -INFINITY;  // reference max, scaled log2 units
     float l_exact = 0.f;      // sum of the fp32 weights: gives the LSE
     float l_round = 0.f;      // sum of the bf16-rounded weights P uses: normalises O
     bool ok = true;
-    const int n_kv_t = n_kv_of(t);
+    const int n_kv_t = n_kv_at(t);
     for (int j = 0; j < n_kv_t; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
-      const int kbase = j * C::BN;
+      const int kbase = j * C::BN;  // split-relative
       // Some key of this tile is not visible to some row of this warp. Warp-uniform:
       // it selects code paths that issue tcgen05.ld, which all 32 lanes must
       // execute together (a lane-divergent .sync.aligned instruction deadlocks).
       const bool masked = __any_sync(0xffffffffu, kbase + C::BN - 1 > kmax);
       float sum_e, sum_r, alpha = 1.0f, mx = 0.f;
       if (j == 0) {
-        m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;  // finite: key 0 is visible
-        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        // -inf only for a row that sees no key of this split (partial mode): its
+        // weights are then exp2(-inf - 0) = 0 throughout.
+        m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;
+        softmax_row_dispatch<false>(tS, s, s_log2, m_ref == -INFINITY ? 0.f : m_ref, kbase, kmax, masked, sum_e,
+                                    sum_r, mx);
       } else {
         // Exponentials against the current reference, taking the row's max on the
         // way; only if some row's max grew by more than 2^8 (rare after the first
         // tiles) is the row redone against the new reference. S is still intact:
         // P is written only below.
-        softmax_row_dispatch<true>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        softmax_row_dispatch<true>(tS, s, s_log2, m_ref == -INFINITY ? 0.f : m_ref, kbase, kmax, masked, sum_e,
+                                   sum_r, mx);
         const float mx_s = mx * s_log2;
         const bool grow = mx_s > m_ref + 8.0f;
         if (__any_sync(0xffffffffu, grow)) {
@@ -428,12 +454,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_p[t]);  // one arrival per warp
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
-    if (ok) {
+    if (ok && n_kv_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
+    const bool in_range = qrow < p.Nq;
+    if (ok && p.o_part != nullptr) {
+      // Partial mode: O of this split's keys in fp32 (normalised by its own
+      // weights) and its LSE; a row with no key of the split gets 0 and -inf.
+      const bool empty = l_exact == 0.f;
+      const size_t prow = (static_cast<size_t>(sp) * p.BH + bh) * p.Nq + (in_range ? qrow : 0);
+      float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+      if (n_kv_t > 0) tc_fence_after();
+      const float inv_l = empty ? 0.f : 1.0f / l_round;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        if (n_kv_t > 0) {
+          tmem_ld32(tO + c0, ov);
+          tmem_wait_ld_dep32(ov);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        }
+        if (in_range) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[c0 / 4 + i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
+                                          __uint_as_float(ov[4 * i + 2]) * inv_l,
+                                          __uint_as_float(ov[4 * i + 3]) * inv_l);
+        }
+      }
+      if (in_range)
+        p.lse_part[prow] = empty ? -INFINITY : (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
+    } else if (ok && n_kv_t > 0) {
       tc_fence_after();
       const float inv_l = 1.0f / l_round;
-      const bool in_range = qrow < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? qrow : 0)) * D;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Nq + (in_range ? qrow : 0)) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
@@ -450,7 +504,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       if (in_range && p.lse != nullptr)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
+        p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     }
   }
 

@@ -10,6 +10,7 @@
 
 #include "../../include/fa.h"
 #include "attn_fwd.cuh"
+#include "merge.cuh"
 #include "quant.cuh"
 #include "tmap.h"
 
@@ -33,16 +34,38 @@ bool set_smem_once(K kernel, int bytes, unsigned long long* done_mask) {
   return true;
 }
 
+// Everything one attention launch needs (argument checks are done by the caller).
+struct FwdArgs {
+  const void *q, *k, *v;
+  void* o;              // bf16 output (direct mode)
+  float* lse;           // may be null (direct mode)
+  float* o_part;        // partial mode (n_split >= 1 blocks of keys, fp32); null = direct mode
+  float* lse_part;
+  int B, H, Nq, Nk, d;
+  bool causal;
+  float scale;
+  fa_dtype qk_dtype;
+  const float* descale_qk;
+  int n_split;
+};
+
+constexpr int kKeyTile = 128;  // keys per K/V tile (FwdCfg::BN)
+
+inline int key_tiles(int Nk) { return (Nk + kKeyTile - 1) / kKeyTile; }
+
+// Query tiles per CTA: two (ping-pong) when d <= 128 and a head has more than
+// one tile of queries; one for d = 256 (TMEM) and for short query blocks.
+inline int nq_for(int d, int Nq) { return (d <= 128 && Nq > 128) ? 2 : 1; }
+
 template <int D, int NQ, bool CAUSAL, bool QK_FP8>
-fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-                     float scale, const float* descale_qk, cudaStream_t stream) {
+fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D, NQ, QK_FP8>;
-  const int BH = B * H;
+  const int BH = a.B * a.H;
   CUtensorMap tmQ, tmK, tmV;
   const CUtensorMapDataType qk_type = QK_FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!fa::make_tmap_3d(&tmQ, q, qk_type, C::EQK, D, N, BH, 128 / C::EQK, C::BM) ||
-      !fa::make_tmap_3d(&tmK, k, qk_type, C::EQK, D, N, BH, 128 / C::EQK, C::BN) ||
-      !fa::make_tmap_3d(&tmV, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64, C::BN))
+  if (!fa::make_tmap_3d(&tmQ, a.q, qk_type, C::EQK, D, a.Nq, BH, 128 / C::EQK, C::BM) ||
+      !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
+      !fa::make_tmap_3d(&tmV, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nk, BH, 64, C::BN))
     return FA_ERR_CUDA;
   auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8>;
   static unsigned long long smem_done = 0;
@@ -60,16 +83,116 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
     }
     if (checked != 1) return FA_ERR_UNSUPPORTED;
   }
+  static_assert(C::BN == kKeyTile, "key tile");
   FwdParams p;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.descale_qk = descale_qk;
-  p.N = N;
-  p.n_qb = (N + NQ * C::BM - 1) / (NQ * C::BM);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  const long long grid = static_cast<long long>(p.n_qb) * BH;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.o_part = a.o_part;
+  p.lse_part = a.lse_part;
+  p.descale_qk = a.descale_qk;
+  p.BH = BH;
+  p.Nq = a.Nq;
+  p.Nk = a.Nk;
+  p.causal_off = a.Nk - a.Nq;
+  p.n_qb = (a.Nq + NQ * C::BM - 1) / (NQ * C::BM);
+  p.n_split = a.n_split;
+  p.split_tiles = (key_tiles(a.Nk) + a.n_split - 1) / a.n_split;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const long long grid = static_cast<long long>(p.n_qb) * a.n_split * BH;
   kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, int NQ, bool QK_FP8>
+fa_status launch_fwd_c(const FwdArgs& a, cudaStream_t s) {
+  return a.causal ? launch_fwd<D, NQ, true, QK_FP8>(a, s) : launch_fwd<D, NQ, false, QK_FP8>(a, s);
+}
+
+// Kernel choice by head dimension, dtype and query length.
+fa_status dispatch_fwd(const FwdArgs& a, cudaStream_t s) {
+  const bool two = nq_for(a.d, a.Nq) == 2;
+  if (a.qk_dtype == FA_BF16) {
+    switch (a.d) {
+      case 64: return two ? launch_fwd_c<64, 2, false>(a, s) : launch_fwd_c<64, 1, false>(a, s);
+      case 128: return two ? launch_fwd_c<128, 2, false>(a, s) : launch_fwd_c<128, 1, false>(a, s);
+      default: return launch_fwd_c<256, 1, false>(a, s);
+    }
+  }
+  switch (a.d) {
+    case 128: return two ? launch_fwd_c<128, 2, true>(a, s) : launch_fwd_c<128, 1, true>(a, s);
+    default: return launch_fwd_c<256, 1, true>(a, s);
+  }
+}
+
+// Checks shared by every attention entry point.
+fa_status check_fwd_args(const void* q, const void* k, const void* v, int B, int H, int Nq, int Nk, int d,
+                         int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, int n_split) {
+  if (q == nullptr || k == nullptr || v == nullptr) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || n_split < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && Nq > Nk) return FA_ERR_INVALID_ARG;  // some query would see no key
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (qk_dtype != FA_BF16 && qk_dtype != FA_E4M3) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (qk_dtype == FA_E4M3 && d == 64) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return FA_ERR_ALIGNMENT;
+  if (qk_dtype == FA_E4M3) {
+    if (descale_qk == nullptr) return FA_ERR_INVALID_ARG;
+    if (!aligned(descale_qk, 4)) return FA_ERR_ALIGNMENT;
+  }
+  const long long rows_per_cta = 128;  // the smallest query block of any kernel
+  const long long n_qb = (static_cast<long long>(Nq) + rows_per_cta - 1) / rows_per_cta;
+  if (n_qb * n_split * B * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * Nk > (1LL << 40)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// Bytes of the split-key workspace: the fp32 partial outputs, then (256-byte
+// aligned) the partial LSEs.
+size_t part_o_bytes(int B, int H, int Nq, int d, int n_split) {
+  return static_cast<size_t>(n_split) * B * H * Nq * d * sizeof(float);
+}
+size_t part_bytes(int B, int H, int Nq, int d, int n_split) {
+  const size_t o = (part_o_bytes(B, H, Nq, d, n_split) + 255) & ~static_cast<size_t>(255);
+  return o + static_cast<size_t>(n_split) * B * H * Nq * sizeof(float);
+}
+
+int device_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) return 148;
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
+// Split count for a launch of `units` CTAs per split over `tiles` key tiles,
+// one CTA per SM: the count with the fewest key-tile steps on the busiest SM,
+// counting two steps of fixed cost per CTA (prologue, epilogue and the partial
+// output) and the merge as one more when splitting; ties go to fewer splits.
+int pick_splits(long long units, int tiles, int sms) {
+  if (units >= sms || tiles <= 2) return 1;
+  long long best_cost = -1;
+  int best = 1;
+  const int max_split = tiles < 128 ? tiles : 128;
+  for (int ns = 1; ns <= max_split; ++ns) {
+    const long long waves = (units * ns + sms - 1) / sms;
+    const long long per_cta = (tiles + ns - 1) / ns + 2;
+    const long long cost = waves * per_cta + (ns > 1 ? 1 : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  return best;
+}
+
+int auto_splits(int B, int H, int Nq, int Nk, int d) {
+  const int nq = nq_for(d, Nq);
+  const long long units = static_cast<long long>(B) * H * ((Nq + nq * 128 - 1) / (nq * 128));
+  return pick_splits(units, key_tiles(Nk), device_sms());
 }
 
 template <int D>
@@ -136,46 +259,101 @@ fa_status launch_quant_fused(const void* x, void* out, float* descale_out, int64
   return FA_OK;
 }
 
+template <int D>
+fa_status launch_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, void* o, float* lse,
+                       cudaStream_t stream) {
+  const int64_t warps_per_block = fa::kMergeThreads / 32;
+  int64_t blocks = (rows + warps_per_block - 1) / warps_per_block;
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  fa::lse_merge_kernel<D><<<static_cast<unsigned>(blocks), fa::kMergeThreads, 0, stream>>>(
+      o_part, lse_part, n_part, rows, static_cast<__nv_bfloat16*>(o), lse);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status dispatch_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
+                         float* lse, cudaStream_t s) {
+  switch (d) {
+    case 64: return launch_merge<64>(o_part, lse_part, n_part, rows, o, lse, s);
+    case 128: return launch_merge<128>(o_part, lse_part, n_part, rows, o, lse, s);
+    default: return launch_merge<256>(o_part, lse_part, n_part, rows, o, lse, s);
+  }
+}
+
 }  // namespace
 
 extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  int causal, float scale, fa_dtype qk_dtype, const float* descale_qk, void* stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (qk_dtype != FA_BF16 && qk_dtype != FA_E4M3) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  if (qk_dtype == FA_E4M3 && d == 64) return FA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return FA_ERR_ALIGNMENT;
+  const fa_status chk = check_fwd_args(q, k, v, B, H, N, N, d, causal, scale, qk_dtype, descale_qk, 1);
+  if (chk != FA_OK) return chk;
+  if (o == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16)) return FA_ERR_ALIGNMENT;
   if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
-  if (qk_dtype == FA_E4M3) {
-    if (descale_qk == nullptr) return FA_ERR_INVALID_ARG;
-    if (!aligned(descale_qk, 4)) return FA_ERR_ALIGNMENT;
-  }
-  const int rows_per_cta = 128;  // the smallest query block of any kernel
-  const long long n_qb = (static_cast<long long>(N) + rows_per_cta - 1) / rows_per_cta;
-  if (n_qb * B * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  FwdArgs a{q, k, v, o, lse, nullptr, nullptr, B, H, N, N, d, causal != 0, scale, qk_dtype, descale_qk, 1};
+  return dispatch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return 1;
+  return auto_splits(B, H, Nq, Nk, d);
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || n_split < 0) return 0;
+  if (n_split == 0) n_split = auto_splits(B, H, Nq, Nk, d);
+  return n_split <= 1 ? 0 : part_bytes(B, H, Nq, d, n_split);
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                         int Nk, int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk,
+                         int n_split, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_split < 0 || B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (n_split == 0) n_split = auto_splits(B, H, Nq, Nk, d);
+  const fa_status chk = check_fwd_args(q, k, v, B, H, Nq, Nk, d, causal, scale, qk_dtype, descale_qk, n_split);
+  if (chk != FA_OK) return chk;
+  if (o == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16)) return FA_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool c = causal != 0;
-  if (qk_dtype == FA_BF16) {
-    switch (d) {
-      case 64: return c ? launch_fwd<64, 2, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
-                        : launch_fwd<64, 2, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
-      case 128: return c ? launch_fwd<128, 2, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
-                         : launch_fwd<128, 2, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
-      default: return c ? launch_fwd<256, 1, true, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s)
-                        : launch_fwd<256, 1, false, false>(q, k, v, o, lse, B, H, N, scale, nullptr, s);
-    }
+  if (n_split == 1) {
+    FwdArgs a{q, k, v, o, lse, nullptr, nullptr, B, H, Nq, Nk, d, causal != 0, scale, qk_dtype, descale_qk, 1};
+    return dispatch_fwd(a, s);
   }
-  switch (d) {
-    case 128: return c ? launch_fwd<128, 2, true, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s)
-                       : launch_fwd<128, 2, false, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s);
-    default: return c ? launch_fwd<256, 1, true, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s)
-                      : launch_fwd<256, 1, false, true>(q, k, v, o, lse, B, H, N, scale, descale_qk, s);
-  }
+  if (workspace == nullptr || workspace_bytes < part_bytes(B, H, Nq, d, n_split)) return FA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return FA_ERR_ALIGNMENT;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             ((part_o_bytes(B, H, Nq, d, n_split) + 255) & ~static_cast<size_t>(255)));
+  FwdArgs a{q, k, v, nullptr, nullptr, o_part, lse_part, B, H, Nq, Nk, d, causal != 0, scale, qk_dtype, descale_qk,
+            n_split};
+  const fa_status r = dispatch_fwd(a, s);
+  if (r != FA_OK) return r;
+  return dispatch_merge(o_part, lse_part, n_split, static_cast<int64_t>(B) * H * Nq, d, o, lse, s);
+}
+
+fa_status fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int H,
+                         int Nq, int Nk, int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk,
+                         int n_split, void* stream) {
+  const fa_status chk = check_fwd_args(q, k, v, B, H, Nq, Nk, d, causal, scale, qk_dtype, descale_qk, n_split);
+  if (chk != FA_OK) return chk;
+  if (o_part == nullptr || lse_part == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned(o_part, 16) || !aligned(lse_part, 4)) return FA_ERR_ALIGNMENT;
+  FwdArgs a{q, k, v, nullptr, nullptr, o_part, lse_part, B, H, Nq, Nk, d, causal != 0, scale, qk_dtype, descale_qk,
+            n_split};
+  return dispatch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
+                       float* lse, void* stream) {
+  if (o_part == nullptr || lse_part == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
+  if (n_part < 1 || rows < 1 || rows > (static_cast<int64_t>(1) << 40)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned(o_part, 16) || !aligned(lse_part, 4) || !aligned(o, 16)) return FA_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  return dispatch_merge(o_part, lse_part, n_part, rows, d, o, lse, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_t rows, int d, int rotate,
@@ -294,6 +472,6 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
   return FA_OK;
 }
 
-int fa_abi_version(void) { return 1; }
+int fa_abi_version(void) { return 2; }
 
 }  // extern "C"

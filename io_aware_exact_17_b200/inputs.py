@@ -8,6 +8,9 @@ Recipe (all on the CPU, ``torch.Generator`` seeded, then moved as needed):
 
 * Q, K, V: fp32 standard normal, drawn in that order from one generator, cast to
   bf16 (round to nearest even). Layout ``[B, H, N, d]``.
+* Decode-shaped problems (few queries, long keys): Q ``[B, H, Nq, d]`` then K and
+  V ``[B, H, Nk, d]``, fp32 standard normal drawn in that order from one
+  generator, cast to bf16.
 * Outliers, reading R1 (default): per head one feature channel, chosen from the
   seed, multiplied by 20 in both Q and K for every token (0.1% of 128 channels
   rounds up to one channel per head).
@@ -40,6 +43,16 @@ def qkv_normal(B: int, H: int, N: int, d: int, seed: int, dtype=torch.bfloat16):
     q = torch.randn(shape, generator=g, dtype=torch.float32).to(dtype)
     k = torch.randn(shape, generator=g, dtype=torch.float32).to(dtype)
     v = torch.randn(shape, generator=g, dtype=torch.float32).to(dtype)
+    return q, k, v
+
+
+def qkv_decode(B: int, H: int, Nq: int, Nk: int, d: int, seed: int, dtype=torch.bfloat16):
+    """Q ``[B, H, Nq, d]``, then K and V ``[B, H, Nk, d]``, all N(0, 1) i.i.d.,
+    drawn in that order; CPU tensors."""
+    g = _gen(seed)
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32).to(dtype)
+    k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32).to(dtype)
+    v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32).to(dtype)
     return q, k, v
 
 
@@ -119,7 +132,8 @@ class Workload:
 
 
 def workloads():
-    """The five workload families, seeds 1000 + family index."""
+    """The five workload families, seeds 1000 + family index. (The decode-shaped
+    problems, family 5, are not square and use :func:`qkv_decode`.)"""
     w = []
     for causal in (False, True):
         w.append(Workload(f"tiny_b1h2n128d64_{'c' if causal else 'nc'}", 1, 2, 128, 64, causal, 1000))

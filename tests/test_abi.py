@@ -28,7 +28,9 @@ def test_every_declared_symbol_is_exported(lib):
     assert {"fa_fwd", "fa_hadamard_quant", "fa_status_string", "fa_device_status", "fa_abi_version"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.fa_abi_version() == 1
+    assert {"fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_splits", "fa_fwd_partial",
+            "fa_lse_merge"} <= set(names)
+    assert lib.fa_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -84,6 +86,52 @@ def test_quant_argument_errors(lib):
     assert _quant(lib, ws=A + 4) == binding.FA_ERR_ALIGNMENT
 
 
+def _skv(lib, q=A, k=A, v=A, o=A, lse=None, B=1, H=1, Nq=1, Nk=300, d=128, causal=0, scale=0.1, dtype=0, desc=None,
+         ns=1, ws=None, wsb=0):
+    return lib.fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, dtype, desc, ns, ws, wsb, None)
+
+
+def test_splitkv_argument_errors(lib):
+    assert _skv(lib, q=None) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, o=None) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, Nq=0) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, Nk=0) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, ns=-1) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, Nq=301, causal=1) == binding.FA_ERR_INVALID_ARG  # a query would see no key
+    assert _skv(lib, scale=-1.0) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, d=32) == binding.FA_ERR_UNSUPPORTED
+    assert _skv(lib, k=MIS) == binding.FA_ERR_ALIGNMENT
+    assert _skv(lib, o=MIS) == binding.FA_ERR_ALIGNMENT
+    # a split needs a workspace of the stated size, 256-byte aligned
+    need = lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 300, 128, 3)
+    assert need >= 3 * 128 * 4 + 3 * 4
+    assert _skv(lib, ns=3) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, ns=3, ws=A, wsb=need - 1) == binding.FA_ERR_INVALID_ARG
+    assert _skv(lib, ns=3, ws=A + 16, wsb=need) == binding.FA_ERR_ALIGNMENT
+    assert lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1, 300, 128, 1) == 0
+    assert lib.fa_fwd_splitkv_workspace_bytes(0, 1, 1, 300, 128, 2) == 0
+
+
+def test_partial_and_merge_argument_errors(lib):
+    part = lambda **kw: lib.fa_fwd_partial(kw.get("q", A), A, A, kw.get("op", A), kw.get("lp", A), 1, 1, 4, 64, 128,
+                                           kw.get("causal", 0), 0.1, 0, None, kw.get("ns", 1), None)
+    assert part(q=None) == binding.FA_ERR_INVALID_ARG
+    assert part(op=None) == binding.FA_ERR_INVALID_ARG
+    assert part(lp=None) == binding.FA_ERR_INVALID_ARG
+    assert part(ns=0) == binding.FA_ERR_INVALID_ARG
+    assert part(op=MIS) == binding.FA_ERR_ALIGNMENT
+    assert part(lp=A + 2) == binding.FA_ERR_ALIGNMENT
+    merge = lambda **kw: lib.fa_lse_merge(kw.get("op", A), kw.get("lp", A), kw.get("n", 2), kw.get("rows", 8),
+                                          kw.get("d", 128), kw.get("o", A), None, None)
+    assert merge(op=None) == binding.FA_ERR_INVALID_ARG
+    assert merge(o=None) == binding.FA_ERR_INVALID_ARG
+    assert merge(n=0) == binding.FA_ERR_INVALID_ARG
+    assert merge(rows=0) == binding.FA_ERR_INVALID_ARG
+    assert merge(d=80) == binding.FA_ERR_UNSUPPORTED
+    assert merge(op=MIS) == binding.FA_ERR_ALIGNMENT
+    assert merge(o=MIS) == binding.FA_ERR_ALIGNMENT
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
 
@@ -92,3 +140,9 @@ def test_python_binding_rejects_cpu_tensors():
         binding.fwd(q, q, q)
     with pytest.raises(binding.FaError):
         binding.hadamard_quant(q)
+    with pytest.raises(binding.FaError):
+        binding.fwd_splitkv(q, q, q)
+    with pytest.raises(binding.FaError):
+        binding.fwd_partial(q, q, q)
+    with pytest.raises(binding.FaError):
+        binding.lse_merge(q.float(), q.float()[..., 0])
