@@ -12,6 +12,12 @@ would otherwise stay resident.
 ``--impl reference`` times the CPU oracle instead (rank 0 only), on a bounded
 row sample of the same workload per step.
 
+``--workload decode`` measures the decode-shaped problem instead: B=4, H=16
+single-query heads (Nq=1) over Nk=32768 keys, d=128, bf16: one step is the
+split-key attention kernel (fp32 partial results per block of keys) and the LSE
+merge. It is HBM-bound (the 1.07 GB of K and V are read once per step), so its
+metric is GB/s of algorithmic traffic.
+
 Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
 torch.distributed.run, one rank per GPU, each rank its own batch: weak scaling,
 no collective on the data path).
@@ -37,6 +43,8 @@ import torch  # noqa: E402
 from io_aware_exact_17_b200 import inputs as fa_inputs  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (4·B·H·N²·d, ½ if causal) and % of B200 BF16/FP8 peak"
+DECODE = {"B": 4, "H": 16, "Nq": 1, "Nk": 32768, "d": 128, "seed": 1005}
+DECODE_METRIC = "decode attention GB/s (algorithmic HBM bytes: K, V, Q read; O, LSE written)"
 B, H, N, D = 4, 16, 2048, 128
 SEED = 1001
 WORKLOAD = f"b{B}h{H}n{N}d{D}: bf16 fwd non-causal + bf16 fwd causal + rotate/quantise Q,K + e4m3-QK fwd non-causal"
@@ -130,22 +138,58 @@ def dist_done(world: int):
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clocks and throttle reasons sampled while the timed region runs: NVML
+    every 5 ms from a thread (a timed region can be a few tens of ms), else
+    nvidia-smi every 200 ms. Reads only; changes no setting."""
 
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        # nvidia-smi numbers GPUs physically; address ours by UUID instead.
+        # nvidia-smi and NVML number GPUs physically; address ours by UUID instead.
         try:
             uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
             self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
             self.gpu = str(gpu_index)
         self.proc = None
+        self.thread = None
+        self.samples = []  # (sm_mhz, max_mhz, reasons bitmask)
+        self.lines = []
+
+    def _nvml_loop(self, handle, nv):
+        import time as _t
+
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            _t.sleep(0.005)
 
     def __enter__(self):
+        self.stop = False
+        try:
+            import threading
+
+            import pynvml as nv
+
+            nv.nvmlInit()
+            try:
+                handle = nv.nvmlDeviceGetHandleByUUID(self.gpu)
+            except Exception:
+                handle = nv.nvmlDeviceGetHandleByUUID(self.gpu.encode())
+            self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -155,7 +199,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -168,6 +214,10 @@ class ClockSampler:
 
     def summary(self):
         sm, smax, reasons = [], None, set()
+        for mhz, mx, bits in self.samples:
+            sm.append(mhz)
+            smax = mx
+            reasons.update(nm for nm, b in self.REASON_BITS.items() if bits & b)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
@@ -182,7 +232,8 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvml 5 ms" if self.samples else ("nvidia-smi 200 ms" if self.lines else None)}
 
 
 # --------------------------------------------------------------- GPU step --
@@ -208,6 +259,7 @@ class Step:
         self.lse_h = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(3)]
         self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         self.launches_per_step = 5  # 3 attention kernels + 2 one-launch quantisations
+        self.groups = 4  # breakdown: bf16 nc, bf16 causal, quantise Q+K, e4m3 nc
 
     def flush_l2(self):
         self.flush_buf.zero_()
@@ -251,7 +303,69 @@ class Step:
         return sum(t.numel() * t.element_size() for t in self.o_h + self.lse_h)
 
 
-def capture_step(step: Step):
+class DecodeStep:
+    """The decode-shaped problem: fp32 partial results per block of keys
+    (fwd_partial) then the LSE merge (lse_merge), the two kernels fwd_splitkv
+    runs, called separately so each is timed. The K/V cache stays on the device
+    between steps, as a decode step's cache does."""
+
+    def __init__(self, seed: int):
+        import io_aware_exact_17_b200 as fa
+
+        self.fa = fa
+        c = DECODE
+        self.B, self.H, self.Nq, self.Nk, self.d = c["B"], c["H"], c["Nq"], c["Nk"], c["d"]
+        q, k, v = fa_inputs.qkv_decode(self.B, self.H, self.Nq, self.Nk, self.d, seed)
+        self.q_h = q.pin_memory()
+        self.q, self.k, self.v = (t.cuda() for t in (q, k, v))
+        self.n_split = fa.splitkv_splits(self.B, self.H, self.Nq, self.Nk, self.d)
+        rows = (self.B, self.H, self.Nq)
+        self.o_part = torch.empty((self.n_split, *rows, self.d), dtype=torch.float32, device="cuda")
+        self.lse_part = torch.empty((self.n_split, *rows), dtype=torch.float32, device="cuda")
+        self.o = torch.empty((*rows, self.d), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty(rows, dtype=torch.float32, device="cuda")
+        self.o_h = torch.empty((*rows, self.d), dtype=torch.bfloat16).pin_memory()
+        self.lse_h = torch.empty(rows, dtype=torch.float32).pin_memory()
+        self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 2
+        self.groups = 2  # breakdown: split-key attention, merge
+        n = self.B * self.H
+        # algorithmic bytes: K, V (bf16) and Q read; O (bf16) and LSE written
+        self.kv_bytes = 2.0 * n * self.Nk * self.d * 2
+        self.bytes = self.kv_bytes + n * self.Nq * self.d * 2 * 2 + n * self.Nq * 4
+        self.part_bytes = self.o_part.numel() * 4 + self.lse_part.numel() * 4
+
+    def flush_l2(self):
+        self.flush_buf.zero_()
+
+    def run(self, ev=None):
+        fa = self.fa
+        if ev is not None:
+            ev[0].record()
+        fa.fwd_partial(self.q, self.k, self.v, n_split=self.n_split, o_part=self.o_part, lse_part=self.lse_part)
+        if ev is not None:
+            ev[1].record()
+        fa.lse_merge(self.o_part, self.lse_part, out=self.o, lse=self.lse)
+        if ev is not None:
+            ev[2].record()
+
+    def run_e2e(self):
+        """Q copied in from pinned host memory, the step, O and LSE copied out."""
+        self.q.copy_(self.q_h, non_blocking=True)
+        self.run()
+        self.o_h.copy_(self.o, non_blocking=True)
+        self.lse_h.copy_(self.lse, non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return self.q_h.numel() * self.q_h.element_size()
+
+    @property
+    def d2h_bytes(self):
+        return self.o_h.numel() * 2 + self.lse_h.numel() * 4
+
+
+def capture_step(step):
     """The step's kernels captured once as a CUDA graph, so a timed step carries
     no host launch overhead (the quantiser kernels are ~10 us each)."""
     s = torch.cuda.Stream()
@@ -267,7 +381,7 @@ def capture_step(step: Step):
     return g
 
 
-def time_steps(step: Step, graph, steps: int, warmup: int, world: int):
+def time_steps(step, graph, steps: int, warmup: int, world: int):
     """K timed steps (graph replays, L2 flushed between them outside the events),
     then K eager steps with events around each kernel group for the breakdown."""
     for _ in range(warmup):
@@ -285,16 +399,16 @@ def time_steps(step: Step, graph, steps: int, warmup: int, world: int):
     torch.cuda.synchronize()
     dist_barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(step.groups + 1)] for _ in range(steps)]
     for i in range(steps):
         step.flush_l2()
         step.run(evs[i])
     torch.cuda.synchronize()
-    per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)]
-    return step_ms, per  # per: ms [bf16 nc, bf16 causal, quant Q+K, fp8 nc] per eager step
+    per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(step.groups)] for i in range(steps)]
+    return step_ms, per  # per: ms of each kernel group per eager step
 
 
-def time_e2e(step: Step, steps: int, warmup: int, world: int):
+def time_e2e(step, steps: int, warmup: int, world: int):
     for _ in range(warmup):
         step.run_e2e()
     torch.cuda.synchronize()
@@ -352,6 +466,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", choices=["step", "decode"], default="step")
     args = ap.parse_args()
     world, rank, local = dist_setup()
 
@@ -381,6 +496,9 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device for --impl ours")
     torch.cuda.set_device(local)
+    if args.workload == "decode":
+        run_decode(args, world, rank)
+        return
     step = Step(SEED + rank)
     graph = capture_step(step)
     with ClockSampler(local) as clk:
@@ -419,13 +537,55 @@ def main():
                     "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},
             "gpu_launches": step.launches_per_step * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                       "reasons": clocks["reasons"]},
+                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
         }
         if not args.no_cpu_baseline and world == 1:
             fl, sec, cores, rows_n = oracle_sample(args.cpu_seconds, SEED)
             line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                                     "sample": f"{rows_n} random query rows x 3 attention passes of the workload, "
                                               f"exact fp64, {sec:.1f} s"}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+def run_decode(args, world: int, rank: int):
+    step = DecodeStep(DECODE["seed"] + rank)
+    graph = capture_step(step)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
+    e2e_ms = dist_max(time_e2e(step, max(3, args.steps // 4), 3, world), world)
+    ms = dist_max(statistics.mean(step_ms), world)
+    comp = [dist_max(statistics.mean(p[j] for p in per), world) for j in range(2)]
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    if rank == 0:
+        # the dominant kernel's algorithmic bytes: K, V, Q read and the partial
+        # results written
+        attn_bytes = step.kv_bytes + step.q_h.numel() * 2 + step.part_bytes
+        achieved = attn_bytes / (comp[0] * 1e-3) / 1e9
+        c = DECODE
+        line = {
+            "metric": DECODE_METRIC, "value": world * step.bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16)",
+            "config": {"workload": f"decode b{c['B']}h{c['H']} nq{c['Nq']} nk{c['Nk']} d{c['d']}: split-key attention "
+                                   f"({step.n_split} blocks) + LSE merge", **{k: c[k] for k in ("B", "H", "Nq", "Nk", "d")},
+                       "n_split": step.n_split, "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (512 MB write outside the timed events); K+V 1.07 GB > L2"},
+            "timing": "value: CUDA-graph replay of the step; breakdown: eager calls, events per kernel",
+            "breakdown_ms": {"splitkv_attention": comp[0], "lse_merge": comp[1]},
+            "roofline": {"kernel": "attn_fwd_kernel<128,1,nc,bf16> (partial mode)", "bound": "hbm",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peak_src} HBM copy bandwidth"},
+            "e2e": {"value": world * step.bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
+                    "note": "K/V cache resident on the device; Q in, O and LSE out per step"},
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
+        }
         print(json.dumps(line), flush=True)
     dist_done(world)
 

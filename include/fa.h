@@ -85,7 +85,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  * B, H, Nq, Nk >= 1; causal requires Nq <= Nk. d, scale, qk_dtype, descale_qk: as fa_fwd.
  * n_split 1 = no split (no workspace; the same kernel as fa_fwd); >= 2 = that many
  *         blocks of ceil(ceil(Nk/128)/n_split) key tiles of 128 keys (the last ones
- *         may be empty); 0 = fa_fwd_splitkv_splits(B, H, Nq, Nk, d).
+ *         may be empty); 0 = automatic: with fewer query blocks (of 128 or 256
+ *         rows) than SMs, fa_fwd_splitkv_splits(B, H, Nq, Nk, d) blocks for every
+ *         query block, else no split.
  * workspace  device, >= fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split)
  *         bytes, 256-byte aligned, owned by the caller (may be NULL if that is 0);
  *         overwritten. Calls that overlap on the GPU must not share it.
@@ -97,7 +99,7 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
                          int n_split, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes of fa_fwd_splitkv for these sizes (n_split = 0: the automatic
- * count on the current device); 0 when no workspace is needed or on bad sizes. */
+ * schedule on the current device); 0 when no workspace is needed or on bad sizes. */
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split);
 
 /* The split count fa_fwd_splitkv uses for n_split = 0 on the current device: the

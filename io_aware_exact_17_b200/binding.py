@@ -96,13 +96,19 @@ def _require_cuda(*ts):
 
 
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=None, out=None, lse=None,
-        return_lse: bool = True):
-    """Attention forward through ``fa_fwd``.
+        return_lse: bool = True, n_split: int = 0):
+    """Attention forward of ``[B, H, N, d]`` inputs.
 
-    q, k: ``[B, H, N, d]`` bf16, or e4m3 codes (uint8 / float8_e4m3fn) with
-    ``qk_descale`` a CUDA fp32 tensor ``[dq, dk]``; v: bf16 ``[B, H, N, d]``.
-    Returns ``(O, LSE)``: bf16 ``[B, H, N, d]`` and fp32 ``[B, H, N]`` (natural log);
-    LSE is ``None`` when ``return_lse`` is false.
+    q, k: bf16, or e4m3 codes (uint8 / float8_e4m3fn) with ``qk_descale`` a
+    CUDA fp32 tensor ``[dq, dk]``; v: bf16. Returns ``(O, LSE)``: bf16
+    ``[B, H, N, d]`` and fp32 ``[B, H, N]`` (natural log); LSE is ``None`` when
+    ``return_lse`` is false.
+
+    ``n_split=0`` (default) runs ``fa_fwd_splitkv`` with its automatic
+    schedule, which splits the keys of some query blocks (all of them when
+    there are fewer blocks than SMs, else those of a mostly empty last wave)
+    and merges by LSE, with a workspace cached per device. ``n_split=1`` runs
+    ``fa_fwd``: one CTA per query block over all its keys, no workspace.
     """
     _require_cuda(q, k, v)
     lib = load_library()
@@ -116,6 +122,8 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
         raise FaError("v must be bf16")
     if fp8 and (qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2):
         raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk]")
+    if n_split not in (0, 1):
+        raise FaError("n_split must be 0 (automatic) or 1 (no split); use fwd_splitkv for a fixed split")
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
@@ -123,12 +131,38 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    desc = _ptr(qk_descale.contiguous()) if fp8 else None
+    dt = FA_E4M3 if fp8 else FA_BF16
     with torch.cuda.device(q.device):
-        rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, N, d,
-                        int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
-                        _ptr(qk_descale.contiguous()) if fp8 else None, _stream(q.device))
-    _check(rc, "fa_fwd")
+        if n_split == 1:
+            rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, N, d,
+                            int(bool(causal)), float(scale), dt, desc, _stream(q.device))
+            _check(rc, "fa_fwd")
+        else:
+            need = int(lib.fa_fwd_splitkv_workspace_bytes(B, H, N, N, d, 0))
+            ws = _split_workspace(q.device, need)
+            rc = lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H,
+                                    N, N, d, int(bool(causal)), float(scale), dt, desc, 0,
+                                    _ptr(ws) if need > 0 else None, need, _stream(q.device))
+            _check(rc, "fa_fwd_splitkv")
     return out, (lse if return_lse else None)
+
+
+_split_workspaces: dict[int, torch.Tensor] = {}
+
+
+def _split_workspace(device, nbytes: int):
+    """A device buffer of at least ``nbytes`` for the split schedules, cached per
+    device and grown when a call needs more (calls on one device share it, so
+    they must be ordered on one stream)."""
+    if nbytes <= 0:
+        return None
+    idx = torch.device(device).index
+    ws = _split_workspaces.get(idx)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _split_workspaces[idx] = ws
+    return ws
 
 
 def _qkv_kinds(q, k, v, qk_descale):

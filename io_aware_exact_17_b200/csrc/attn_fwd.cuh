@@ -96,6 +96,9 @@ struct FwdParams {
   int n_split;               // key splits per head (1: all keys)
   int split_tiles;           // key tiles per split
   float scale_log2;          // scale * log2(e)
+  // The grid covers the query blocks unit_base, unit_base + 1, ... (query block
+  // = bh * n_qb + qb), each with n_split CTAs in partial mode.
+  int unit_base;
 };
 
 // Bounded wait used only while tearing down after an abort: ignores the abort
@@ -217,7 +220,9 @@ __device__ __forceinline__ float row_max_tmem(uint32_t tS, uint32_t* s, int kbas
   return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
 }
 
-template <int D, int NQ, bool CAUSAL, bool QK_FP8>
+// PARTIAL: the CTA's keys are one block of a split (p.n_split blocks) and it
+// writes fp32 partial results (o_part, lse_part) instead of O and LSE.
+template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, QK_FP8>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -236,9 +241,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   // Work item: head bh, key split sp, query block qb (heaviest causal blocks of
   // a head first).
-  const int bh = blockIdx.x / (p.n_qb * p.n_split);
-  const int sp = (blockIdx.x / p.n_qb) % p.n_split;
-  int qb = blockIdx.x % p.n_qb;
+  const int n_split = PARTIAL ? p.n_split : 1;
+  const int unit_rel = PARTIAL ? static_cast<int>(blockIdx.x) / n_split : static_cast<int>(blockIdx.x);
+  const int sp = PARTIAL ? static_cast<int>(blockIdx.x) % n_split : 0;
+  const int unit = p.unit_base + unit_rel;  // query block bh * n_qb + qb
+  const int bh = unit / p.n_qb;
+  int qb = unit % p.n_qb;
   if (CAUSAL) qb = p.n_qb - 1 - qb;
   const int q0 = qb * NQ * C::BM;
   // Key tiles of this split: kt0 .. kt0 + split_tiles - 1 (clipped to Nk). Query
@@ -246,13 +254,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // else up to the tile holding its last visible key, so a causal tile never
   // spends a step on keys entirely in its future. The CTA streams the most any
   // tile needs.
-  const int kt0 = sp * p.split_tiles;
+  const int kt0 = PARTIAL ? sp * p.split_tiles : 0;
   auto n_kv_of = [&](int t) {
     const int row0 = q0 + t * C::BM;
     if (row0 >= p.Nq) return 0;
     const int end = CAUSAL ? min(p.Nk, min(p.Nq, row0 + C::BM) + p.causal_off) : p.Nk;  // keys [0, end)
-    const int tiles = min((end + C::BN - 1) / C::BN, kt0 + p.split_tiles);
-    return max(0, tiles - kt0);
+    const int tiles = (end + C::BN - 1) / C::BN;
+    if (!PARTIAL) return tiles;
+    return max(0, min(tiles, kt0 + p.split_tiles) - kt0);
   };
   const int n_kv0 = n_kv_of(0);
   const int n_kv1 = NQ > 1 ? n_kv_of(NQ - 1) : n_kv0;
@@ -412,18 +421,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const bool masked = __any_sync(0xffffffffu, kbase + C::BN - 1 > kmax);
       float sum_e, sum_r, alpha = 1.0f, mx = 0.f;
       if (j == 0) {
-        // -inf only for a row that sees no key of this split (partial mode): its
-        // weights are then exp2(-inf - 0) = 0 throughout.
+        // A row that sees no key of this split (partial mode only) has max -inf;
+        // it takes reference 0, so its weights are exp2(-inf) = 0 throughout and
+        // it is recognised at the end by its zero sum.
         m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;
-        softmax_row_dispatch<false>(tS, s, s_log2, m_ref == -INFINITY ? 0.f : m_ref, kbase, kmax, masked, sum_e,
-                                    sum_r, mx);
+        if (PARTIAL && m_ref == -INFINITY) m_ref = 0.f;
+        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
       } else {
         // Exponentials against the current reference, taking the row's max on the
         // way; only if some row's max grew by more than 2^8 (rare after the first
         // tiles) is the row redone against the new reference. S is still intact:
         // P is written only below.
-        softmax_row_dispatch<true>(tS, s, s_log2, m_ref == -INFINITY ? 0.f : m_ref, kbase, kmax, masked, sum_e,
-                                   sum_r, mx);
+        softmax_row_dispatch<true>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
         const float mx_s = mx * s_log2;
         const bool grow = mx_s > m_ref + 8.0f;
         if (__any_sync(0xffffffffu, grow)) {
@@ -456,34 +465,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (ok && n_kv_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
     const bool in_range = qrow < p.Nq;
-    if (ok && p.o_part != nullptr) {
-      // Partial mode: O of this split's keys in fp32 (normalised by its own
-      // weights) and its LSE; a row with no key of the split gets 0 and -inf.
-      const bool empty = l_exact == 0.f;
-      const size_t prow = (static_cast<size_t>(sp) * p.BH + bh) * p.Nq + (in_range ? qrow : 0);
-      float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
-      if (n_kv_t > 0) tc_fence_after();
-      const float inv_l = empty ? 0.f : 1.0f / l_round;
+    if constexpr (PARTIAL) {
+      if (ok) {
+        // O of this split's keys in fp32 (normalised by its own weights) and its
+        // LSE; a row with no key of the split gets 0 and -inf.
+        const bool empty = l_exact == 0.f;
+        const size_t prow = (static_cast<size_t>(sp) * p.BH + bh) * p.Nq + (in_range ? qrow : 0);
+        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+        if (n_kv_t > 0) tc_fence_after();
+        const float inv_l = empty ? 0.f : 1.0f / l_round;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t ov[32];
-        if (n_kv_t > 0) {
-          tmem_ld32(tO + c0, ov);
-          tmem_wait_ld_dep32(ov);
-        } else {
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          if (n_kv_t > 0) {
+            tmem_ld32(tO + c0, ov);
+            tmem_wait_ld_dep32(ov);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0u;
-        }
-        if (in_range) {
+            for (int i = 0; i < 32; ++i) ov[i] = 0u;
+          }
+          if (in_range) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[c0 / 4 + i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
-                                          __uint_as_float(ov[4 * i + 2]) * inv_l,
-                                          __uint_as_float(ov[4 * i + 3]) * inv_l);
+            for (int i = 0; i < 8; ++i)
+              dst[c0 / 4 + i] = make_float4(
+                  __uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
+                  __uint_as_float(ov[4 * i + 2]) * inv_l, __uint_as_float(ov[4 * i + 3]) * inv_l);
+          }
         }
+        if (in_range)
+          p.lse_part[prow] = empty ? -INFINITY : (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
       }
-      if (in_range)
-        p.lse_part[prow] = empty ? -INFINITY : (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     } else if (ok && n_kv_t > 0) {
       tc_fence_after();
       const float inv_l = 1.0f / l_round;

@@ -47,6 +47,8 @@ struct FwdArgs {
   fa_dtype qk_dtype;
   const float* descale_qk;
   int n_split;
+  int unit_base = 0;  // first query block of the launch (bh * n_qb + qb)
+  int n_units = 0;    // query blocks in the launch (0: all)
 };
 
 constexpr int kKeyTile = 128;  // keys per K/V tile (FwdCfg::BN)
@@ -57,7 +59,7 @@ inline int key_tiles(int Nk) { return (Nk + kKeyTile - 1) / kKeyTile; }
 // one tile of queries; one for d = 256 (TMEM) and for short query blocks.
 inline int nq_for(int d, int Nq) { return (d <= 128 && Nq > 128) ? 2 : 1; }
 
-template <int D, int NQ, bool CAUSAL, bool QK_FP8>
+template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL>
 fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D, NQ, QK_FP8>;
   const int BH = a.B * a.H;
@@ -67,7 +69,7 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
       !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
       !fa::make_tmap_3d(&tmV, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nk, BH, 64, C::BN))
     return FA_ERR_CUDA;
-  auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8>;
+  auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8, PARTIAL>;
   static unsigned long long smem_done = 0;
   if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
   if constexpr (C::SPLIT_REGS) {
@@ -98,14 +100,19 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   p.n_split = a.n_split;
   p.split_tiles = (key_tiles(a.Nk) + a.n_split - 1) / a.n_split;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  const long long grid = static_cast<long long>(p.n_qb) * a.n_split * BH;
+  p.unit_base = a.unit_base;
+  const long long units = a.n_units > 0 ? a.n_units : static_cast<long long>(p.n_qb) * BH;
+  const long long grid = units * (PARTIAL ? a.n_split : 1);
+  if (grid < 1) return FA_OK;
   kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, int NQ, bool QK_FP8>
 fa_status launch_fwd_c(const FwdArgs& a, cudaStream_t s) {
-  return a.causal ? launch_fwd<D, NQ, true, QK_FP8>(a, s) : launch_fwd<D, NQ, false, QK_FP8>(a, s);
+  if (a.o_part != nullptr)
+    return a.causal ? launch_fwd<D, NQ, true, QK_FP8, true>(a, s) : launch_fwd<D, NQ, false, QK_FP8, true>(a, s);
+  return a.causal ? launch_fwd<D, NQ, true, QK_FP8, false>(a, s) : launch_fwd<D, NQ, false, QK_FP8, false>(a, s);
 }
 
 // Kernel choice by head dimension, dtype and query length.
@@ -193,6 +200,33 @@ int auto_splits(int B, int H, int Nq, int Nk, int d) {
   const int nq = nq_for(d, Nq);
   const long long units = static_cast<long long>(B) * H * ((Nq + nq * 128 - 1) / (nq * 128));
   return pick_splits(units, key_tiles(Nk), device_sms());
+}
+
+// The automatic schedule of fa_fwd_splitkv (n_split = 0): with fewer query
+// blocks than SMs, every block's keys are split (auto_splits) and merged; else one
+// CTA per query block. (Measured on B200 and dropped: splitting only the blocks
+// of a mostly empty last wave, either by keys with the merge in the kernel or as
+// one-tile CTAs, was slower than leaving that wave as it is: the split CTAs' fp32
+// partial stores and merge, or the one-tile CTAs' unhidden softmax, cost as much
+// as the wave they save.)
+struct Plan {
+  int n_split = 1;
+  int nq = 1;
+  long long units = 0;
+};
+
+Plan plan_fwd(int B, int H, int Nq, int Nk, int d, bool causal) {
+  (void)causal;
+  Plan pl;
+  pl.nq = nq_for(d, Nq);
+  pl.units = static_cast<long long>(B) * H * ((Nq + pl.nq * 128 - 1) / (pl.nq * 128));
+  const int sms = device_sms();
+  if (pl.units < sms) pl.n_split = pick_splits(pl.units, key_tiles(Nk), sms);
+  return pl;
+}
+
+size_t plan_bytes(const Plan& pl, int B, int H, int Nq, int d) {
+  return pl.n_split <= 1 ? 0 : part_bytes(B, H, Nq, d, pl.n_split);
 }
 
 template <int D>
@@ -303,7 +337,13 @@ int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d) {
 
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split) {
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || n_split < 0) return 0;
-  if (n_split == 0) n_split = auto_splits(B, H, Nq, Nk, d);
+  if (d != 64 && d != 128 && d != 256) return 0;
+  if (n_split == 0) {
+    // enough for the automatic schedule with either mask
+    const size_t a = plan_bytes(plan_fwd(B, H, Nq, Nk, d, false), B, H, Nq, d);
+    const size_t c = plan_bytes(plan_fwd(B, H, Nq, Nk, d, true), B, H, Nq, d);
+    return a > c ? a : c;
+  }
   return n_split <= 1 ? 0 : part_bytes(B, H, Nq, d, n_split);
 }
 
@@ -311,7 +351,12 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
                          int Nk, int d, int causal, float scale, fa_dtype qk_dtype, const float* descale_qk,
                          int n_split, void* workspace, size_t workspace_bytes, void* stream) {
   if (n_split < 0 || B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
-  if (n_split == 0) n_split = auto_splits(B, H, Nq, Nk, d);
+  Plan pl;
+  if (n_split == 0 && d >= 64 && d <= 256) {
+    pl = plan_fwd(B, H, Nq, Nk, d, causal != 0);
+    n_split = pl.n_split;
+  }
+  if (n_split == 0) n_split = 1;
   const fa_status chk = check_fwd_args(q, k, v, B, H, Nq, Nk, d, causal, scale, qk_dtype, descale_qk, n_split);
   if (chk != FA_OK) return chk;
   if (o == nullptr) return FA_ERR_INVALID_ARG;

@@ -14,18 +14,18 @@ from helpers import BF16_LSE_ATOL, BF16_O_ATOL, bf16_out_tol, max_abs, record, t
 pytestmark = pytest.mark.gpu
 
 
-def _run(q, k, v, causal, scale=None):
-    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+def _run(q, k, v, causal, scale=None, n_split=0):
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale, n_split=n_split)
     torch.cuda.synchronize()
     code, site, block = fa.device_status()
     assert code == 0, f"device wait ran out at site {site}, block {block}"
     return o, lse
 
 
-def _check_full(B, H, N, d, causal, seed):
+def _check_full(B, H, N, d, causal, seed, n_split=0):
     q, k, v = inputs.qkv_normal(B, H, N, d, seed)
     scale = d ** -0.5
-    o, lse = _run(q, k, v, causal)
+    o, lse = _run(q, k, v, causal, n_split=n_split)
     o_ref, lse_ref = oracle.attention(q, k, v, causal, scale)
     eo, el = max_abs(to_np(o), o_ref), max_abs(to_np(lse), lse_ref)
     record(f"bf16 B{B} H{H} N{N} d{d} {'causal' if causal else 'non-causal'}", o_max_abs=eo, lse_max_abs=el)
@@ -42,13 +42,29 @@ def test_tiny_config(causal):
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("N", [1, 17, 129, 200, 384, 700])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ragged_sizes(d, N, causal):
-    _check_full(2, 3, N, d, causal, 7 + N + d)
+@pytest.mark.parametrize("n_split", [0, 1])
+def test_ragged_sizes(d, N, causal, n_split):
+    # n_split 0: the automatic schedule (these few heads: keys split and merged);
+    # 1: one CTA per query block (fa_fwd)
+    _check_full(2, 3, N, d, causal, 7 + N + d, n_split)
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_b4_h16_n2048_d128_full(causal):
-    _check_full(4, 16, 2048, 128, causal, 1001)
+@pytest.mark.parametrize("n_split", [0, 1])
+def test_b4_h16_n2048_d128_full(causal, n_split):
+    _check_full(4, 16, 2048, 128, causal, 1001, n_split)
+
+
+def test_few_heads_long_sequence_split_keys():
+    # 2 heads x 8 two-tile query blocks = 16 CTAs on 148 SMs: the automatic
+    # schedule splits every block's keys and merges
+    B, H, N, d = 1, 2, 2048, 128
+    q, k, v = inputs.qkv_normal(B, H, N, d, 1010)
+    for causal in (False, True):
+        o, lse = _run(q, k, v, causal)
+        o_ref, lse_ref = oracle.attention(q, k, v, causal, d ** -0.5)
+        eo, el = max_abs(to_np(o), o_ref), max_abs(to_np(lse), lse_ref)
+        assert eo <= BF16_O_ATOL and el <= BF16_LSE_ATOL, (causal, eo, el)
 
 
 @pytest.mark.parametrize("n", [512, 1024, 2048, 4096, 8192, 16384])
@@ -149,14 +165,25 @@ def test_deterministic():
 
 
 def test_lse_optional_and_no_nxn_buffer():
-    # Linear memory: the call allocates nothing beyond O (and LSE when asked).
+    # Linear memory. One CTA per query block (n_split=1): nothing is allocated
+    # beyond O (and LSE when asked). The automatic schedule (these 128 query
+    # blocks are fewer than the SMs, so keys are split) adds a workspace of fp32
+    # partial outputs: O(N d) per head, far below one N x N matrix.
     B, H, N, d = 1, 8, 4096, 128
     q, k, v = (t.cuda() for t in inputs.qkv_normal(B, H, N, d, 37))
     o = torch.empty_like(q)
     torch.cuda.synchronize()
     before = torch.cuda.memory_allocated()
-    fa.fwd(q, k, v, causal=False, out=o, return_lse=False)
+    fa.fwd(q, k, v, causal=False, out=o, return_lse=False, n_split=1)
     torch.cuda.synchronize()
     assert torch.cuda.memory_allocated() == before
-    o2, _ = fa.fwd(q, k, v, causal=False)
+    o2, _ = fa.fwd(q, k, v, causal=False, n_split=1)
     assert torch.equal(o, o2)
+    o3 = torch.empty_like(q)
+    fa.fwd(q, k, v, causal=False, out=o3, return_lse=False)
+    torch.cuda.synchronize()
+    grown = torch.cuda.memory_allocated() - before
+    assert 0 < grown <= 8 * B * H * N * d * 4 < B * H * N * N * 4
+    o4, _ = fa.fwd(q, k, v, causal=False)
+    assert torch.equal(o3, o4)
+    assert max_abs(to_np(o3), to_np(o)) <= 2 * BF16_O_ATOL

@@ -111,7 +111,7 @@ def test_no_split_is_the_square_kernel_bitwise():
     q, k, v = inputs.qkv_normal(2, 3, 700, 128, 79)
     q, k, v = q.cuda(), k.cuda(), v.cuda()
     for causal in (False, True):
-        o1, l1 = fa.fwd(q, k, v, causal=causal)
+        o1, l1 = fa.fwd(q, k, v, causal=causal, n_split=1)
         o2, l2 = fa.fwd_splitkv(q, k, v, causal=causal, n_split=1)
         _status_ok()
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
