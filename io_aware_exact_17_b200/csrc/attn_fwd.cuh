@@ -220,13 +220,204 @@ __device__ __forceinline__ float row_max_tmem(uint32_t tS, uint32_t* s, int kbas
   return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
 }
 
+// Softmax warps of a DEC CTA (see attn_fwd_kernel): warp w, lane r holds query
+// row r's online softmax over keys 32w .. 32w+31 of each key tile (TMEM lane
+// 32w + r), then the four warps merge through shared memory.
+template <int D, bool CAUSAL, bool QK_FP8, bool PARTIAL, typename C, typename P>
+__device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint32_t warp, uint32_t lane, int q0, int bh,
+                                               int sp, int kt0, int n_kv, uint8_t* sbuf, uint64_t* bar_s,
+                                               uint64_t* bar_p, uint64_t* bar_o, volatile int* abort_flag,
+                                               DevStatus* st) {
+  const int w = static_cast<int>(warp & 3u);  // key quarter
+  const uint32_t row_addr = tbase + ((32u * w) << 16);
+  const uint32_t tS = row_addr + C::S_COL(0) + 32u * w;  // this quarter's 32 columns of S
+  const uint32_t tP = row_addr + C::P_COL(0);
+  const uint32_t tO = row_addr + C::O_COL(0);
+  const int qrow = q0 + static_cast<int>(lane);
+  float s_log2 = p.scale_log2;
+  if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
+  // last visible key, relative to this quarter's first key of the split's first tile
+  const int kmax = (CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1) - kt0 * C::BN - 32 * w;
+  float m_ref = -INFINITY, l_exact = 0.f, l_round = 0.f;
+  bool ok = true;
+  uint32_t zero[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) zero[i] = 0u;
+  for (int j = 0; j < n_kv; ++j) {
+    ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[0], j & 1, abort_flag, st, 50));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t s[32];
+    const int kbase = j * C::BN;  // this quarter's keys are kbase + 32w + c
+    const bool masked = __any_sync(0xffffffffu, kbase + 31 > kmax);  // warp-uniform
+    const uint64_t s2 = f2_pack(s_log2, s_log2);
+    uint64_t acc_e[2] = {0ull, 0ull}, acc_r[2] = {0ull, 0ull};
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float alpha = 1.0f;
+    tmem_ld32(tS, s);
+    tmem_wait_ld_dep32(s);
+    if (masked) mask_chunk32(s, kbase, kmax);
+    if (j == 0) {
+      float a = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) a = fmax3(a, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      // a quarter with no visible key keeps reference 0 and zero weights (its
+      // later tiles hold only later keys, so it stays empty)
+      m_ref = a == -INFINITY ? 0.f : a * s_log2;
+      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+      exp_chunk32<false, false>(s, s, s2, nm2, acc_e, acc_r, mx);
+    } else {
+      uint32_t keep[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) keep[c] = s[c];
+      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+      exp_chunk32<false, true>(s, s, s2, nm2, acc_e, acc_r, mx);
+      const float mx_s = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * s_log2;
+      const bool grow = mx_s > m_ref + 8.0f;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_new = grow ? mx_s : m_ref;
+        alpha = ex2_approx(m_ref - m_new);
+        m_ref = m_new;
+        acc_e[0] = acc_e[1] = acc_r[0] = acc_r[1] = 0ull;
+        const uint64_t nm2b = f2_pack(-m_ref, -m_ref);
+        exp_chunk32<false, false>(keep, s, s2, nm2b, acc_e, acc_r, mx);
+        // rescale this warp's O rows (PV of the previous tile has completed)
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c0, ov);
+          tmem_wait_ld_dep32(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tO + c0, ov);
+        }
+      }
+    }
+    float e0, e1, e2, e3, r0, r1, r2, r3;
+    f2_unpack(acc_e[0], e0, e1);
+    f2_unpack(acc_e[1], e2, e3);
+    f2_unpack(acc_r[0], r0, r1);
+    f2_unpack(acc_r[1], r2, r3);
+    l_exact = l_exact * alpha + ((e0 + e1) + (e2 + e3));
+    l_round = l_round * alpha + ((r0 + r1) + (r2 + r3));
+    // P: this quarter's 16 bf16-pair columns, zeros in the other three quarters
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (q == w)  // warp-uniform
+        tmem_st16(tP + 16u * q, s);
+      else
+        tmem_st16(tP + 16u * q, zero);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar_p[0]);
+  }
+  if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[0], 0, abort_flag, st, 51));
+  if (n_kv > 0) tc_fence_after();
+  // Merge the four quarters of each row: stats through static shared memory,
+  // then warps 1-3 hand their scaled O rows to warp 0 through the (now idle)
+  // K/V ring. Every softmax thread passes both barriers.
+  __shared__ float stat[3][4][32];
+  stat[0][w][lane] = m_ref;
+  stat[1][w][lane] = l_exact;
+  stat[2][w][lane] = l_round;
+  named_barrier_sync(1, 128);
+  float M = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if (stat[1][u][lane] > 0.f) M = fmaxf(M, stat[0][u][lane]);
+  float le = 0.f, lr = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float a = stat[1][u][lane] > 0.f ? ex2_approx(stat[0][u][lane] - M) : 0.f;
+    le += a * stat[1][u][lane];
+    lr += a * stat[2][u][lane];
+  }
+  const float my_a = l_exact > 0.f ? ex2_approx(m_ref - M) : 0.f;
+  const bool empty = le == 0.f;  // no visible key in any quarter (partial mode only)
+  const float inv = empty ? 0.f : 1.0f / lr;
+  const bool in_range = qrow < p.Nq;
+  float* buf = reinterpret_cast<float*>(sbuf);  // [3][32][D]: quarters 1..3
+  if (w > 0 && ok && n_kv > 0) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t ov[32];
+      tmem_ld32(tO + c0, ov);
+      tmem_wait_ld_dep32(ov);
+      if (in_range) {
+        float4* dst = reinterpret_cast<float4*>(buf + ((w - 1) * 32 + lane) * D + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(ov[4 * i]) * my_a, __uint_as_float(ov[4 * i + 1]) * my_a,
+                               __uint_as_float(ov[4 * i + 2]) * my_a, __uint_as_float(ov[4 * i + 3]) * my_a);
+      }
+    }
+  }
+  named_barrier_sync(1, 128);
+  if (w != 0 || !ok) return;
+  const bool any = n_kv > 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t ov[32];
+    if (any) {
+      tmem_ld32(tO + c0, ov);
+      tmem_wait_ld_dep32(ov);
+    }
+    if (!in_range) continue;
+    float o[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = any ? __uint_as_float(ov[i]) * my_a : 0.f;
+    if (any) {
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const float4* src = reinterpret_cast<const float4*>(buf + (u * 32 + lane) * D + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 v = src[i];
+          o[4 * i] += v.x; o[4 * i + 1] += v.y; o[4 * i + 2] += v.z; o[4 * i + 3] += v.w;
+        }
+      }
+    }
+    if constexpr (PARTIAL) {
+      float4* dst = reinterpret_cast<float4*>(p.o_part + ((static_cast<size_t>(sp) * p.BH + bh) * p.Nq + qrow) * D + c0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.Nq + qrow) * D + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pack_bf16x2(o[8 * i] * inv, o[8 * i + 1] * inv), pack_bf16x2(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                            pack_bf16x2(o[8 * i + 4] * inv, o[8 * i + 5] * inv), pack_bf16x2(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+    }
+  }
+  if (!in_range) return;
+  const float lse = empty ? -INFINITY : (M + __log2f(le)) * 0.69314718055994530942f;
+  if constexpr (PARTIAL)
+    p.lse_part[(static_cast<size_t>(sp) * p.BH + bh) * p.Nq + qrow] = lse;
+  else if (p.lse != nullptr)
+    p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = lse;
+}
+
 // PARTIAL: the CTA's keys are one block of a split (p.n_split blocks) and it
 // writes fp32 partial results (o_part, lse_part) instead of O and LSE.
-template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL>
+//
+// DEC (decode-shaped problems, Nq <= 32, one query tile): the Nq query rows are
+// loaded four times, into TMEM lanes 0-31, 32-63, 64-95 and 96-127 of S and O
+// (the Q tile map's box is 32 rows), and softmax warp w takes only keys
+// 32w .. 32w+31 of every key tile for its copy of the rows: P is zero outside
+// that quarter, so O lanes 32w+r accumulate query r's output over quarter w of
+// the keys, each with its own online softmax. The epilogue merges the four by
+// their maxima and sums (the same combination as for blocks of a split). A thread
+// thus takes 32 exponentials per key tile instead of 128, which shortens the
+// serial softmax -> P V -> S chain that bounds a CTA with one query tile.
+template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, QK_FP8>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, NQ, QK_FP8>;
+  static_assert(!DEC || NQ == 1, "the decode layout uses one query tile");
+  static_assert(!DEC || C::NSLOT * C::SLOT >= 3 * 32 * D * 4, "decode merge buffer lives in the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                      // NQ tiles
@@ -303,10 +494,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bar_q, NQ * C::Q_TILE);
-      for (int t = 0; t < NQ; ++t)
-        for (int c = 0; c < C::QK_CHUNKS; ++c)
-          tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK), q0 + t * C::BM,
-                      bh);
+      if constexpr (DEC) {
+        // rows q0 .. q0+31 into each 32-row quarter of the tile (4 KB apart per chunk)
+        for (int w = 0; w < 4; ++w)
+          for (int c = 0; c < C::QK_CHUNKS; ++c)
+            tma_load_3d(sQ + c * (C::BM * 128) + w * 32 * 128, &tmQ, &bar_q, c * (128 / C::EQK), q0, bh);
+      } else {
+        for (int t = 0; t < NQ; ++t)
+          for (int c = 0; c < C::QK_CHUNKS; ++c)
+            tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK), q0 + t * C::BM,
+                        bh);
+      }
       int pos = 0;
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -391,6 +589,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else {
     // ----------------------------------------------------------- softmax --
     if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
+    if constexpr (DEC) {
+      decode_softmax<D, CAUSAL, QK_FP8, PARTIAL, C>(p, tbase, warp, lane, q0, bh, sp, kt0, n_kv, sRing, bar_s,
+                                                    bar_p, bar_o, &abort_flag, st);
+    } else {
     const int t = static_cast<int>(warp >> 2);
     const uint32_t lane_base = (warp & 3u) * 32u;
     const int r = static_cast<int>(lane_base + lane);  // row within the tile = TMEM lane
@@ -517,6 +719,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (in_range && p.lse != nullptr)
         p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     }
+    }  // not DEC
   }
 
   tc_fence_before();

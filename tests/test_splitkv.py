@@ -2,7 +2,10 @@
 (fa_fwd_splitkv, fa_fwd_partial, fa_lse_merge through the C ABI) against the
 fp64 oracle: the per-block partial results (O = 0 and LSE = -inf exactly where a
 row sees no key of a block), the merge, and the merged output for split counts
-from 1 (no split) up to more blocks than key tiles."""
+from 1 (no split) up to more blocks than key tiles. Up to 32 queries per head
+run the decode layout (each softmax warp on one quarter of every key tile);
+the cases include 32 and 33 queries and key counts that leave whole quarters
+without a visible key."""
 import math
 
 import numpy as np
@@ -37,6 +40,7 @@ def _block_bounds(Nk, n_split):
 
 
 @pytest.mark.parametrize("B,H,Nq,Nk,d", [(1, 2, 1, 1, 128), (2, 3, 1, 777, 128), (1, 2, 5, 300, 64),
+                                         (1, 2, 32, 40, 128), (2, 2, 16, 70, 256), (1, 2, 33, 500, 64),
                                          (1, 2, 128, 1000, 128), (1, 1, 200, 4100, 128), (2, 2, 3, 2000, 256),
                                          (1, 2, 700, 700, 64)])
 @pytest.mark.parametrize("causal", [False, True])
