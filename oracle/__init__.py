@@ -33,6 +33,10 @@ Pieces, each citing the passage it follows:
   finite 448), encoded with round-to-nearest-even and saturation.
 * :func:`quantize_per_tensor` — step 3 of the same subsection ("quantização para
   FP8") with one scale per tensor: descale = amax/448 after rotation.
+* :func:`quantize_per_block` — the same step with one scale per block of 128
+  consecutive rows of a head (the attention kernel's tile), so that a block's
+  codes use the range its own values need. The pages name no block size; this is
+  the finer-grained variant of the per-tensor step.
 """
 from __future__ import annotations
 
@@ -276,3 +280,31 @@ def quantize_per_tensor(x, rotate_qk: bool, signs=None, return_scaled: bool = Fa
     if return_scaled:
         return codes, descale, scaled
     return codes, descale
+
+
+def quantize_per_block(x, rotate_qk: bool, signs=None, block_rows: int = 128):
+    """Rotate (optionally) then quantise ``x`` ``[B, H, N, d]`` to e4m3 with one
+    scale per block of ``block_rows`` rows of each head (the last block of a head
+    holds the remaining N mod block_rows rows).
+
+    Per block b: amax_b = max |x'| over its rows, descale_b = amax_b / 448 (1 if
+    amax_b = 0), codes = e4m3_encode(x' * 448 / amax_b). Returns ``(codes,
+    descales)`` with descales ``[B, H, ceil(N / block_rows)]``.
+    """
+    xr = rotate(x, signs) if rotate_qk else _as_f64(x)
+    B, H, N, d = xr.shape
+    nb = -(-N // block_rows)
+    codes = np.zeros(xr.shape, dtype=np.uint8)
+    descales = np.ones((B, H, nb), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                rows = slice(i * block_rows, min(N, (i + 1) * block_rows))
+                blk = xr[b, h, rows]
+                amax = float(np.max(np.abs(blk)))
+                if amax == 0.0:
+                    codes[b, h, rows] = e4m3_encode(np.zeros_like(blk))
+                    continue
+                codes[b, h, rows] = e4m3_encode(blk * (E4M3_MAX / amax))
+                descales[b, h, i] = amax / E4M3_MAX
+    return codes, descales

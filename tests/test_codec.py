@@ -128,3 +128,60 @@ def test_rotation_lowers_logit_error_with_shared_outlier_channels():
         approx = np.einsum("hid,hjd->hij", oracle.e4m3_decode(cq) * dq, oracle.e4m3_decode(ck) * dk)
         err[rot] = np.linalg.norm(approx - exact) / np.linalg.norm(exact)
     assert err[True] < err[False] / 3, err
+
+
+# ------------------------------------------------------ per-block scales --
+def _rand_bf16(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g).to(torch.bfloat16).double().numpy()
+
+
+def test_per_block_one_block_equals_per_tensor():
+    x = _rand_bf16((1, 1, 100, 64), 60)
+    c1, d1 = oracle.quantize_per_tensor(x, True)
+    c2, d2 = oracle.quantize_per_block(x, True)
+    assert np.array_equal(c1, c2) and d2.shape == (1, 1, 1) and d2[0, 0, 0] == d1
+
+
+def test_per_block_max_maps_to_448_and_blocks_are_independent():
+    x = _rand_bf16((2, 3, 300, 64), 61).astype(np.float64)  # 3 blocks per head, the last of 44 rows
+    codes, desc = oracle.quantize_per_block(x, False)
+    assert desc.shape == (2, 3, 3)
+    for b in range(2):
+        for h in range(3):
+            for i, (lo, hi) in enumerate(((0, 128), (128, 256), (256, 300))):
+                blk = np.abs(x[b, h, lo:hi])
+                assert desc[b, h, i] == pytest.approx(blk.max() / 448.0, rel=0, abs=0)
+                # the block's largest magnitude is coded as +-448 (0x7e / 0xfe)
+                at = np.unravel_index(np.argmax(blk), blk.shape)
+                assert codes[b, h, lo + at[0], at[1]] & 0x7F == 0x7E
+    # scaling one block by a power of two changes only that block's descale
+    y = x.copy()
+    y[1, 2, 128:256] *= 8.0
+    codes2, desc2 = oracle.quantize_per_block(y, False)
+    assert np.array_equal(codes2, codes)
+    assert desc2[1, 2, 1] == 8.0 * desc[1, 2, 1]
+    mask = np.ones(desc.shape, dtype=bool)
+    mask[1, 2, 1] = False
+    assert np.array_equal(desc2[mask], desc[mask])
+
+
+def test_per_block_zero_block_and_error_bound():
+    x = _rand_bf16((1, 2, 256, 128), 62).astype(np.float64)
+    x[0, 1, :128] = 0.0
+    x[0, 0, 128:] *= 65536.0  # blocks of very different ranges
+    codes, desc = oracle.quantize_per_block(x, True)
+    assert desc[0, 1, 0] == 1.0 and np.all(codes[0, 1, :128] & 0x7F == 0)
+    xr = oracle.rotate(x)
+    deq = oracle.e4m3_decode(codes) * np.repeat(desc, 128, axis=2)[..., None]
+    # within half an e4m3 spacing (relative 2^-4) of the block's scale, per element
+    scale = np.repeat(desc, 128, axis=2)[..., None] * 448.0
+    assert np.all(np.abs(deq - xr) <= np.maximum(np.abs(xr) * 2.0 ** -4, scale * 2.0 ** -10) + 1e-12)
+    # e4m3 is a floating-point code, so a scale only matters where it pushes
+    # values into the subnormal range: with one scale for the whole tensor, the
+    # block 65536x smaller than the largest lands there and loses precision
+    c_t, d_t = oracle.quantize_per_tensor(x, True)
+    small = (0, 0, slice(0, 128))
+    err_t = np.linalg.norm(oracle.e4m3_decode(c_t)[small] * d_t - xr[small])
+    err_b = np.linalg.norm(deq[small] - xr[small])
+    assert err_b < 0.5 * err_t
