@@ -34,8 +34,9 @@ typedef enum {
 } fa_status;
 
 typedef enum {
-  FA_BF16 = 0, /* Q and K are bf16 */
-  FA_E4M3 = 1  /* Q and K are e4m3 codes (one byte each) with per-tensor descales */
+  FA_BF16 = 0,       /* Q and K are bf16 */
+  FA_E4M3 = 1,       /* Q and K are e4m3 codes (one byte each) with per-tensor descales */
+  FA_E4M3_BLOCK = 2  /* e4m3 codes with one descale per 128-row block of a head */
 } fa_dtype;
 
 /*
@@ -58,8 +59,11 @@ typedef enum {
  * lse     device, fp32 [B][H][N] output (natural log), 4-byte aligned; may be NULL.
  * B, H, N >= 1; d in {64, 128, 256} for FA_BF16, {128, 256} for FA_E4M3.
  * scale   finite and > 0 (usually 1/sqrt(d)).
- * descale_qk  device, two fp32 {dq, dk} for FA_E4M3 (as written by
- *         fa_hadamard_quant); ignored (may be NULL) for FA_BF16.
+ * descale_qk  device fp32: for FA_E4M3 two values {dq, dk} (as written by
+ *         fa_hadamard_quant); for FA_E4M3_BLOCK the B*H*ceil(N/128) query-block
+ *         descales followed by the B*H*ceil(N/128) key-block descales, each
+ *         [B][H][block] (as written by fa_hadamard_quant_blocks); ignored (may be
+ *         NULL) for FA_BF16.
  * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
@@ -82,7 +86,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  * q       device, [B][H][Nq][d] (bf16, or e4m3 codes for FA_E4M3), 16-byte aligned.
  * k, v    device, [B][H][Nk][d] (k: bf16 or e4m3 codes; v: bf16), 16-byte aligned.
  * o       device, bf16 [B][H][Nq][d] output; lse fp32 [B][H][Nq] (natural log) or NULL.
- * B, H, Nq, Nk >= 1; causal requires Nq <= Nk. d, scale, qk_dtype, descale_qk: as fa_fwd.
+ * B, H, Nq, Nk >= 1; causal requires Nq <= Nk. d, scale, qk_dtype: as fa_fwd;
+ *         descale_qk as fa_fwd, with FA_E4M3_BLOCK holding B*H*ceil(Nq/128) query
+ *         blocks then B*H*ceil(Nk/128) key blocks.
  * n_split 1 = no split (no workspace; the same kernel as fa_fwd); >= 2 = that many
  *         blocks of ceil(ceil(Nk/128)/n_split) key tiles of 128 keys (the last ones
  *         may be empty); 0 = automatic: with fewer query blocks (of 128 or 256
@@ -173,6 +179,27 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
                             const float* signs, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_hadamard_quant_blocks — rotate (optionally) and quantise one tensor to e4m3
+ * with one scale per block of 128 consecutive rows of each head (the attention
+ * kernel's query and key tiles), in one pass over the input.
+ *
+ * Defined by: the same steps as fa_hadamard_quant ("FlashAttention-3 (PT)",
+ * section "Inovações técnicas", subsection 3), with the amax taken per block
+ * instead of per tensor; the pages give no block size. Per block b of a head (rows
+ * 128b .. min(N, 128b+128)):
+ *   amax_b = max |x'| over the block;  descales[head][b] = amax_b / 448 (1 if 0);
+ *   out = e4m3(x' * 448 / amax_b), round to nearest even, saturating.
+ *
+ * x         device, bf16 [BH][N][d], 16-byte aligned.
+ * out       device, e4m3 codes [BH][N][d], 16-byte aligned.
+ * descales  device, fp32 [BH][ceil(N/128)], 4-byte aligned.
+ * BH, N >= 1; d in {64, 128, 256}; rotate, signs: as fa_hadamard_quant.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int d, int rotate,
+                                   const float* signs, void* stream);
+
+/*
  * fa_hadamard_quant_noalloc — fa_hadamard_quant for callers that cannot allocate
  * device memory, for up to 64 tensors of one shape (e.g. Q and K) per call.
  *
@@ -212,7 +239,8 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
 
-/* ABI version of this header: 2 (1 plus the split-key, partial and merge calls). */
+/* ABI version of this header: 3 (1, plus the split-key, partial and merge calls in 2,
+ * plus per-block e4m3 scales in 3). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

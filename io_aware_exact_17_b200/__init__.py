@@ -14,11 +14,12 @@ from .binding import (  # noqa: F401
     fwd_partial,
     fwd_splitkv,
     hadamard_quant,
+    hadamard_quant_blocks,
     library_path,
     load_library,
     lse_merge,
     splitkv_splits,
 )
 
-__all__ = ["fwd", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant", "device_status",
-           "load_library", "library_path", "FaError"]
+__all__ = ["fwd", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
+           "hadamard_quant_blocks", "device_status", "load_library", "library_path", "FaError"]

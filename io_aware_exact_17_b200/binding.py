@@ -21,7 +21,8 @@ _lib = None
 _workspaces: dict[int, torch.Tensor] = {}
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
-FA_BF16, FA_E4M3 = 0, 1
+FA_BF16, FA_E4M3, FA_E4M3_BLOCK = 0, 1, 2
+BLOCK_ROWS = 128  # rows per scale block of fa_hadamard_quant_blocks
 QUANT_WORKSPACE_BYTES = 256
 E4M3_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
@@ -69,6 +70,8 @@ def load_library():
         lib.fa_fwd_partial.restype = i
         lib.fa_lse_merge.argtypes = [vp, vp, i, i64, i, vp, vp, vp]
         lib.fa_lse_merge.restype = i
+        lib.fa_hadamard_quant_blocks.argtypes = [vp, vp, vp, i, i, i, i, vp, vp]
+        lib.fa_hadamard_quant_blocks.restype = i
         _lib = lib
         return lib
 
@@ -87,6 +90,23 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _descale_arg(qk_descale, B, H, Nq, Nk):
+    """(fa_dtype, fp32 CUDA tensor) for e4m3 inputs: a 2-element tensor [dq, dk]
+    is one scale per tensor; a pair (dq_blocks [B, H, ceil(Nq/128)], dk_blocks
+    [B, H, ceil(Nk/128)]) is one scale per 128-row block."""
+    if isinstance(qk_descale, (tuple, list)):
+        dq, dk = qk_descale
+        nbq, nbk = -(-Nq // BLOCK_ROWS), -(-Nk // BLOCK_ROWS)
+        if dq.numel() != B * H * nbq or dk.numel() != B * H * nbk:
+            raise FaError(f"per-block descales must hold B*H*ceil(N/128) values ({B * H * nbq}, {B * H * nbk})")
+        if dq.dtype != torch.float32 or dk.dtype != torch.float32 or not (dq.is_cuda and dk.is_cuda):
+            raise FaError("per-block descales must be CUDA fp32 tensors")
+        return FA_E4M3_BLOCK, torch.cat([dq.reshape(-1), dk.reshape(-1)])
+    if qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2:
+        raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk] or a pair of per-block tensors")
+    return FA_E4M3, qk_descale.contiguous()
+
+
 def _require_cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -100,7 +120,9 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
     """Attention forward of ``[B, H, N, d]`` inputs.
 
     q, k: bf16, or e4m3 codes (uint8 / float8_e4m3fn) with ``qk_descale`` a
-    CUDA fp32 tensor ``[dq, dk]``; v: bf16. Returns ``(O, LSE)``: bf16
+    CUDA fp32 tensor ``[dq, dk]`` (one scale per tensor, as ``hadamard_quant``
+    gives) or a pair of per-block descales (as ``hadamard_quant_blocks`` gives);
+    v: bf16. Returns ``(O, LSE)``: bf16
     ``[B, H, N, d]`` and fp32 ``[B, H, N]`` (natural log); LSE is ``None`` when
     ``return_lse`` is false.
 
@@ -120,8 +142,6 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
         raise FaError("q and k must both be bf16 or both e4m3")
     if v.dtype != torch.bfloat16:
         raise FaError("v must be bf16")
-    if fp8 and (qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2):
-        raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk]")
     if n_split not in (0, 1):
         raise FaError("n_split must be 0 (automatic) or 1 (no split); use fwd_splitkv for a fixed split")
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
@@ -131,8 +151,8 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    desc = _ptr(qk_descale.contiguous()) if fp8 else None
-    dt = FA_E4M3 if fp8 else FA_BF16
+    dt, desc_t = _descale_arg(qk_descale, B, H, N, N) if fp8 else (FA_BF16, None)
+    desc = _ptr(desc_t)
     with torch.cuda.device(q.device):
         if n_split == 1:
             rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, N, d,
@@ -175,8 +195,6 @@ def _qkv_kinds(q, k, v, qk_descale):
         raise FaError("q and k must both be bf16 or both e4m3")
     if v.dtype != torch.bfloat16:
         raise FaError("v must be bf16")
-    if fp8 and (qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2):
-        raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk]")
     B, H, Nq, d = q.shape
     return B, H, Nq, k.shape[2], d, fp8
 
@@ -213,9 +231,9 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, qk_de
         if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk) if fp8 else (FA_BF16, None)
         rc = lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, Nq,
-                                Nk, d, int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
-                                _ptr(qk_descale.contiguous()) if fp8 else None, int(n_split),
+                                Nk, d, int(bool(causal)), float(scale), dt, _ptr(desc_t), int(n_split),
                                 _ptr(workspace) if need > 0 else None, ws_bytes, _stream(q.device))
     _check(rc, "fa_fwd_splitkv")
     return out, (lse if return_lse else None)
@@ -238,9 +256,9 @@ def fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, qk_de
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(q.device):
+        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk) if fp8 else (FA_BF16, None)
         rc = lib.fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, Nq, Nk, d,
-                                int(bool(causal)), float(scale), FA_E4M3 if fp8 else FA_BF16,
-                                _ptr(qk_descale.contiguous()) if fp8 else None, int(n_split), _stream(q.device))
+                                int(bool(causal)), float(scale), dt, _ptr(desc_t), int(n_split), _stream(q.device))
     _check(rc, "fa_fwd_partial")
     return o_part, lse_part
 
@@ -303,6 +321,32 @@ def hadamard_quant(x, rotate: bool = True, signs=None, out=None, descale=None, w
                                    workspace.numel() * workspace.element_size(), _stream(x.device))
     _check(rc, "fa_hadamard_quant")
     return out, descale
+
+
+def hadamard_quant_blocks(x, rotate: bool = True, signs=None, out=None, descales=None):
+    """Rotate (optionally) and quantise ``x`` (bf16 ``[B, H, N, d]``) to e4m3
+    with one scale per block of 128 rows of each head, through
+    ``fa_hadamard_quant_blocks``. Returns ``(codes, descales)``: uint8 codes
+    shaped like ``x`` and CUDA fp32 ``[B, H, ceil(N/128)]``."""
+    _require_cuda(x)
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 4:
+        raise FaError("x must be bf16 [B, H, N, d]")
+    x = x.contiguous()
+    B, H, N, d = x.shape
+    nb = -(-N // BLOCK_ROWS)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if descales is None:
+        descales = torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
+    if signs is not None:
+        signs = signs.to(device=x.device, dtype=torch.float32).contiguous()
+    with torch.cuda.device(x.device):
+        rc = lib.fa_hadamard_quant_blocks(_ptr(x), _ptr(out), _ptr(descales), B * H, N, d, int(bool(rotate)),
+                                          _ptr(signs) if (rotate and signs is not None) else None,
+                                          _stream(x.device))
+    _check(rc, "fa_hadamard_quant_blocks")
+    return out, descales
 
 
 def device_status():

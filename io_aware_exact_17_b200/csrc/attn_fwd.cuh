@@ -88,7 +88,12 @@ struct FwdParams {
   float* lse;                // [BH][Nq], may be null
   float* o_part;             // partial mode: [n_split][BH][Nq][D] fp32, O of the split's keys; else null
   float* lse_part;           // partial mode: [n_split][BH][Nq], -inf where a row sees no key of the split
-  const float* descale_qk;   // e4m3 path: {dq, dk}; else null
+  const float* descale_qk;   // e4m3 path, one scale per tensor: {dq, dk}; else null
+  // e4m3 path, one scale per 128-row block of a head (descale_qk unused):
+  // dq_block[bh * nbq + query tile], dk_block[bh * nbk + key tile]; else null
+  const float* dq_block;
+  const float* dk_block;
+  int nbq, nbk;
   int BH;                    // batch * heads
   int Nq, Nk;                // query rows and keys per head
   int causal_off;            // Nk - Nq: key j is visible to query i iff j <= i + causal_off (causal)
@@ -234,8 +239,16 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
   const uint32_t tP = row_addr + C::P_COL(0);
   const uint32_t tO = row_addr + C::O_COL(0);
   const int qrow = q0 + static_cast<int>(lane);
-  float s_log2 = p.scale_log2;
-  if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
+  float s_q = p.scale_log2;
+  const float* dkb = nullptr;
+  if constexpr (QK_FP8) {
+    if (p.dq_block != nullptr) {
+      s_q *= __ldg(p.dq_block + static_cast<size_t>(bh) * p.nbq);  // Nq <= 32: query block 0
+      dkb = p.dk_block + static_cast<size_t>(bh) * p.nbk + kt0;
+    } else {
+      s_q *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
+    }
+  }
   // last visible key, relative to this quarter's first key of the split's first tile
   const int kmax = (CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1) - kt0 * C::BN - 32 * w;
   float m_ref = -INFINITY, l_exact = 0.f, l_round = 0.f;
@@ -243,7 +256,10 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
   uint32_t zero[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) zero[i] = 0u;
+  float dk_next = (QK_FP8 && dkb != nullptr && n_kv > 0) ? __ldg(dkb) : 1.0f;
   for (int j = 0; j < n_kv; ++j) {
+    const float s_log2 = s_q * dk_next;
+    if (QK_FP8 && dkb != nullptr && j + 1 < n_kv) dk_next = __ldg(dkb + j + 1);
     ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[0], j & 1, abort_flag, st, 50));
     if (!ok) break;
     tc_fence_after();
@@ -601,8 +617,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tS = row_addr + C::S_COL(t);
     const uint32_t tP = row_addr + C::P_COL(t);
     const uint32_t tO = row_addr + C::O_COL(t);
-    float s_log2 = p.scale_log2;
-    if constexpr (QK_FP8) s_log2 *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
+    // exp2 scale: scale * log2(e), times the descales of the query tile and (per
+    // key tile, when scales are per block) of the key tile
+    float s_q = p.scale_log2;
+    const float* dkb = nullptr;
+    if constexpr (QK_FP8) {
+      if (p.dq_block != nullptr) {
+        if (q0 + t * C::BM < p.Nq) s_q *= __ldg(p.dq_block + static_cast<size_t>(bh) * p.nbq + (q0 + t * C::BM) / C::BM);
+        dkb = p.dk_block + static_cast<size_t>(bh) * p.nbk + kt0;
+      } else {
+        s_q *= __ldg(p.descale_qk) * __ldg(p.descale_qk + 1);
+      }
+    }
     // Last visible key of this row, counted from the split's first key (so the
     // loop below works in split-relative key indices).
     const int kmax = (CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1) - kt0 * C::BN;
@@ -611,7 +637,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float l_round = 0.f;      // sum of the bf16-rounded weights P uses: normalises O
     bool ok = true;
     const int n_kv_t = n_kv_at(t);
+    float dk_next = (QK_FP8 && dkb != nullptr && n_kv_t > 0) ? __ldg(dkb) : 1.0f;
     for (int j = 0; j < n_kv_t; ++j) {
+      const float s_log2 = s_q * dk_next;
+      if (QK_FP8 && dkb != nullptr && j + 1 < n_kv_t) dk_next = __ldg(dkb + j + 1);  // in flight during this step
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
       if (!ok) break;
       tc_fence_after();

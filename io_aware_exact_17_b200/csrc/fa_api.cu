@@ -95,6 +95,15 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   p.o_part = a.o_part;
   p.lse_part = a.lse_part;
   p.descale_qk = a.descale_qk;
+  p.dq_block = nullptr;
+  p.dk_block = nullptr;
+  p.nbq = (a.Nq + 127) / 128;
+  p.nbk = (a.Nk + 127) / 128;
+  if (a.qk_dtype == FA_E4M3_BLOCK) {
+    // one descale per 128-row block: the query blocks of every head, then the key blocks
+    p.dq_block = a.descale_qk;
+    p.dk_block = a.descale_qk + static_cast<size_t>(BH) * p.nbq;
+  }
   p.BH = BH;
   p.Nq = a.Nq;
   p.Nk = a.Nk;
@@ -150,11 +159,11 @@ fa_status check_fwd_args(const void* q, const void* k, const void* v, int B, int
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || n_split < 1) return FA_ERR_INVALID_ARG;
   if (causal != 0 && Nq > Nk) return FA_ERR_INVALID_ARG;  // some query would see no key
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (qk_dtype != FA_BF16 && qk_dtype != FA_E4M3) return FA_ERR_INVALID_ARG;
+  if (qk_dtype != FA_BF16 && qk_dtype != FA_E4M3 && qk_dtype != FA_E4M3_BLOCK) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  if (qk_dtype == FA_E4M3 && d == 64) return FA_ERR_UNSUPPORTED;
+  if (qk_dtype != FA_BF16 && d == 64) return FA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return FA_ERR_ALIGNMENT;
-  if (qk_dtype == FA_E4M3) {
+  if (qk_dtype != FA_BF16) {
     if (descale_qk == nullptr) return FA_ERR_INVALID_ARG;
     if (!aligned(descale_qk, 4)) return FA_ERR_ALIGNMENT;
   }
@@ -436,6 +445,38 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
   }
 }
 
+fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int d, int rotate,
+                                   const float* signs, void* stream) {
+  if (x == nullptr || out == nullptr || descales == nullptr) return FA_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1 || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const long long nb = (static_cast<long long>(N) + fa::kBlockRows - 1) / fa::kBlockRows;
+  if (nb * BH > 0x7fffffffLL || static_cast<long long>(BH) * N > (1LL << 40)) return FA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(descales, 4)) return FA_ERR_ALIGNMENT;
+  if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
+  const float* sg = rotate ? signs : nullptr;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  uint8_t* ob = static_cast<uint8_t*>(out);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(nb * BH);
+  const int nbi = static_cast<int>(nb);
+  switch (d) {
+    case 64:
+      if (rotate) fa::quant_block_kernel<64, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
+      else fa::quant_block_kernel<64, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
+      break;
+    case 128:
+      if (rotate) fa::quant_block_kernel<128, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
+      else fa::quant_block_kernel<128, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
+      break;
+    default:
+      if (rotate) fa::quant_block_kernel<256, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
+      else fa::quant_block_kernel<256, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
+      break;
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -531,6 +572,6 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
   return FA_OK;
 }
 
-int fa_abi_version(void) { return 2; }
+int fa_abi_version(void) { return 3; }
 
 }  // extern "C"

@@ -353,3 +353,74 @@ quant_fused_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
 }
 
 }  // namespace fa
+
+namespace fa {
+
+// ---------------------------------------------------------------------------
+// Per-block scales: one CTA per block of 128 consecutive rows of a head. The
+// block's rotated values stay in registers between its amax and its codes, so
+// the input is read once, with no second pass and no grid-wide barrier (every
+// scale depends on one CTA's data only). The rotation is hadamard_rotate32's.
+// ---------------------------------------------------------------------------
+constexpr int kBlockRows = 128;
+constexpr int kBlockThreads = 256;
+
+template <int D, bool ROT>
+__global__ void __launch_bounds__(kBlockThreads)
+quant_block_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ out, int N, int nb,
+                   const float* __restrict__ signs, float* __restrict__ descales) {
+  using C = FusedCfg<D>;
+  constexpr int WARPS = kBlockThreads / 32;
+  constexpr int STEPS = kBlockRows / (WARPS * C::RPW);  // rows of a warp / rows per warp-step
+  static_assert(STEPS * WARPS * C::RPW == kBlockRows, "block rows");
+  const int bh = blockIdx.x / nb, blk = blockIdx.x % nb;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lr = lane % C::L, sub = lane / C::L;
+  const int row0 = blk * kBlockRows;
+  const __nv_bfloat16* xh = x + static_cast<int64_t>(bh) * N * D;
+  uint8_t* oh = out + static_cast<int64_t>(bh) * N * D;
+  float v[STEPS][32];
+  float m = 0.f;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int row = row0 + (s * WARPS + warp) * C::RPW + sub;
+    if (row < N) {
+      load_bf16x32<D>(xh + static_cast<int64_t>(row) * D, lr, v[s]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[s][e] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    if (ROT) hadamard_rotate32<D>(v[s], lr, signs);
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) m = fmax3(m, fabsf(v[s][e]), fabsf(v[s][e + 1]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float warp_max[WARPS];
+  if (lane == 0) warp_max[warp] = m;
+  __syncthreads();
+  float amax = warp_max[0];
+#pragma unroll
+  for (int i = 1; i < WARPS; ++i) amax = fmaxf(amax, warp_max[i]);
+  const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
+  if (threadIdx.x == 0) descales[blockIdx.x] = amax > 0.f ? amax / 448.0f : 1.0f;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int row = row0 + (s * WARPS + warp) * C::RPW + sub;
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      q[i] = static_cast<uint32_t>(pack_e4m3x2(v[s][4 * i] * scale, v[s][4 * i + 1] * scale)) |
+             (static_cast<uint32_t>(pack_e4m3x2(v[s][4 * i + 2] * scale, v[s][4 * i + 3] * scale)) << 16);
+    if (row < N) {
+      uint2* dst = reinterpret_cast<uint2*>(oh + static_cast<int64_t>(row) * D);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
+    }
+  }
+}
+
+}  // namespace fa

@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
     assert {"fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_splits", "fa_fwd_partial",
             "fa_lse_merge"} <= set(names)
-    assert lib.fa_abi_version() == 2
+    assert lib.fa_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -130,6 +130,23 @@ def test_partial_and_merge_argument_errors(lib):
     assert merge(d=80) == binding.FA_ERR_UNSUPPORTED
     assert merge(op=MIS) == binding.FA_ERR_ALIGNMENT
     assert merge(o=MIS) == binding.FA_ERR_ALIGNMENT
+
+
+def test_block_quant_argument_errors(lib):
+    bq = lambda **kw: lib.fa_hadamard_quant_blocks(kw.get("x", A), kw.get("out", A), kw.get("ds", A), kw.get("BH", 2),
+                                                   kw.get("N", 300), kw.get("d", 128), kw.get("rot", 1), None, None)
+    assert bq(x=None) == binding.FA_ERR_INVALID_ARG
+    assert bq(ds=None) == binding.FA_ERR_INVALID_ARG
+    assert bq(BH=0) == binding.FA_ERR_INVALID_ARG
+    assert bq(N=0) == binding.FA_ERR_INVALID_ARG
+    assert bq(rot=3) == binding.FA_ERR_INVALID_ARG
+    assert bq(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert bq(x=MIS) == binding.FA_ERR_ALIGNMENT
+    assert bq(ds=A + 2) == binding.FA_ERR_ALIGNMENT
+    # per-block descales are an e4m3 dtype: not for d = 64, and they are required
+    assert _fwd(lib, dtype=2, desc=A, d=64) == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=2, desc=None) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=3, desc=A) == binding.FA_ERR_INVALID_ARG
 
 
 def test_python_binding_rejects_cpu_tensors():
