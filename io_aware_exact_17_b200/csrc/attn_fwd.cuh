@@ -659,14 +659,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (PARTIAL && m_ref == -INFINITY) m_ref = 0.f;
         softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
       } else {
-        // Exponentials against the current reference, taking the row's max on the
-        // way; only if some row's max grew by more than 2^8 (rare after the first
-        // tiles) is the row redone against the new reference. S is still intact:
-        // P is written only below.
-        softmax_row_dispatch<true>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
-        const float mx_s = mx * s_log2;
-        const bool grow = mx_s > m_ref + 8.0f;
-        if (__any_sync(0xffffffffu, grow)) {
+        // Exponentials against the current reference. A row whose max grew by more
+        // than 8 (log2 units) has a weight above 2^8, so its tile sum exceeds 2^8:
+        // only then (rare after the first tiles) is its exact max taken, and the
+        // tile redone, against the new reference if the max did grow that much.
+        // S is still intact: P is written only below.
+        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        if (__any_sync(0xffffffffu, sum_e > 256.0f)) {
+          const float mx_s = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;
+          const bool grow = mx_s > m_ref + 8.0f;
           const float m_new = grow ? mx_s : m_ref;
           alpha = ex2_approx(m_ref - m_new);  // 1 for rows that did not grow
           m_ref = m_new;
@@ -674,14 +675,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
           // completed (the commit that signalled S_t for tile j also covers it),
           // and PV of tile j is issued only after this warpgroup arrives below.
+          if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c0, ov);
-            tmem_wait_ld_dep32(ov);
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld32(tO + c0, ov);
+              tmem_wait_ld_dep32(ov);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tO + c0, ov);
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st32(tO + c0, ov);
+            }
           }
         }
       }

@@ -214,54 +214,78 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* row, int lr, f
 template <int D>
 __device__ __forceinline__ void hadamard_rotate32(float (&v)[32], int lr, const float* signs) {
   constexpr int L = D / 32;
+  // Stages over index bits 1 and up pair neighbouring elements (v[2i], v[2i+1])
+  // with another such pair, so they run as packed f32x2 operations: the same
+  // two IEEE additions (or subtractions, multiplications) per instruction, hence
+  // the same results as the scalar form.
+  uint64_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = f2_pack(v[2 * i], v[2 * i + 1]);
   if (signs != nullptr) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 s0 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q)));
       const float4 s1 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q) + 4));
-      v[8 * q + 0] *= s0.x; v[8 * q + 1] *= s0.y; v[8 * q + 2] *= s0.z; v[8 * q + 3] *= s0.w;
-      v[8 * q + 4] *= s1.x; v[8 * q + 5] *= s1.y; v[8 * q + 6] *= s1.z; v[8 * q + 7] *= s1.w;
+      w[4 * q + 0] = f2_mul(w[4 * q + 0], f2_pack(s0.x, s0.y));
+      w[4 * q + 1] = f2_mul(w[4 * q + 1], f2_pack(s0.z, s0.w));
+      w[4 * q + 2] = f2_mul(w[4 * q + 2], f2_pack(s1.x, s1.y));
+      w[4 * q + 3] = f2_mul(w[4 * q + 3], f2_pack(s1.z, s1.w));
     }
   }
-  // index bits 0..2
+  // index bit 0: inside each pair (scalar)
 #pragma unroll
-  for (int h = 1; h < 8; h <<= 1) {
+  for (int i = 0; i < 16; ++i) {
+    float a, b;
+    f2_unpack(w[i], a, b);
+    w[i] = f2_pack(a + b, a - b);
+  }
+  // index bits 1, 2: pair i with pair i + h/2 inside each 8-element chunk
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      if ((e & h) == 0) {
-        const float a = v[e], b = v[e + h];
-        v[e] = a + b;
-        v[e + h] = a - b;
+  for (int h = 1; h < 4; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const uint64_t a = w[i], b = w[i + h];
+        w[i] = f2_add(a, b);
+        w[i + h] = f2_sub(a, b);
       }
     }
   }
-  // index bits 3 .. 2+log2(L): across the L lanes of the row
+  // index bits 3 .. 2+log2(L): across the L lanes of the row. Lower lane:
+  // v + other; upper lane: other - v; both as one fma with +-1 (exact: the same
+  // single rounding as the add or subtract).
 #pragma unroll
   for (int m = 1; m < L; m <<= 1) {
-    // lower lane: v + other; upper lane: other - v; both as one fma with +-1
-    // (exact: the same single rounding as the add or subtract).
-    const float sgn = (lr & m) != 0 ? -1.0f : 1.0f;
+    const float sg = (lr & m) != 0 ? -1.0f : 1.0f;
+    const uint64_t sgn = f2_pack(sg, sg);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[e], m);
-      v[e] = fmaf(v[e], sgn, other);
+    for (int i = 0; i < 16; ++i) {
+      float a, b;
+      f2_unpack(w[i], a, b);
+      const float oa = __shfl_xor_sync(0xffffffffu, a, m);
+      const float ob = __shfl_xor_sync(0xffffffffu, b, m);
+      w[i] = f2_fma(w[i], sgn, f2_pack(oa, ob));
     }
   }
-  // the two bits of q
+  // the two bits of q: pair i with pair i + 4 and i + 8
 #pragma unroll
-  for (int h = 8; h < 32; h <<= 1) {
+  for (int h = 4; h < 16; h <<= 1) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      if ((e & h) == 0) {
-        const float a = v[e], b = v[e + h];
-        v[e] = a + b;
-        v[e + h] = a - b;
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const uint64_t a = w[i], b = w[i + h];
+        w[i] = f2_add(a, b);
+        w[i + h] = f2_sub(a, b);
       }
     }
   }
   constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
+  const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) v[e] *= inv_sqrt_d;
+  for (int i = 0; i < 16; ++i) {
+    w[i] = f2_mul(w[i], isd);
+    f2_unpack(w[i], v[2 * i], v[2 * i + 1]);
+  }
 }
 
 // ws[0]: amax bits, ws[1]: arrival counter of the grid barrier; both zero at launch.
