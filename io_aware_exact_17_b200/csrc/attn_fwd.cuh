@@ -129,11 +129,11 @@ constexpr int kPolyEvery = FA_EXP_POLY_EVERY;  // 1 pair in kPolyEvery uses the 
 constexpr uint32_t kMmaWaitSleepNs = FA_MMA_WAIT_SLEEP_NS;
 
 // Exponentials of one 32-key chunk of a row of S: p = 2^(x*s - m), packed to
-// bf16 pairs into pk[0..15]; accumulates the fp32 weights and the rounded ones
-// into the packed-pair sums and (WITH_MAX) the raw-score max into mx[0..3].
-// With EMU (a tile with no masked key) one pair in kPolyEvery goes to the
-// FMA-pipe polynomial.
-template <bool EMU, bool WITH_MAX>
+// bf16 pairs into pk[0..15]; accumulates the fp32 weights, with ROUND also the
+// bf16-rounded ones, into the packed-pair sums and (WITH_MAX) the raw-score max
+// into mx[0..3]. With EMU (a tile with no masked key) one pair in kPolyEvery goes
+// to the FMA-pipe polynomial.
+template <bool EMU, bool WITH_MAX, bool ROUND = true>
 __device__ __forceinline__ void exp_chunk32(const uint32_t* s, uint32_t* pk, uint64_t s2, uint64_t nm2,
                                             uint64_t* acc_e, uint64_t* acc_r, float* mx) {
 #pragma unroll
@@ -150,7 +150,7 @@ __device__ __forceinline__ void exp_chunk32(const uint32_t* s, uint32_t* pk, uin
     const uint32_t q = pack_bf16x2(p0, p1);
     const int a = (c >> 1) & 1;
     acc_e[a] = f2_add(acc_e[a], f2_pack(p0, p1));
-    acc_r[a] = f2_add(acc_r[a], f2_pack(__uint_as_float(q << 16), __uint_as_float(q & 0xFFFF0000u)));
+    if (ROUND) acc_r[a] = f2_add(acc_r[a], f2_pack(__uint_as_float(q << 16), __uint_as_float(q & 0xFFFF0000u)));
     pk[c >> 1] = q;
   }
 }
@@ -166,8 +166,14 @@ __device__ __forceinline__ void mask_chunk32(uint32_t* s, int kbase, int kmax) {
 // (tcgen05.wait::ld waits for all earlier loads, so chunk c+1 is issued before
 // chunk c is computed). P is packed in place: chunk c's 16 bf16 pairs go to
 // s[16c .. 16c+15], scores already consumed (chunk c/2's) and never the target of
-// a pending load, so only 128 registers are live. Returns the fp32 and rounded
-// weight sums and, with WITH_MAX, the max of the raw scores.
+// a pending load, so only 128 registers are live. Returns the fp32 weight sum,
+// the sum that normalises O and, with WITH_MAX, the max of the raw scores.
+//
+// The normalising sum is the sum of the bf16-rounded weights P holds when some
+// key of the tile is masked (EMU false: the row's last tile, which holds every
+// key of a row with few keys), else the fp32 sum: over a full tile of 128 keys
+// the rounding errors of P average out to about 2^-9 / sqrt(128) of the sum, and
+// skipping the rounded sum saves three of the eight instructions per key pair.
 template <bool EMU, bool WITH_MAX>
 __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
                                             int kbase, int kmax, bool masked, float& sum_e, float& sum_r,
@@ -182,7 +188,7 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_lo
   for (int ch = 0; ch < 4; ++ch) {
     if (ch < 3) tmem_ld32(tS + 32 * (ch + 1), &s[32 * (ch + 1)]);
     if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
-    exp_chunk32<EMU, WITH_MAX>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
+    exp_chunk32<EMU, WITH_MAX, !EMU>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
     if (ch < 3) tmem_wait_ld_dep32(&s[32 * (ch + 1)]);
   }
   float e0, e1, e2, e3, r0, r1, r2, r3;
@@ -191,7 +197,7 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_lo
   f2_unpack(acc_r[0], r0, r1);
   f2_unpack(acc_r[1], r2, r3);
   sum_e = (e0 + e1) + (e2 + e3);
-  sum_r = (r0 + r1) + (r2 + r3);
+  sum_r = EMU ? sum_e : (r0 + r1) + (r2 + r3);
   if (WITH_MAX) raw_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
