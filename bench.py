@@ -55,8 +55,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the SHA-256 of the kernel's sources at that capture. When the sources differ
 # the figure no longer describes the kernel and `traffic` is reported as null.
 KERNEL_SOURCES = ("io_aware_exact_17_b200/csrc/attn_fwd.cuh", "io_aware_exact_17_b200/csrc/sm100.cuh")
-NCU_TRAFFIC_BYTES = 113745920  # 100.837120 MB read + 12.908800 MB written
-NCU_TRAFFIC_SHA256 = "6d072f683a539f1e75dff09f2f28ceafb119541020228db82c0ecd319d0ca483"
+NCU_TRAFFIC_BYTES = 112214272  # 100.743936 MB read + 11.470336 MB written
+NCU_TRAFFIC_SHA256 = "1192e9b965d1ac0182a5bd0b568935b0bd23bb04636a97133619222995bf06ed"
 
 
 def kernel_sources_sha256() -> str:
