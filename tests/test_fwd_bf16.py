@@ -157,6 +157,27 @@ def test_increasing_logits_force_rescales():
         assert max_abs(to_np(lse), lse_ref) <= BF16_LSE_ATOL * max(1.0, float(np.max(np.abs(lse_ref))) / 100)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_growth_in_the_second_half_of_key_tiles(causal):
+    # Scores that stay flat over keys 0..63 of every 128-key tile and jump over
+    # keys 64..127, higher tile after tile: the row max grows by more than 2^8
+    # (log2 units) inside the second half, after P V of the first half is already
+    # issued against the old reference. Exercises the wait for that product and
+    # the rescale of O that follow.
+    B, H, N, d = 1, 2, 640, 64
+    q = torch.full((B, H, N, d), 0.125).to(torch.bfloat16)
+    t = torch.zeros(N)
+    for j in range(128, N):
+        if j % 128 >= 64:
+            t[j] = 2.0 * (j // 128)  # score 8 t: +16 per tile (23 in log2 units)
+    k = (torch.ones(B, H, N, d) * t.view(1, 1, N, 1)).to(torch.bfloat16)
+    _, _, v = inputs.qkv_normal(B, H, N, d, 38)
+    o, lse = _run(q, k, v, causal, scale=1.0)
+    o_ref, lse_ref = oracle.attention(q, k, v, causal, 1.0)
+    assert np.all(np.abs(to_np(o) - o_ref) <= bf16_out_tol(o_ref))
+    assert max_abs(to_np(lse), lse_ref) <= BF16_LSE_ATOL * max(1.0, float(np.max(np.abs(lse_ref))) / 100)
+
+
 def test_deterministic():
     q, k, v = inputs.qkv_normal(2, 4, 1000, 128, 36)
     o1, l1 = _run(q, k, v, True)
