@@ -101,9 +101,18 @@ struct FwdParams {
   int n_split;               // key splits per head (1: all keys)
   int split_tiles;           // key tiles per split
   float scale_log2;          // scale * log2(e)
-  // The grid covers the query blocks unit_base, unit_base + 1, ... (query block
-  // = bh * n_qb + qb), each with n_split CTAs in partial mode.
+  // Work items: the query blocks unit_base, unit_base + 1, ... (query block
+  // = bh * n_qb + qb), times n_split key blocks each in partial mode; n_items of
+  // them. CTA c takes items c, c + gridDim.x, ... (persistent when the grid is
+  // smaller than n_items).
   int unit_base;
+  int n_items;
+};
+
+// One work item of a CTA: head, key split, first query row, first key tile and
+// the key tiles its query tiles step through.
+struct FwdItem {
+  int bh, sp, q0, kt0, n_kv0, n_kv1, n_kv;
 };
 
 // Bounded wait used only while tearing down after an abort: ignores the abort
@@ -446,40 +455,43 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint8_t* sRing = smem + NQ * C::Q_TILE;  // NSLOT slots
 
   __shared__ __align__(8) uint64_t bar_full[C::NSLOT], bar_empty[C::NSLOT];
-  __shared__ __align__(8) uint64_t bar_q, bar_drain, bar_s[NQ], bar_p[NQ], bar_o[NQ];
+  // bar_qfree: the S MMAs that read the current item's Q tiles are done (the
+  // producer may load the next item's Q)
+  __shared__ __align__(8) uint64_t bar_q, bar_qfree, bar_drain, bar_s[NQ], bar_p[NQ], bar_o[NQ];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
   const uint32_t warp = warp_id(), lane = lane_id();
 
-  // Work item: head bh, key split sp, query block qb (heaviest causal blocks of
-  // a head first).
-  const int n_split = PARTIAL ? p.n_split : 1;
-  const int unit_rel = PARTIAL ? static_cast<int>(blockIdx.x) / n_split : static_cast<int>(blockIdx.x);
-  const int sp = PARTIAL ? static_cast<int>(blockIdx.x) % n_split : 0;
-  const int unit = p.unit_base + unit_rel;  // query block bh * n_qb + qb
-  const int bh = unit / p.n_qb;
-  int qb = unit % p.n_qb;
-  if (CAUSAL) qb = p.n_qb - 1 - qb;
-  const int q0 = qb * NQ * C::BM;
-  // Key tiles of this split: kt0 .. kt0 + split_tiles - 1 (clipped to Nk). Query
-  // tile t steps through n_kv_of(t) of them: none if it has no row (past Nq),
-  // else up to the tile holding its last visible key, so a causal tile never
-  // spends a step on keys entirely in its future. The CTA streams the most any
-  // tile needs.
-  const int kt0 = PARTIAL ? sp * p.split_tiles : 0;
-  auto n_kv_of = [&](int t) {
-    const int row0 = q0 + t * C::BM;
-    if (row0 >= p.Nq) return 0;
-    const int end = CAUSAL ? min(p.Nk, min(p.Nq, row0 + C::BM) + p.causal_off) : p.Nk;  // keys [0, end)
-    const int tiles = (end + C::BN - 1) / C::BN;
-    if (!PARTIAL) return tiles;
-    return max(0, min(tiles, kt0 + p.split_tiles) - kt0);
+  // Work item `it`: head bh, key split sp, query block qb (heaviest causal blocks
+  // of a head first). Key tiles of the split: kt0 .. kt0 + split_tiles - 1
+  // (clipped to Nk). Query tile t steps through n_kv_of(t) of them: none if it
+  // has no row (past Nq), else up to the tile holding its last visible key, so a
+  // causal tile never spends a step on keys entirely in its future. The CTA
+  // streams the most any tile needs.
+  auto item_at = [&](int it) {
+    FwdItem w;
+    const int n_split = PARTIAL ? p.n_split : 1;
+    const int unit = p.unit_base + (PARTIAL ? it / n_split : it);  // query block bh * n_qb + qb
+    w.sp = PARTIAL ? it % n_split : 0;
+    w.bh = unit / p.n_qb;
+    int qb = unit % p.n_qb;
+    if (CAUSAL) qb = p.n_qb - 1 - qb;
+    w.q0 = qb * NQ * C::BM;
+    w.kt0 = PARTIAL ? w.sp * p.split_tiles : 0;
+    auto n_kv_of = [&](int t) {
+      const int row0 = w.q0 + t * C::BM;
+      if (row0 >= p.Nq) return 0;
+      const int end = CAUSAL ? min(p.Nk, min(p.Nq, row0 + C::BM) + p.causal_off) : p.Nk;  // keys [0, end)
+      const int tiles = (end + C::BN - 1) / C::BN;
+      if (!PARTIAL) return tiles;
+      return max(0, min(tiles, w.kt0 + p.split_tiles) - w.kt0);
+    };
+    w.n_kv0 = n_kv_of(0);
+    w.n_kv1 = NQ > 1 ? n_kv_of(NQ - 1) : w.n_kv0;
+    w.n_kv = max(w.n_kv0, w.n_kv1);
+    return w;
   };
-  const int n_kv0 = n_kv_of(0);
-  const int n_kv1 = NQ > 1 ? n_kv_of(NQ - 1) : n_kv0;
-  const int n_kv = max(n_kv0, n_kv1);
-  auto n_kv_at = [&](int t) { return t == 0 ? n_kv0 : n_kv1; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -488,6 +500,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(&bar_q, 1);
+    mbar_init(&bar_qfree, 1);
     mbar_init(&bar_drain, 1);
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&bar_s[t], 1);
@@ -515,6 +528,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      int pos = 0, iter = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x, ++iter) {
+      const FwdItem w = item_at(it);
+      const int bh = w.bh, q0 = w.q0, kt0 = w.kt0, n_kv = w.n_kv;
+      // the previous item's S MMAs read sQ until they complete
+      if (iter > 0) ok = mbar_wait(&bar_qfree, (iter - 1) & 1, &abort_flag, st, 11);
+      if (!ok) break;
       mbar_arrive_expect_tx(&bar_q, NQ * C::Q_TILE);
       if constexpr (DEC) {
         // rows q0 .. q0+31 into each 32-row quarter of the tile (4 KB apart per chunk)
@@ -527,8 +548,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK), q0 + t * C::BM,
                         bh);
       }
-      int pos = 0;
-      bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
         for (int kind = 0; kind < 2 && ok; ++kind, ++pos) {
           const int slot = pos % C::NSLOT;
@@ -548,8 +567,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
+      }  // items
       // Let every load this thread issued land before the CTA can exit.
-      mbar_drain(&bar_q, 0);
+      if (iter > 0) mbar_drain(&bar_q, (iter - 1) & 1);
       for (int q = pos - C::NSLOT; q < pos; ++q)
         if (q >= 0) mbar_drain(&bar_full[q % C::NSLOT], (q / C::NSLOT) & 1);
     } else if (warp == C::MMA_WARP && lane == 0) {
@@ -558,9 +578,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       constexpr uint32_t idesc_pv = idesc_make(1u, 128, D, true);
       const uint32_t ring = smem_u32(sRing);
       const uint32_t qaddr = smem_u32(sQ);
-      bool ok = mbar_wait(&bar_q, 0, &abort_flag, st, 20);
+      int pos = 0, iter = 0;
+      uint32_t pc0 = 0, pc1 = 0;  // P-barrier phases waited, per query tile
+      bool ok = true;
+      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x, ++iter) {
+      const FwdItem w = item_at(it);
+      const int n_kv = w.n_kv;
+      auto n_kv_at = [&](int t) { return t == 0 ? w.n_kv0 : w.n_kv1; };
+      ok = mbar_wait(&bar_q, iter & 1, &abort_flag, st, 20);
       for (int j = 0; j <= n_kv && ok; ++j) {
-        const int kpos = 2 * j, vpos = 2 * j - 1;
+        const int kpos = pos + 2 * j, vpos = pos + 2 * j - 1;
         const int kslot = kpos % C::NSLOT, vslot = (vpos + C::NSLOT) % C::NSLOT;
         if (j < n_kv) ok = mbar_wait(&bar_full[kslot], (kpos / C::NSLOT) & 1, &abort_flag, st, 21);
         if (ok && j > 0) ok = mbar_wait(&bar_full[vslot], (vpos / C::NSLOT) & 1, &abort_flag, st, 22);
@@ -570,7 +597,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int n_kv_t = n_kv_at(t);
           if (j > 0 && j - 1 < n_kv_t) {
             // The single issuer polls: its wake-up is on the critical path.
-            ok = mbar_wait(&bar_p[t], (j - 1) & 1, &abort_flag, st, 23, kMmaWaitSleepNs);
+            const uint32_t ph = (t == 0 ? pc0 : pc1) & 1u;
+            if (t == 0) ++pc0; else ++pc1;
+            ok = mbar_wait(&bar_p[t], ph, &abort_flag, st, 23, kMmaWaitSleepNs);
             if (!ok) break;
             tc_fence_after();
             // O_t += P_t V_{j-1}: A = P_t from TMEM (bf16 pairs), B = V tile (MN-major).
@@ -604,6 +633,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (j > 0) mma_commit(&bar_empty[vslot]);
         if (j < n_kv) mma_commit(&bar_empty[kslot]);
       }
+      if (!ok) break;
+      mma_commit(&bar_qfree);  // done when this item's S MMAs (readers of sQ) are
+      pos += 2 * n_kv;
+      }  // items
       // Drain: TMEM is freed below only after every issued MMA has finished.
       mma_commit(&bar_drain);
       mbar_drain(&bar_drain, 0);
@@ -612,10 +645,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ----------------------------------------------------------- softmax --
     if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
     if constexpr (DEC) {
-      decode_softmax<D, CAUSAL, QK_FP8, PARTIAL, C>(p, tbase, warp, lane, q0, bh, sp, kt0, n_kv, sRing, bar_s,
-                                                    bar_p, bar_o, &abort_flag, st);
+      // one item per CTA (the merge buffer is the K/V ring)
+      const FwdItem w = item_at(blockIdx.x);
+      decode_softmax<D, CAUSAL, QK_FP8, PARTIAL, C>(p, tbase, warp, lane, w.q0, w.bh, w.sp, w.kt0, w.n_kv, sRing,
+                                                    bar_s, bar_p, bar_o, &abort_flag, st);
     } else {
     const int t = static_cast<int>(warp >> 2);
+    uint32_t sc = 0, oc = 0;  // phases of bar_s[t] and bar_o[t] waited
+    bool ok = true;
+    for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+    const FwdItem w = item_at(it);
+    const int bh = w.bh, q0 = w.q0, kt0 = w.kt0, sp = w.sp;
     const uint32_t lane_base = (warp & 3u) * 32u;
     const int r = static_cast<int>(lane_base + lane);  // row within the tile = TMEM lane
     const int qrow = q0 + t * C::BM + r;
@@ -641,13 +681,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float m_ref = -INFINITY;  // reference max, scaled log2 units
     float l_exact = 0.f;      // sum of the fp32 weights: gives the LSE
     float l_round = 0.f;      // sum of the bf16-rounded weights P uses: normalises O
-    bool ok = true;
-    const int n_kv_t = n_kv_at(t);
+    const int n_kv_t = t == 0 ? w.n_kv0 : w.n_kv1;
     float dk_next = (QK_FP8 && dkb != nullptr && n_kv_t > 0) ? __ldg(dkb) : 1.0f;
     for (int j = 0; j < n_kv_t; ++j) {
       const float s_log2 = s_q * dk_next;
       if (QK_FP8 && dkb != nullptr && j + 1 < n_kv_t) dk_next = __ldg(dkb + j + 1);  // in flight during this step
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], j & 1, &abort_flag, st, 30 + t));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[t], sc & 1u, &abort_flag, st, 30 + t));
+      ++sc;
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
@@ -703,7 +743,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_p[t]);  // one arrival per warp
     }
-    if (ok && n_kv_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], 0, &abort_flag, st, 40 + t));
+    if (ok && n_kv_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], oc & 1u, &abort_flag, st, 40 + t));
+    if (n_kv_t > 0) ++oc;
     const bool in_range = qrow < p.Nq;
     if constexpr (PARTIAL) {
       if (ok) {
@@ -757,6 +798,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (in_range && p.lse != nullptr)
         p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     }
+    }  // items
     }  // not DEC
   }
 
