@@ -107,6 +107,11 @@ struct FwdParams {
   // smaller than n_items).
   int unit_base;
   int n_items;
+  // snake (causal, persistent): item i is query block rank i / BH of head i % BH,
+  // blocks ranked heaviest first across all heads, and CTA c takes item
+  // r * gridDim.x + c in even rounds r, r * gridDim.x + gridDim.x - 1 - c in odd
+  // ones, which balances work that decreases with i
+  int snake;
 };
 
 // One work item of a CTA: head, key split, first query row, first key tile and
@@ -469,13 +474,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // has no row (past Nq), else up to the tile holding its last visible key, so a
   // causal tile never spends a step on keys entirely in its future. The CTA
   // streams the most any tile needs.
+  // The CTA's items: blockIdx.x + r * gridDim.x in round r, or the snake order.
+  auto next_item = [&](int r) {
+    const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return r * g + ((p.snake && (r & 1)) ? g - 1 - c : c);
+  };
+  auto first_item = [&]() { return next_item(0); };
   auto item_at = [&](int it) {
     FwdItem w;
     const int n_split = PARTIAL ? p.n_split : 1;
     const int unit = p.unit_base + (PARTIAL ? it / n_split : it);  // query block bh * n_qb + qb
     w.sp = PARTIAL ? it % n_split : 0;
-    w.bh = unit / p.n_qb;
-    int qb = unit % p.n_qb;
+    w.bh = p.snake ? unit % p.BH : unit / p.n_qb;
+    int qb = p.snake ? unit / p.BH : unit % p.n_qb;
     if (CAUSAL) qb = p.n_qb - 1 - qb;
     w.q0 = qb * NQ * C::BM;
     w.kt0 = PARTIAL ? w.sp * p.split_tiles : 0;
@@ -530,7 +541,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmV);
       int pos = 0, iter = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x, ++iter) {
+      for (int it = first_item(); it < p.n_items && ok; it = next_item(iter + 1), ++iter) {
       const FwdItem w = item_at(it);
       const int bh = w.bh, q0 = w.q0, kt0 = w.kt0, n_kv = w.n_kv;
       // the previous item's S MMAs read sQ until they complete
@@ -581,7 +592,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int pos = 0, iter = 0;
       uint32_t pc0 = 0, pc1 = 0;  // P-barrier phases waited, per query tile
       bool ok = true;
-      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x, ++iter) {
+      for (int it = first_item(); it < p.n_items && ok; it = next_item(iter + 1), ++iter) {
       const FwdItem w = item_at(it);
       const int n_kv = w.n_kv;
       auto n_kv_at = [&](int t) { return t == 0 ? w.n_kv0 : w.n_kv1; };
@@ -653,7 +664,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int t = static_cast<int>(warp >> 2);
     uint32_t sc = 0, oc = 0;  // phases of bar_s[t] and bar_o[t] waited
     bool ok = true;
-    for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+    for (int round = 0, it = first_item(); it < p.n_items && ok; it = next_item(++round)) {
     const FwdItem w = item_at(it);
     const int bh = w.bh, q0 = w.q0, kt0 = w.kt0, sp = w.sp;
     const uint32_t lane_base = (warp & 3u) * 32u;

@@ -68,6 +68,10 @@ int device_sms();  // SM count of the current device (cached)
 #define FA_PERSISTENT 1
 #endif
 constexpr bool kPersistent = FA_PERSISTENT != 0;
+#ifndef FA_PERSIST_CAUSAL
+#define FA_PERSIST_CAUSAL 1
+#endif
+constexpr bool kPersistCausal = FA_PERSIST_CAUSAL != 0;
 
 template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC>
 fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
@@ -124,14 +128,18 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   const long long items = units * (PARTIAL ? a.n_split : 1);
   if (items < 1) return FA_OK;
   p.n_items = static_cast<int>(items);
-  // Persistent when not causal: at most one CTA per SM, each looping over work
-  // items, so the next item's Q load and first S MMA overlap the current item's
-  // last steps and epilogue (+1-6% on B200). Causal items differ in length, and
-  // a fixed round-robin over them balances worse than the hardware's dynamic
-  // dispatch of one CTA per item (-5-11%), so causal launches stay one item per
-  // CTA, as does the decode layout (its epilogue uses the K/V ring).
+  // Persistent: at most one CTA per SM, each looping over work items, so the
+  // next item's Q load and first S MMA overlap the current item's last steps and
+  // epilogue (non-causal: +1-6% on B200). Causal items differ in length: a plain
+  // round-robin over them balanced worse than the hardware's dispatch of one CTA
+  // per item (-5-11%), but ranking the query blocks heaviest first across all
+  // heads and dealing them in snake order (p.snake) beats it (+11-22%). Split-key
+  // causal launches and the decode layout (whose epilogue uses the K/V ring) run
+  // one item per CTA.
   long long grid = items;
-  if (kPersistent && !DEC && !CAUSAL) {
+  const bool persist = kPersistent && !DEC && (!CAUSAL || (kPersistCausal && !PARTIAL));
+  p.snake = (persist && CAUSAL) ? 1 : 0;
+  if (persist) {
     const long long sms = device_sms();
     if (grid > sms) grid = sms;
   }
