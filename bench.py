@@ -248,10 +248,19 @@ class Step:
         q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
         self.signs = fa_inputs.hadamard_signs(D, seed).cuda()
         self.q_h, self.k_h, self.v_h = (t.pin_memory() for t in (q, k, v))
-        self.q, self.k, self.v = (t.cuda() for t in (q, k, v))
         shp = (B, H, N, D)
-        self.o = [torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
-        self.lse = [torch.empty((B, H, N), dtype=torch.float32, device="cuda") for _ in range(3)]
+        # two sets of device inputs and outputs, so that pipelined end-to-end steps
+        # can copy one set while computing on the other (the timed device-only
+        # steps use set 0)
+        self.bufs = []
+        for _ in range(2):
+            self.bufs.append({
+                "q": q.cuda(), "k": k.cuda(), "v": v.cuda(),
+                "o": [torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(3)],
+                "lse": [torch.empty((B, H, N), dtype=torch.float32, device="cuda") for _ in range(3)],
+            })
+        self.q, self.k, self.v = self.bufs[0]["q"], self.bufs[0]["k"], self.bufs[0]["v"]
+        self.o, self.lse = self.bufs[0]["o"], self.bufs[0]["lse"]
         self.q8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
         self.k8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
         self.desc = torch.empty(2, dtype=torch.float32, device="cuda")
@@ -264,35 +273,39 @@ class Step:
     def flush_l2(self):
         self.flush_buf.zero_()
 
-    def run(self, ev=None):
+    def run(self, ev=None, b=0):
         fa = self.fa
+        q, k, v, o, lse = (self.bufs[b][n] for n in ("q", "k", "v", "o", "lse"))
         if ev is not None:
             ev[0].record()
-        fa.fwd(self.q, self.k, self.v, causal=False, out=self.o[0], lse=self.lse[0])
+        fa.fwd(q, k, v, causal=False, out=o[0], lse=lse[0])
         if ev is not None:
             ev[1].record()
-        fa.fwd(self.q, self.k, self.v, causal=True, out=self.o[1], lse=self.lse[1])
+        fa.fwd(q, k, v, causal=True, out=o[1], lse=lse[1])
         if ev is not None:
             ev[2].record()
-        fa.hadamard_quant(self.q, rotate=True, signs=self.signs, out=self.q8, descale=self.desc[0:1])
-        fa.hadamard_quant(self.k, rotate=True, signs=self.signs, out=self.k8, descale=self.desc[1:2])
+        fa.hadamard_quant(q, rotate=True, signs=self.signs, out=self.q8, descale=self.desc[0:1])
+        fa.hadamard_quant(k, rotate=True, signs=self.signs, out=self.k8, descale=self.desc[1:2])
         if ev is not None:
             ev[3].record()
-        fa.fwd(self.q8, self.k8, self.v, causal=False, qk_descale=self.desc, out=self.o[2], lse=self.lse[2])
+        fa.fwd(self.q8, self.k8, v, causal=False, qk_descale=self.desc, out=o[2], lse=lse[2])
         if ev is not None:
             ev[4].record()
 
-    def run_e2e(self):
-        """The step through the same public calls with host buffers: pinned
-        host -> device copies of Q, K, V, the step, device -> host copies of
-        every O and LSE."""
-        self.q.copy_(self.q_h, non_blocking=True)
-        self.k.copy_(self.k_h, non_blocking=True)
-        self.v.copy_(self.v_h, non_blocking=True)
-        self.run()
+    # End to end, through the same public calls with host buffers: pinned
+    # host -> device copies of Q, K, V, the step, device -> host copies of every
+    # O and LSE, each part on the current stream, for buffer set b.
+    def h2d(self, b):
+        for n, h in (("q", self.q_h), ("k", self.k_h), ("v", self.v_h)):
+            self.bufs[b][n].copy_(h, non_blocking=True)
+
+    def compute(self, b):
+        self.run(b=b)
+
+    def d2h(self, b):
         for i in range(3):
-            self.o_h[i].copy_(self.o[i], non_blocking=True)
-            self.lse_h[i].copy_(self.lse[i], non_blocking=True)
+            self.o_h[i].copy_(self.bufs[b]["o"][i], non_blocking=True)
+            self.lse_h[i].copy_(self.bufs[b]["lse"][i], non_blocking=True)
 
     @property
     def h2d_bytes(self):
@@ -318,6 +331,7 @@ class DecodeStep:
         q, k, v = fa_inputs.qkv_decode(self.B, self.H, self.Nq, self.Nk, self.d, seed)
         self.q_h = q.pin_memory()
         self.q, self.k, self.v = (t.cuda() for t in (q, k, v))
+        self.qs = [self.q, q.cuda()]  # two query buffers for pipelined end-to-end steps
         self.n_split = fa.splitkv_splits(self.B, self.H, self.Nq, self.Nk, self.d)
         rows = (self.B, self.H, self.Nq)
         self.o_part = torch.empty((self.n_split, *rows, self.d), dtype=torch.float32, device="cuda")
@@ -349,10 +363,17 @@ class DecodeStep:
         if ev is not None:
             ev[2].record()
 
-    def run_e2e(self):
-        """Q copied in from pinned host memory, the step, O and LSE copied out."""
-        self.q.copy_(self.q_h, non_blocking=True)
-        self.run()
+    # End to end: Q copied in from pinned host memory, the step, O and LSE
+    # copied out (the K/V cache stays on the device).
+    def h2d(self, b):
+        self.qs[b].copy_(self.q_h, non_blocking=True)
+
+    def compute(self, b):
+        fa = self.fa
+        fa.fwd_partial(self.qs[b], self.k, self.v, n_split=self.n_split, o_part=self.o_part, lse_part=self.lse_part)
+        fa.lse_merge(self.o_part, self.lse_part, out=self.o, lse=self.lse)
+
+    def d2h(self, b):
         self.o_h.copy_(self.o, non_blocking=True)
         self.lse_h.copy_(self.lse, non_blocking=True)
 
@@ -409,21 +430,54 @@ def time_steps(step, graph, steps: int, warmup: int, world: int):
 
 
 def time_e2e(step, steps: int, warmup: int, world: int):
-    for _ in range(warmup):
-        step.run_e2e()
+    """End-to-end steps, pipelined as a serving loop would run them: three CUDA
+    streams (host -> device copies, compute, device -> host copies) and two
+    sets of device buffers, so that step i+1's inputs travel in and step i-1's
+    results travel out while step i computes. Every step still copies all of its
+    inputs in and all of its results out. Returns ms per step over the timed
+    steps (events on the current stream, which waits for all three)."""
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def one(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_c[b])  # step i-2 has finished reading set b's inputs
+            step.h2d(b)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_c):
+            s_c.wait_event(ev_in[b])
+            if i >= 2:
+                s_c.wait_event(ev_out[b])  # step i-2's results in set b are copied out
+            step.compute(b)
+            ev_c[b].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c[b])
+            step.d2h(b)
+            ev_out[b].record(s_out)
+
+    for i in range(warmup):
+        one(i)
     torch.cuda.synchronize()
     dist_barrier(world)
-    total = 0.0
-    for _ in range(steps):
-        step.flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step.run_e2e()
-        e1.record()
-        e1.synchronize()
-        total += e0.elapsed_time(e1)
+    step.flush_l2()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for s in (s_in, s_c, s_out):
+        s.wait_stream(cur)
+    for i in range(steps):
+        one(i)
+    for s in (s_in, s_c, s_out):
+        cur.wait_stream(s)
+    e1.record(cur)
+    e1.synchronize()
     dist_barrier(world)
-    return total / steps
+    return e0.elapsed_time(e1) / steps
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -503,7 +557,7 @@ def main():
     graph = capture_step(step)
     with ClockSampler(local) as clk:
         step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
-    e2e_ms = time_e2e(step, max(3, args.steps // 4), 3, world)
+    e2e_ms = time_e2e(step, max(8, args.steps // 2), 3, world)
     ms_local = statistics.mean(step_ms)
     ms = dist_max(ms_local, world)
     e2e_ms = dist_max(e2e_ms, world)
@@ -534,7 +588,9 @@ def main():
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "peak_source": f"{peak_src} cuBLAS bf16 (burst)"},
             "e2e": {"value": world * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
-                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes},
+                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
+                    "note": "steps pipelined over three CUDA streams (copy in, compute, copy out) with two sets of "
+                            "device buffers; every step copies its inputs in and its results out"},
             "gpu_launches": step.launches_per_step * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
@@ -553,7 +609,7 @@ def run_decode(args, world: int, rank: int):
     graph = capture_step(step)
     with ClockSampler(torch.cuda.current_device()) as clk:
         step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
-    e2e_ms = dist_max(time_e2e(step, max(3, args.steps // 4), 3, world), world)
+    e2e_ms = dist_max(time_e2e(step, max(8, args.steps // 2), 3, world), world)
     ms = dist_max(statistics.mean(step_ms), world)
     comp = [dist_max(statistics.mean(p[j] for p in per), world) for j in range(2)]
     peaks, peak_src = load_peaks()
@@ -581,7 +637,8 @@ def run_decode(args, world: int, rank: int):
                          "peak_source": f"{peak_src} HBM copy bandwidth"},
             "e2e": {"value": world * step.bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
-                    "note": "K/V cache resident on the device; Q in, O and LSE out per step"},
+                    "note": "K/V cache resident on the device; Q in, O and LSE out per step; steps pipelined over "
+                            "three CUDA streams (copy in, compute, copy out)"},
             "gpu_launches": step.launches_per_step * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
