@@ -3,7 +3,7 @@
 One step = one pass of the whole hot path over one batch of synthetic input of
 the B=4, H=16, N=2048, d=128 workload (Q, K, V ~ N(0,1) bf16, scale 1/sqrt(128)):
   1. BF16 forward, non-causal;   2. BF16 forward, causal;
-  3. Hadamard rotate + e4m3 quantise of Q and of K;   4. e4m3-QK forward, non-causal.
+  3. Hadamard rotate + e4m3 quantise of Q and K (one launch, a scale each);   4. e4m3-QK forward, non-causal.
 Metric: attention TFLOPS = sum of 4*B*H*N^2*d (halved when causal) over the
 three forward passes / step time. L2 (126 MB) is flushed between steps by
 writing a 512 MB buffer outside the timed events, since the inputs (100 MB)
@@ -267,7 +267,7 @@ class Step:
         self.o_h = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
         self.lse_h = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(3)]
         self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-        self.launches_per_step = 5  # 3 attention kernels + 2 one-launch quantisations
+        self.launches_per_step = 4  # 3 attention kernels + 1 quantisation of Q and K
         self.groups = 4  # breakdown: bf16 nc, bf16 causal, quantise Q+K, e4m3 nc
 
     def flush_l2(self):
@@ -284,8 +284,7 @@ class Step:
         fa.fwd(q, k, v, causal=True, out=o[1], lse=lse[1])
         if ev is not None:
             ev[2].record()
-        fa.hadamard_quant(q, rotate=True, signs=self.signs, out=self.q8, descale=self.desc[0:1])
-        fa.hadamard_quant(k, rotate=True, signs=self.signs, out=self.k8, descale=self.desc[1:2])
+        fa.hadamard_quant_multi([q, k], rotate=True, signs=self.signs, outs=[self.q8, self.k8], descales=self.desc)
         if ev is not None:
             ev[3].record()
         fa.fwd(self.q8, self.k8, v, causal=False, qk_descale=self.desc, out=o[2], lse=lse[2])

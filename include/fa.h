@@ -179,6 +179,24 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
                             const float* signs, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_hadamard_quant_multi — fa_hadamard_quant for up to 8 tensors of one shape
+ * (for example Q and K) in one launch, each with its own scale: the same codes
+ * and descales as one call per tensor, with one grid-wide barrier in place of one
+ * per tensor.
+ *
+ * Defined by: as fa_hadamard_quant.
+ * xs, outs  host arrays of `ntensors` device pointers: bf16 inputs [rows][d] and
+ *           e4m3 outputs [rows][d], each 16-byte aligned (may be NULL if rows = 0).
+ * descales  device, ntensors fp32 (tensor i's descale at descales[i]).
+ * ntensors  1..8. rows, d, rotate, signs, workspace: as fa_hadamard_quant (the
+ *           workspace holds the amax words and the barrier counter).
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, float* descales, int ntensors,
+                                  int64_t rows, int d, int rotate, const float* signs, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * fa_hadamard_quant_blocks — rotate (optionally) and quantise one tensor to e4m3
  * with one scale per block of 128 consecutive rows of each head (the attention
  * kernel's query and key tiles), in one pass over the input.

@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     fwd_splitkv,
     hadamard_quant,
     hadamard_quant_blocks,
+    hadamard_quant_multi,
     library_path,
     load_library,
     lse_merge,
@@ -22,4 +23,4 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = ["fwd", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
-           "hadamard_quant_blocks", "device_status", "load_library", "library_path", "FaError"]
+           "hadamard_quant_blocks", "hadamard_quant_multi", "device_status", "load_library", "library_path", "FaError"]

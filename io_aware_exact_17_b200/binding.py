@@ -72,6 +72,8 @@ def load_library():
         lib.fa_lse_merge.restype = i
         lib.fa_hadamard_quant_blocks.argtypes = [vp, vp, vp, i, i, i, i, vp, vp]
         lib.fa_hadamard_quant_blocks.restype = i
+        lib.fa_hadamard_quant_multi.argtypes = [vp, vp, vp, i, i64, i, i, vp, vp, sz, vp]
+        lib.fa_hadamard_quant_multi.restype = i
         _lib = lib
         return lib
 
@@ -321,6 +323,38 @@ def hadamard_quant(x, rotate: bool = True, signs=None, out=None, descale=None, w
                                    workspace.numel() * workspace.element_size(), _stream(x.device))
     _check(rc, "fa_hadamard_quant")
     return out, descale
+
+
+def hadamard_quant_multi(xs, rotate: bool = True, signs=None, outs=None, descales=None, workspace=None):
+    """Rotate (optionally) and quantise up to 8 bf16 tensors of one shape (e.g.
+    Q and K) in one launch through ``fa_hadamard_quant_multi``, each with its own
+    scale. Returns ``(codes, descales)``: a list of uint8 code tensors and a CUDA
+    fp32 tensor of one descale per input; the same as ``hadamard_quant`` per
+    tensor."""
+    xs = [x.contiguous() for x in xs]
+    _require_cuda(*xs)
+    lib = load_library()
+    if not xs or any(x.dtype != torch.bfloat16 or x.shape != xs[0].shape for x in xs):
+        raise FaError("xs must be bf16 tensors of one shape")
+    d = xs[0].shape[-1]
+    rows = xs[0].numel() // d if d else 0
+    if outs is None:
+        outs = [torch.empty(x.shape, dtype=torch.uint8, device=x.device) for x in xs]
+    if descales is None:
+        descales = torch.empty(len(xs), dtype=torch.float32, device=xs[0].device)
+    if workspace is None:
+        workspace = _workspace(xs[0].device)
+    if signs is not None:
+        signs = signs.to(device=xs[0].device, dtype=torch.float32).contiguous()
+    n = len(xs)
+    x_arr = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
+    o_arr = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    with torch.cuda.device(xs[0].device):
+        rc = lib.fa_hadamard_quant_multi(x_arr, o_arr, _ptr(descales), n, rows, d, int(bool(rotate)),
+                                         _ptr(signs) if (rotate and signs is not None) else None, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(xs[0].device))
+    _check(rc, "fa_hadamard_quant_multi")
+    return outs, descales
 
 
 def hadamard_quant_blocks(x, rotate: bool = True, signs=None, out=None, descales=None):

@@ -307,13 +307,14 @@ fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t row
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// Both quantisation passes in one cooperative launch (quant_fused_kernel): the
-// workspace holds the amax word and the grid barrier's counter, zeroed here.
+// Both quantisation passes in one cooperative launch (quant_fused_kernel) for
+// the tensors of `b`: the workspace holds their amax words and the grid
+// barrier's counter, zeroed here.
 template <int D>
-fa_status launch_quant_fused(const void* x, void* out, float* descale_out, int64_t rows, int rotate,
+fa_status launch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int rotate,
                              const float* signs, unsigned int* ws, cudaStream_t stream) {
   using FC = fa::FusedCfg<D>;
-  if (cudaMemsetAsync(ws, 0, 2 * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, (b.n + 1) * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
   auto kernel = rotate ? fa::quant_fused_kernel<D, true> : fa::quant_fused_kernel<D, false>;
   // Co-resident blocks per SM and SM count, looked up once per device (this is
   // host time in front of a ~10 us kernel).
@@ -329,18 +330,26 @@ fa_status launch_quant_fused(const void* x, void* out, float* descale_out, int64
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, fa::kFusedThreads, 0) != cudaSuccess)
     return FA_ERR_CUDA;
   if (per_sm < 1 || sms < 1) return FA_ERR_CUDA;
-  const int64_t steps = (rows + FC::RPW - 1) / FC::RPW;  // warp-steps of work
+  const int64_t steps = (rows + FC::RPW - 1) / FC::RPW;  // warp-steps of work per tensor
   int64_t blocks = (steps + fa::kFusedThreads / 32 - 1) / (fa::kFusedThreads / 32);
   const int64_t cap = static_cast<int64_t>(per_sm) * sms;  // all blocks co-resident
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  uint8_t* ob = static_cast<uint8_t*>(out);
-  void* args[] = {&xb, &ob, &rows, &signs, &ws, &descale_out};
+  fa::QuantBatch bb = b;
+  void* args[] = {&bb, &rows, &signs, &ws, &descale_out};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(static_cast<unsigned>(blocks)),
                                   dim3(fa::kFusedThreads), args, 0, stream) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
+}
+
+fa_status dispatch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int d, int rotate,
+                               const float* signs, unsigned int* ws, cudaStream_t s) {
+  switch (d) {
+    case 64: return launch_quant_fused<64>(b, descale_out, rows, rotate, signs, ws, s);
+    case 128: return launch_quant_fused<128>(b, descale_out, rows, rotate, signs, ws, s);
+    default: return launch_quant_fused<256>(b, descale_out, rows, rotate, signs, ws, s);
+  }
 }
 
 template <int D>
@@ -364,6 +373,7 @@ fa_status dispatch_merge(const float* o_part, const float* lse_part, int n_part,
     default: return launch_merge<256>(o_part, lse_part, n_part, rows, o, lse, s);
   }
 }
+
 
 }  // namespace
 
@@ -463,13 +473,34 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
     return FA_ERR_ALIGNMENT;
   if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
   const float* sg = rotate ? signs : nullptr;
-  unsigned int* amax = static_cast<unsigned int*>(workspace);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch (d) {
-    case 64: return launch_quant_fused<64>(x, out, descale_out, rows, rotate, sg, amax, s);
-    case 128: return launch_quant_fused<128>(x, out, descale_out, rows, rotate, sg, amax, s);
-    default: return launch_quant_fused<256>(x, out, descale_out, rows, rotate, sg, amax, s);
+  fa::QuantBatch b = {};
+  b.x[0] = static_cast<const __nv_bfloat16*>(x);
+  b.out[0] = static_cast<uint8_t*>(out);
+  b.n = 1;
+  return dispatch_quant_fused(b, descale_out, rows, d, rotate, sg, static_cast<unsigned int*>(workspace),
+                              static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, float* descales, int ntensors,
+                                  int64_t rows, int d, int rotate, const float* signs, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (xs == nullptr || outs == nullptr || descales == nullptr || workspace == nullptr) return FA_ERR_INVALID_ARG;
+  if (ntensors < 1 || ntensors > fa::kQuantBatch) return FA_ERR_INVALID_ARG;
+  if (rows < 0 || rows > (static_cast<int64_t>(1) << 40) || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < FA_QUANT_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned(descales, 4) || !aligned(workspace, 16)) return FA_ERR_ALIGNMENT;
+  if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
+  fa::QuantBatch b = {};
+  for (int i = 0; i < ntensors; ++i) {
+    if (rows > 0 && (xs[i] == nullptr || outs[i] == nullptr)) return FA_ERR_INVALID_ARG;
+    if (!aligned(xs[i], 16) || !aligned(outs[i], 16)) return FA_ERR_ALIGNMENT;
+    b.x[i] = static_cast<const __nv_bfloat16*>(xs[i]);
+    b.out[i] = static_cast<uint8_t*>(outs[i]);
   }
+  b.n = ntensors;
+  return dispatch_quant_fused(b, descales, rows, d, rotate, rotate ? signs : nullptr,
+                              static_cast<unsigned int*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int d, int rotate,

@@ -288,51 +288,68 @@ __device__ __forceinline__ void hadamard_rotate32(float (&v)[32], int lr, const 
   }
 }
 
-// ws[0]: amax bits, ws[1]: arrival counter of the grid barrier; both zero at launch.
+// Up to kQuantBatch tensors of one shape, rotated and quantised in one launch,
+// each with its own scale.
+constexpr int kQuantBatch = 8;
+struct QuantBatch {
+  const __nv_bfloat16* x[kQuantBatch];
+  uint8_t* out[kQuantBatch];
+  int n;
+};
+
+// ws[0 .. n-1]: amax bits of each tensor, ws[n]: arrival counter of the grid
+// barrier; all zero at launch. descale_out[i]: tensor i's descale.
 template <int D, bool ROT>
-__global__ void __launch_bounds__(kFusedThreads)
-quant_fused_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ out, int64_t rows,
-                   const float* __restrict__ signs, unsigned int* ws, float* descale_out) {
+__global__ void __launch_bounds__(kFusedThreads, 3)
+quant_fused_kernel(const QuantBatch b, int64_t rows, const float* __restrict__ signs, unsigned int* ws,
+                   float* descale_out) {
   DevStatus* st = &g_fa_status;
   using C = FusedCfg<D>;
   const int lane = threadIdx.x & 31;
   const int lr = lane % C::L, sub = lane / C::L;
   const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * kFusedThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kFusedThreads) >> 5;
-  // pass 1: amax of the rotated tensor
-  float m = 0.f;
-  for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
-    const int64_t row = w * C::RPW + sub;
-    float v[32];
-    if (row < rows) {
-      load_bf16x32<D>(x + row * D, lr, v);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = 0.f;
-    }
-    if (ROT) hadamard_rotate32<D>(v, lr, signs);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(v[e]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ float warp_max[kFusedThreads / 32];
-  __shared__ unsigned int amax_sh;
-  if (lane == 0) warp_max[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = warp_max[0];
+  __shared__ unsigned int amax_sh[kQuantBatch];
+  // pass 1: amax of each rotated tensor
+#pragma unroll 1
+  for (int t = 0; t < b.n; ++t) {
+    const __nv_bfloat16* x = b.x[t];
+    float m = 0.f;
+    for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
+      const int64_t row = w * C::RPW + sub;
+      float v[32];
+      if (row < rows) {
+        load_bf16x32<D>(x + row * D, lr, v);
+      } else {
 #pragma unroll
-    for (int i = 1; i < kFusedThreads / 32; ++i) b = fmaxf(b, warp_max[i]);
-    atomicMax(&ws[0], __float_as_uint(b));
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      }
+      if (ROT) hadamard_rotate32<D>(v, lr, signs);
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) m = fmax3(m, fabsf(v[e]), fabsf(v[e + 1]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float bm = warp_max[0];
+#pragma unroll
+      for (int i = 1; i < kFusedThreads / 32; ++i) bm = fmaxf(bm, warp_max[i]);
+      atomicMax(&ws[t], __float_as_uint(bm));
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
     // Grid-wide barrier: every block is resident (cooperative launch). The wait
     // is bounded; if it runs out the status word records it and the block goes on.
     __threadfence();
-    atomicAdd(&ws[1], 1u);
+    atomicAdd(&ws[b.n], 1u);
     const unsigned long long t0 = globaltimer_ns();
     unsigned int arrived;
     for (;;) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + 1) : "memory");
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + b.n) : "memory");
       if (arrived >= gridDim.x) break;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         if (atomicCAS(&st->code, 0u, 5u) == 0u) {
@@ -343,35 +360,42 @@ quant_fused_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
       }
       __nanosleep(64);
     }
-    unsigned int a;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(ws) : "memory");
-    amax_sh = a;
+    for (int t = 0; t < b.n; ++t) {
+      unsigned int a;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(ws + t) : "memory");
+      amax_sh[t] = a;
+    }
   }
   __syncthreads();
-  // pass 2: quantise (the tensor is re-read, mostly from L2)
-  const float amax = __uint_as_float(amax_sh);
-  const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *descale_out = amax > 0.f ? amax / 448.0f : 1.0f;
-  for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
-    const int64_t row = w * C::RPW + sub;
-    float v[32];
-    if (row < rows) {
-      load_bf16x32<D>(x + row * D, lr, v);
-    } else {
+  // pass 2: quantise (each tensor is re-read, mostly from L2)
+#pragma unroll 1
+  for (int t = 0; t < b.n; ++t) {
+    const __nv_bfloat16* x = b.x[t];
+    uint8_t* out = b.out[t];
+    const float amax = __uint_as_float(amax_sh[t]);
+    const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) descale_out[t] = amax > 0.f ? amax / 448.0f : 1.0f;
+    for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
+      const int64_t row = w * C::RPW + sub;
+      float v[32];
+      if (row < rows) {
+        load_bf16x32<D>(x + row * D, lr, v);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = 0.f;
-    }
-    if (ROT) hadamard_rotate32<D>(v, lr, signs);
-    uint32_t q[8];
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      }
+      if (ROT) hadamard_rotate32<D>(v, lr, signs);
+      uint32_t q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      q[i] = static_cast<uint32_t>(pack_e4m3x2(v[4 * i] * scale, v[4 * i + 1] * scale)) |
-             (static_cast<uint32_t>(pack_e4m3x2(v[4 * i + 2] * scale, v[4 * i + 3] * scale)) << 16);
-    if (row < rows) {
-      // chunk c of the row (8 codes, 8 bytes) goes to out[row*D + 8c]
-      uint2* dst = reinterpret_cast<uint2*>(out + row * D);
+      for (int i = 0; i < 8; ++i)
+        q[i] = static_cast<uint32_t>(pack_e4m3x2(v[4 * i] * scale, v[4 * i + 1] * scale)) |
+               (static_cast<uint32_t>(pack_e4m3x2(v[4 * i + 2] * scale, v[4 * i + 3] * scale)) << 16);
+      if (row < rows) {
+        // chunk c of the row (8 codes, 8 bytes) goes to out[row*D + 8c]
+        uint2* dst = reinterpret_cast<uint2*>(out + row * D);
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
+        for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
+      }
     }
   }
 }

@@ -132,6 +132,23 @@ def test_partial_and_merge_argument_errors(lib):
     assert merge(o=MIS) == binding.FA_ERR_ALIGNMENT
 
 
+def test_quant_multi_argument_errors(lib):
+    arr = (ctypes.c_void_p * 9)(*([A] * 9))
+    mq = lambda **kw: lib.fa_hadamard_quant_multi(kw.get("xs", arr), kw.get("outs", arr), kw.get("ds", A),
+                                                  kw.get("n", 2), kw.get("rows", 4), kw.get("d", 128),
+                                                  kw.get("rot", 1), None, kw.get("ws", A), kw.get("wsb", 256), None)
+    assert mq(xs=None) == binding.FA_ERR_INVALID_ARG
+    assert mq(ws=None) == binding.FA_ERR_INVALID_ARG
+    assert mq(n=0) == binding.FA_ERR_INVALID_ARG
+    assert mq(n=9) == binding.FA_ERR_INVALID_ARG
+    assert mq(wsb=8) == binding.FA_ERR_INVALID_ARG
+    assert mq(rows=-1) == binding.FA_ERR_INVALID_ARG
+    assert mq(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert mq(ds=A + 2) == binding.FA_ERR_ALIGNMENT
+    mis = (ctypes.c_void_p * 2)(A, MIS)
+    assert mq(xs=mis) == binding.FA_ERR_ALIGNMENT
+
+
 def test_block_quant_argument_errors(lib):
     bq = lambda **kw: lib.fa_hadamard_quant_blocks(kw.get("x", A), kw.get("out", A), kw.get("ds", A), kw.get("BH", 2),
                                                    kw.get("N", 300), kw.get("d", 128), kw.get("rot", 1), None, None)

@@ -61,6 +61,24 @@ def test_quant_matches_oracle(d, rotate, rows):
         _quant_check(x, True, inputs.hadamard_signs(d, seed=rows))
 
 
+@pytest.mark.parametrize("n", [1, 2, 3])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_quant_multi_equals_one_call_per_tensor(n, rotate):
+    # tensors of very different ranges, one launch, one scale each
+    xs = []
+    for i in range(n):
+        q, _, _ = inputs.qkv_normal(2, 3, 700, 128, 70 + i)
+        xs.append((q.float() * 10.0 ** (2 * i - 2)).to(torch.bfloat16).cuda())
+    signs = inputs.hadamard_signs(128, 70).cuda() if rotate else None
+    codes, ds = fa.hadamard_quant_multi(xs, rotate=rotate, signs=signs)
+    torch.cuda.synchronize()
+    for i, x in enumerate(xs):
+        c1, d1 = fa.hadamard_quant(x, rotate=rotate, signs=signs)
+        torch.cuda.synchronize()
+        assert torch.equal(codes[i], c1)
+        assert float(ds[i].item()) == float(d1.item())
+
+
 def test_quant_zero_and_empty():
     codes, ds = fa.hadamard_quant(torch.zeros(5, 128, dtype=torch.bfloat16, device="cuda"))
     assert float(ds.item()) == 1.0 and int(codes.abs().sum()) == 0
