@@ -101,11 +101,9 @@ struct FwdParams {
   int n_split;               // key splits per head (1: all keys)
   int split_tiles;           // key tiles per split
   float scale_log2;          // scale * log2(e)
-  // Work items: the query blocks unit_base, unit_base + 1, ... (query block
-  // = bh * n_qb + qb), times n_split key blocks each in partial mode; n_items of
-  // them. CTA c takes items c, c + gridDim.x, ... (persistent when the grid is
-  // smaller than n_items).
-  int unit_base;
+  // Work items: the query blocks (query block = bh * n_qb + qb), times n_split
+  // key blocks each in partial mode; n_items of them. CTA c takes items c,
+  // c + gridDim.x, ... (persistent when the grid is smaller than n_items).
   int n_items;
   // snake (causal, persistent): item i is query block rank i / BH of head i % BH,
   // blocks ranked heaviest first across all heads, and CTA c takes item
@@ -181,28 +179,27 @@ __device__ __forceinline__ void mask_chunk32(uint32_t* s, int kbase, int kmax) {
 // chunk c is computed). P is packed in place: chunk c's 16 bf16 pairs go to
 // s[16c .. 16c+15], scores already consumed (chunk c/2's) and never the target of
 // a pending load, so only 128 registers are live. Returns the fp32 weight sum,
-// the sum that normalises O and, with WITH_MAX, the max of the raw scores.
+// and the sum that normalises O.
 //
 // The normalising sum is the sum of the bf16-rounded weights P holds when some
 // key of the tile is masked (EMU false: the row's last tile, which holds every
 // key of a row with few keys), else the fp32 sum: over a full tile of 128 keys
 // the rounding errors of P average out to about 2^-9 / sqrt(128) of the sum, and
 // skipping the rounded sum saves three of the eight instructions per key pair.
-template <bool EMU, bool WITH_MAX>
+template <bool EMU>
 __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
-                                            int kbase, int kmax, bool masked, float& sum_e, float& sum_r,
-                                            float& raw_max) {
+                                            int kbase, int kmax, bool masked, float& sum_e, float& sum_r) {
   const uint64_t s2 = f2_pack(s_log2, s_log2);
   const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
   uint64_t acc_e[2] = {0ull, 0ull}, acc_r[2] = {0ull, 0ull};
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  float mx[4];  // unused: no running max
   tmem_ld32(tS + 0, &s[0]);
   tmem_wait_ld_dep32(&s[0]);
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     if (ch < 3) tmem_ld32(tS + 32 * (ch + 1), &s[32 * (ch + 1)]);
     if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
-    exp_chunk32<EMU, WITH_MAX, !EMU>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
+    exp_chunk32<EMU, false, !EMU>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
     if (ch < 3) tmem_wait_ld_dep32(&s[32 * (ch + 1)]);
   }
   float e0, e1, e2, e3, r0, r1, r2, r3;
@@ -212,18 +209,15 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_lo
   f2_unpack(acc_r[1], r2, r3);
   sum_e = (e0 + e1) + (e2 + e3);
   sum_r = EMU ? sum_e : (r0 + r1) + (r2 + r3);
-  if (WITH_MAX) raw_max = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
 // `masked` must be warp-uniform: both paths issue tcgen05.ld.
-template <bool WITH_MAX>
-__device__ __forceinline__ void softmax_row_dispatch(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
-                                                     int kbase, int kmax, bool masked, float& se, float& sr,
-                                                     float& mx) {
+__device__ __forceinline__ void softmax_row_dispatch(uint32_t tS, uint32_t* s, float s_log2, float m_ref, int kbase,
+                                                     int kmax, bool masked, float& se, float& sr) {
   if (masked)
-    softmax_row<false, WITH_MAX>(tS, s, s_log2, m_ref, kbase, kmax, true, se, sr, mx);
+    softmax_row<false>(tS, s, s_log2, m_ref, kbase, kmax, true, se, sr);
   else
-    softmax_row<true, WITH_MAX>(tS, s, s_log2, m_ref, kbase, kmax, false, se, sr, mx);
+    softmax_row<true>(tS, s, s_log2, m_ref, kbase, kmax, false, se, sr);
 }
 
 // Raw-score max of one row of S (first tile only, before any reference exists).
@@ -483,7 +477,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   auto item_at = [&](int it) {
     FwdItem w;
     const int n_split = PARTIAL ? p.n_split : 1;
-    const int unit = p.unit_base + (PARTIAL ? it / n_split : it);  // query block bh * n_qb + qb
+    const int unit = PARTIAL ? it / n_split : it;  // query block
     w.sp = PARTIAL ? it % n_split : 0;
     w.bh = p.snake ? unit % p.BH : unit / p.n_qb;
     int qb = p.snake ? unit / p.BH : unit % p.n_qb;
@@ -707,28 +701,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // it selects code paths that issue tcgen05.ld, which all 32 lanes must
       // execute together (a lane-divergent .sync.aligned instruction deadlocks).
       const bool masked = __any_sync(0xffffffffu, kbase + C::BN - 1 > kmax);
-      float sum_e, sum_r, alpha = 1.0f, mx = 0.f;
+      float sum_e, sum_r, alpha = 1.0f;
       if (j == 0) {
         // A row that sees no key of this split (partial mode only) has max -inf;
         // it takes reference 0, so its weights are exp2(-inf) = 0 throughout and
         // it is recognised at the end by its zero sum.
         m_ref = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;
         if (PARTIAL && m_ref == -INFINITY) m_ref = 0.f;
-        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        softmax_row_dispatch(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r);
       } else {
         // Exponentials against the current reference. A row whose max grew by more
         // than 8 (log2 units) has a weight above 2^8, so its tile sum exceeds 2^8:
         // only then (rare after the first tiles) is its exact max taken, and the
         // tile redone, against the new reference if the max did grow that much.
         // S is still intact: P is written only below.
-        softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+        softmax_row_dispatch(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r);
         if (__any_sync(0xffffffffu, sum_e > 256.0f)) {
           const float mx_s = row_max_tmem(tS, s, kbase, kmax, masked) * s_log2;
           const bool grow = mx_s > m_ref + 8.0f;
           const float m_new = grow ? mx_s : m_ref;
           alpha = ex2_approx(m_ref - m_new);  // 1 for rows that did not grow
           m_ref = m_new;
-          softmax_row_dispatch<false>(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r, mx);
+          softmax_row_dispatch(tS, s, s_log2, m_ref, kbase, kmax, masked, sum_e, sum_r);
           // Rescale this warp's O rows in TMEM. The PV product of tile j-1 has
           // completed (the commit that signalled S_t for tile j also covers it),
           // and PV of tile j is issued only after this warpgroup arrives below.

@@ -47,8 +47,6 @@ struct FwdArgs {
   fa_dtype qk_dtype;
   const float* descale_qk;
   int n_split;
-  int unit_base = 0;  // first query block of the launch (bh * n_qb + qb)
-  int n_units = 0;    // query blocks in the launch (0: all)
 };
 
 constexpr int kKeyTile = 128;  // keys per K/V tile (FwdCfg::BN)
@@ -123,8 +121,7 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   p.n_split = a.n_split;
   p.split_tiles = (key_tiles(a.Nk) + a.n_split - 1) / a.n_split;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.unit_base = a.unit_base;
-  const long long units = a.n_units > 0 ? a.n_units : static_cast<long long>(p.n_qb) * BH;
+  const long long units = static_cast<long long>(p.n_qb) * BH;
   const long long items = units * (PARTIAL ? a.n_split : 1);
   if (items < 1) return FA_OK;
   p.n_items = static_cast<int>(items);
