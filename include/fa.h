@@ -147,7 +147,8 @@ fa_status fa_fwd_partial(const void* q, const void* k, const void* v, float* o_p
 fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
                        float* lse, void* stream);
 
-/* Bytes of device workspace fa_hadamard_quant needs (the amax word and a grid-barrier counter, padded). */
+/* Bytes of device workspace fa_hadamard_quant and fa_hadamard_quant_multi need (the amax
+ * words and a grid-barrier counter, padded). */
 #define FA_QUANT_WORKSPACE_BYTES 256
 
 /*
@@ -166,7 +167,7 @@ fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, i
  * x           device, bf16 [rows][d], 16-byte aligned (e.g. [B][H][N][d], rows = B*H*N);
  *             may be NULL when rows = 0.
  * out         device, e4m3 codes [rows][d], 16-byte aligned; may be NULL when rows = 0.
- * descale_out device, one fp32 (written last, by the second kernel).
+ * descale_out device, one fp32 (written in the second pass, after the grid-wide amax).
  * rows >= 0;  d in {64, 128, 256}.
  * rotate      0 = quantise only, 1 = rotate first.
  * signs       device, d fp32 values +-1 (16-byte aligned), or NULL for no sign flips.

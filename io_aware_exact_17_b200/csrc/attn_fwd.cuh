@@ -9,9 +9,11 @@
 // FlashAttention-2" (tiling and fusing matmul + softmax + matmul in one kernel).
 //
 // Blackwell design (the pages' Hopper design is prior art):
-//  * one CTA = NQ query tiles of 128 rows of one (batch, head); NQ = 2 for
+//  * a work item = NQ query tiles of 128 rows of one (batch, head); NQ = 2 for
 //    d <= 128 so that the softmax of one tile overlaps the tensor-core work of
-//    the other (the pages' "ping-pong", section "Inovações técnicas", 1);
+//    the other (the pages' "ping-pong", section "Inovações técnicas", 1). CTAs
+//    are persistent where the host says so (one per SM, looping over items, the
+//    next item's Q load overlapping the current item's tail);
 //  * warp roles (section "Inovações técnicas", 1, producer/consumer warps):
 //      warps 0..4*NQ-1 : softmax, one thread per query row, one warpgroup per tile;
 //      warp 4*NQ       : tcgen05.mma issuer (one elected thread), TMEM owner;
@@ -22,8 +24,9 @@
 //    in four 32-column chunks, each load overlapping the previous chunk's exps,
 //    writes P_t = exp2(..) as bf16 pairs over the first 64 columns, and the MMA
 //    warp issues O_t += P_t V_j with P_t taken straight from TMEM;
-//  * online softmax in base 2 with the scale folded into one FMA; the running
-//    reference max is moved only when a row's max grows by more than 2^8, so
+//  * online softmax in base 2 with the scale folded into one FMA; the reference
+//    max is moved only when a row's max grows by more than 8 (log2 units),
+//    which a tile weight sum above 2^8 reveals without a per-key running max, so
 //    the O rescale (a TMEM read-modify-write) is rare. The final O / l and the
 //    LSE use the same reference, so the result is exact, not approximated;
 //  * the QK product can take e4m3 Q and K (the FP8 path with Hadamard-rotated

@@ -15,8 +15,10 @@
 //   pass 2: rotate again, scale, convert, store the codes.
 // A tensor of up to ~60 MB stays in the 126 MB L2 between the passes, so the
 // second read mostly hits L2. quant_fused_kernel runs both passes in one
-// cooperative launch; quant_amax_kernel + quant_apply_kernel are the two-launch
-// form (used where the scratch is the library's own static array).
+// cooperative launch, for up to 8 tensors at once (each with its own scale);
+// quant_amax_kernel + quant_apply_kernel are the two-launch form (used where
+// the scratch is the library's own static array). quant_block_kernel (end of
+// the file) takes one scale per 128-row block of a head, in one pass.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
