@@ -24,6 +24,14 @@ Pieces, each citing the passage it follows:
   glossary page (second paragraph) applied to whole partial results, as
   splitting the keys over several processors needs (same page, fourth
   paragraph, ring attention over several devices).
+* :func:`attention_bwd` — the gradients dQ, dK, dV of a scalar loss through
+  exact attention, given dO = dLoss/dO. The pages name training with the method
+  ("FlashAttention-3 (PT)", opening paragraph and section "Desempenho e
+  importância": faster training)
+  but print no backward algorithm, so this is the chain rule through the plain
+  definition, written out with the whole N x N probability matrix per head:
+  dV = Pᵀ dO, dP = dO Vᵀ, dS = P ∘ (dP - rowsum(P ∘ dP)) (the softmax Jacobian),
+  dQ = scale dS K, dK = scale dSᵀ Q. fp64 numpy.
 * :func:`sylvester_hadamard`, :func:`rotation_matrix`, :func:`rotate` — the
   orthogonal transform of "FlashAttention-3 (PT)", section "Inovações técnicas",
   subsection 3 ("Baixa precisão (FP8)"), steps 1 and 4: Q and K multiplied by a
@@ -190,6 +198,54 @@ def lse_merge(o_parts, lse_parts):
     with np.errstate(divide="ignore"):
         lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, total)))
     return o, lse
+
+
+def attention_bwd(q, k, v, do, causal: bool, scale: float, return_bounds: bool = False):
+    """Gradients of a loss L through O = softmax(scale Q Kᵀ) V, per (batch, head),
+    for square heads (N queries over the same N positions' keys).
+
+    ``do`` is dL/dO ``[B, H, N, d]``; ``causal`` hides key j from query i when
+    j > i. Per head, with S = scale Q Kᵀ (hidden entries -inf) and P its row
+    softmax:
+
+    * dV = Pᵀ dO;
+    * dP = dO Vᵀ and, since dP_i·P_i = Σ_j P_ij dP_ij is the derivative of the
+      softmax normaliser, dS = P ∘ (dP - rowsum(P ∘ dP));
+    * dQ = scale dS K and dK = scale dSᵀ Q.
+
+    Returns ``(dQ, dK, dV)``, each ``[B, H, N, d]``. With ``return_bounds`` it
+    also returns ``(mQ, mK, mV)``: the same products taken over absolute values,
+    with |dS| replaced by P (|dP| + A), A_i = Σ_c |dO_ic O_ic| — the envelope
+    that bounds how far rounding the products' operands can move each entry.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    if not (q.shape == k.shape == v.shape == do.shape) or q.ndim != 4:
+        raise ValueError("q, k, v and do must share one [B, H, N, d] shape")
+    B, H, N, d = q.shape
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    if return_bounds:
+        mq, mk, mv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    hidden = np.triu(np.ones((N, N), dtype=bool), 1) if causal else np.zeros((N, N), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh, doh = q[b, h], k[b, h], v[b, h], do[b, h]
+            s = np.where(hidden, -np.inf, scale * (qh @ kh.T))
+            w = np.exp(s - s.max(axis=1, keepdims=True))
+            p = w / w.sum(axis=1, keepdims=True)
+            dv[b, h] = p.T @ doh
+            dp = doh @ vh.T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dq[b, h] = scale * (ds @ kh)
+            dk[b, h] = scale * (ds.T @ qh)
+            if return_bounds:
+                a = np.abs(doh * (p @ vh)).sum(axis=1, keepdims=True)
+                e = p * (np.abs(dp) + a)
+                mv[b, h] = p.T @ np.abs(doh)
+                mq[b, h] = scale * (e @ np.abs(kh))
+                mk[b, h] = scale * (e.T @ np.abs(qh))
+    if return_bounds:
+        return (dq, dk, dv), (mq, mk, mv)
+    return dq, dk, dv
 
 
 # ----------------------------------------------------------------- rotation --
