@@ -1,7 +1,7 @@
 /*
  * fa.h — C ABI of libfa.so: fused exact-attention forward on B200 (sm_100a),
- * BF16 and FP8-e4m3 (for Q Kᵀ), and the Hadamard rotate-and-quantise step that
- * prepares FP8 queries and keys.
+ * BF16 and FP8-e4m3 (for Q Kᵀ), its BF16 backward pass, and the Hadamard
+ * rotate-and-quantise step that prepares FP8 queries and keys.
  *
  * Conventions for every entry point:
  *  - Pointers marked "device" must point to memory of the CUDA device that is
@@ -147,6 +147,33 @@ fa_status fa_fwd_partial(const void* q, const void* k, const void* v, float* o_p
 fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
                        float* lse, void* stream);
 
+/*
+ * fa_bwd — gradients of a loss through exact attention: given dO = dLoss/dO for
+ * O = softmax(scale Q Kᵀ) V (square heads, as fa_fwd computes it), return
+ *   dV = Pᵀ dO,  dS = P ∘ (dO Vᵀ - D),  D_i = dO_i · O_i,
+ *   dQ = scale dS K,  dK = scale dSᵀ Q,
+ * per batch and head, with P the attention probabilities (causal: key j hidden
+ * from query i when j > i). The pages name training with the method
+ * ("FlashAttention-3 (PT)", opening paragraph and section "Desempenho e
+ * importância") but give no backward algorithm: this is the chain rule through
+ * the definition fa_fwd documents. P is recomputed on chip from Q, K and the
+ * forward's LSE, so no N x N matrix is written ("Flash Attention" glossary page,
+ * second paragraph). D_i uses the given O, as the forward returned it.
+ *
+ * q, k, v, o, dout   device, bf16 [B][H][N][d], 16-byte aligned (o: fa_fwd's output).
+ * lse                device, fp32 [B][H][N]: fa_fwd's LSE (natural log), 4-byte aligned.
+ * dq, dk, dv         device, bf16 [B][H][N][d] outputs (round to nearest even), 16-byte aligned.
+ * B, H, N >= 1; d in {64, 128} (d = 256 returns FA_ERR_UNSUPPORTED: dK and dV of a
+ * 128-key tile would need all of a CTA's tensor memory); scale finite and > 0.
+ * workspace          device, >= fa_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte
+ *                    aligned: the fp32 dQ accumulator and the per-row D and LSE.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace fa_hadamard_quant and fa_hadamard_quant_multi need (the amax
  * words and a grid-barrier counter, padded). */
 #define FA_QUANT_WORKSPACE_BYTES 256
@@ -258,8 +285,8 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
 
-/* ABI version of this header: 3 (1, plus the split-key, partial and merge calls in 2,
- * plus per-block e4m3 scales in 3). */
+/* ABI version of this header: 4 (1, plus the split-key, partial and merge calls in 2,
+ * plus per-block e4m3 scales in 3, plus the backward pass in 4). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

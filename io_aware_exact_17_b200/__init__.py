@@ -1,5 +1,6 @@
 """Fused exact-attention forward for B200 (sm_100a): BF16 and FP8-e4m3 kernels,
-the Hadamard rotate-and-quantise step of the FP8 path, and attention of few
+the BF16 backward pass, the Hadamard rotate-and-quantise step of the FP8 path,
+and attention of few
 queries over long key sequences with the keys split across CTAs and merged by
 their LSEs.
 
@@ -9,6 +10,8 @@ call does, and fails loudly if the library or a GPU is missing.
 """
 from .binding import (  # noqa: F401
     FaError,
+    bwd,
+    bwd_workspace_bytes,
     device_status,
     fwd,
     fwd_partial,
@@ -22,5 +25,5 @@ from .binding import (  # noqa: F401
     splitkv_splits,
 )
 
-__all__ = ["fwd", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
+__all__ = ["fwd", "bwd", "bwd_workspace_bytes", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
            "hadamard_quant_blocks", "hadamard_quant_multi", "device_status", "load_library", "library_path", "FaError"]

@@ -74,6 +74,10 @@ def load_library():
         lib.fa_hadamard_quant_blocks.restype = i
         lib.fa_hadamard_quant_multi.argtypes = [vp, vp, vp, i, i64, i, i, vp, vp, sz, vp]
         lib.fa_hadamard_quant_multi.restype = i
+        lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        lib.fa_bwd_workspace_bytes.restype = sz
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+        lib.fa_bwd.restype = i
         _lib = lib
         return lib
 
@@ -287,6 +291,38 @@ def lse_merge(o_part, lse_part, out=None, lse=None, return_lse: bool = True):
                               _ptr(lse) if return_lse else None, _stream(o_part.device))
     _check(rc, "fa_lse_merge")
     return out, (lse if return_lse else None)
+
+
+def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, workspace=None):
+    """Gradients ``(dQ, dK, dV)`` (bf16 ``[B, H, N, d]``) of a loss through
+    ``fwd(q, k, v, causal, scale)``, given its output ``o``, its ``lse`` and
+    ``dout`` = dLoss/dO, through ``fa_bwd``. d is 64 or 128. ``workspace``: an
+    optional CUDA uint8 tensor of at least ``fa_bwd_workspace_bytes`` bytes."""
+    _require_cuda(q, k, v, o, lse, dout)
+    lib = load_library()
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or tuple(t.shape) != tuple(q.shape):
+            raise FaError(f"{name} must be bf16 [B, H, N, d] like q")
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise FaError("lse must be fp32 [B, H, N]")
+    scale = d ** -0.5 if scale is None else scale
+    q, k, v, o, dout, lse = (t.contiguous() for t in (q, k, v, o, dout, lse))
+    need = lib.fa_bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    with torch.cuda.device(q.device):
+        rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                        B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    """Bytes of device workspace ``fa_bwd`` needs (0 for an unsupported shape)."""
+    return int(load_library().fa_bwd_workspace_bytes(B, H, N, d))
 
 
 def _workspace(device) -> torch.Tensor:

@@ -1,0 +1,444 @@
+// attn_bwd.cuh — backward pass of exact attention for sm_100a: the gradients
+// dQ, dK, dV of a loss through O = softmax(scale Q Kᵀ) V, given dO, the forward
+// output O and its per-row LSE.
+//
+// The pages name training with the method ("FlashAttention-3 (PT)", opening
+// paragraph and section "Desempenho e importância") but give no backward
+// algorithm. This computes the chain rule through the plain definition, with
+// the probabilities recomputed on chip from Q, K and the LSE, so that no N x N
+// matrix reaches memory (the IO-aware principle of the "Flash Attention"
+// glossary page, second paragraph):
+//   P = exp(scale Q Kᵀ - LSE), dV = Pᵀ dO, dP = dO Vᵀ, D_i = dO_i · O_i,
+//   dS = P ∘ (dP - D), dQ = scale dS K, dK = scale dSᵀ Q.
+// (D_i = Σ_j P_ij dP_ij because O_i = Σ_j P_ij v_j.)
+//
+// Blackwell design:
+//  * one CTA per (batch·head, tile of 128 keys). Its K_j and V_j stay in
+//    shared memory, and dK_j and dV_j accumulate in TMEM over the query tiles
+//    (causal: from the diagonal tile on, heaviest key tiles launched first);
+//  * per query tile i (128 rows, Q_i and dO_i through a ring of stages loaded
+//    by TMA): Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ in TMEM, keys on the lanes;
+//  * two softmax warpgroups, 64 queries each, form P and dS = P (dP - D) for
+//    their key rows. They write P back over Sᵀ as bf16 pairs: the A operand of
+//    dV += Pᵀ dO_i, read from TMEM. They write dSᵀ to shared memory in the
+//    128-byte-swizzle layout: the K-major A operand of dK += dSᵀ Q_i and, read
+//    MN-major, the A operand of dQ_i = dS K_j;
+//  * dQ_i lands in the dP columns. The same warps add it into an fp32
+//    workspace with vector reductions while the tensor core runs dV, dK and
+//    the next Sᵀ;
+//  * a prologue kernel forms D_i and the LSE in log2 units, padded per head to
+//    whole tiles (+inf and 0, so that padded queries get P = 0). An epilogue
+//    kernel scales dQ and rounds it to bf16.
+// TMEM holds Sᵀ (128 columns), dPᵀ / dQ (128), dV (d) and dK (d): d <= 128.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "sm100.cuh"
+
+namespace fa {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BK = 128;                 // keys per CTA (TMEM lanes)
+  static constexpr int BQ = 128;                 // queries per step
+  static constexpr int TILE = 128 * D * 2;       // one 128 x D bf16 tile
+  static constexpr int CHUNK = 128 * 128;        // one 128-byte swizzle column of a 128-row tile
+  static constexpr int DS_TILE = BK * BQ * 2;    // dSᵀ, 128 keys x 128 queries bf16
+  static constexpr int NST = D == 128 ? 2 : 3;   // Q_i / dO_i stages
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int SMEM_BYTES = 1024 + 2 * TILE + DS_TILE + NST * STAGE;
+  static constexpr int THREADS = 384;            // 8 softmax warps, MMA warp, TMA warp, 2 idle
+  static constexpr int MMA_WARP = 8;
+  static constexpr int TMA_WARP = 9;
+  static constexpr uint32_t S_COL = 0;           // Sᵀ, then P as bf16 pairs (64 columns)
+  static constexpr uint32_t DP_COL = 128;        // dPᵀ, then dQ_i (D columns)
+  static constexpr uint32_t DV_COL = 256;
+  static constexpr uint32_t DK_COL = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(SMEM_BYTES + 256 <= 227 * 1024, "shared memory");
+};
+
+struct BwdParams {
+  __nv_bfloat16* dk;        // [BH][N][D]
+  __nv_bfloat16* dv;        // [BH][N][D]
+  float* dq_acc;            // [BH][N][D] fp32, zeroed by the prologue; dQ / scale
+  const float* lse2;        // [BH][Npad]: LSE * log2(e), +inf past N
+  const float* dvec;        // [BH][Npad]: D_i = dO_i · O_i, 0 past N
+  int BH, N, Npad, n_t;     // n_t = Npad / 128 tiles per head
+  float scale, scale_log2;  // scale, scale * log2(e)
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core reads its shared-memory operands through it).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bounded wait used only while tearing down after an abort.
+__device__ __forceinline__ void mbar_drain_bwd(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = sm;
+  uint8_t* sV = sK + C::TILE;
+  uint8_t* sdS = sV + C::TILE;
+  uint8_t* sStage = sdS + C::DS_TILE;  // stage s: Q_i then dO_i
+
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[C::NST], bar_empty[C::NST];
+  __shared__ __align__(8) uint64_t bar_s, bar_sread, bar_p, bar_dq, bar_dqfree, bar_done, bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  // causal: key tile 0 (the most query tiles) first
+  const int kt = static_cast<int>(blockIdx.x) / p.BH;
+  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  const int qt0 = CAUSAL ? kt : 0;
+  const int n_steps = p.n_t - qt0;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_kv, 1);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_sread, 8);  // one arrival per softmax warp
+    mbar_init(&bar_p, 8);
+    mbar_init(&bar_dq, 1);
+    mbar_init(&bar_dqfree, 8);
+    mbar_init(&bar_done, 1);
+    mbar_init(&bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(&tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+  DevStatus* st = &g_fa_status;
+
+  if (warp == C::TMA_WARP && lane == 0) {
+    // ------------------------------------------------------------ producer --
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmdO);
+    mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, kt * C::BK, bh);
+      tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, kt * C::BK, bh);
+    }
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; i < n_steps && ok; ++i) {
+      const int slot = i % C::NST, round = i / C::NST;
+      if (round > 0) ok = mbar_wait(&bar_empty[slot], (round - 1) & 1, &abort_flag, st, 50);
+      if (!ok) break;
+      uint8_t* dst = sStage + slot * C::STAGE;
+      const int q0 = (qt0 + i) * C::BQ;
+      mbar_arrive_expect_tx(&bar_full[slot], 2 * C::TILE);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(dst + c * C::CHUNK, &tmQ, &bar_full[slot], c * 64, q0, bh);
+        tma_load_3d(dst + C::TILE + c * C::CHUNK, &tmdO, &bar_full[slot], c * 64, q0, bh);
+      }
+      ++issued;
+    }
+    // every load this thread issued lands before the CTA can exit
+    mbar_drain_bwd(&bar_kv, 0);
+    for (int i = issued - C::NST; i < issued; ++i)
+      if (i >= 0) mbar_drain_bwd(&bar_full[i % C::NST], (i / C::NST) & 1);
+  } else if (warp == C::MMA_WARP && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer --
+    constexpr uint32_t idesc_kq = idesc_make(1u, 128, 128, false);        // A, B K-major
+    constexpr uint32_t idesc_bmn = idesc_make(1u, 128, D, true);          // B MN-major
+    constexpr uint32_t idesc_dq = idesc_make(1u, 128, D, true) | (1u << 15);  // A and B MN-major
+    const uint32_t kaddr = smem_u32(sK), vaddr = smem_u32(sV), dsaddr = smem_u32(sdS);
+    const uint32_t stage0 = smem_u32(sStage);
+    // D_tmem = A Bᵀ over d: A a 128-row K-major tile (keys), B one (queries)
+    auto issue_rows = [&](uint32_t dcol, uint32_t a, uint32_t b) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int kb = kk * 32, chunk = kb / 128, within = kb % 128;
+        mma_bf16_ss(tbase + dcol, sdesc_sw128(a + chunk * C::CHUNK + within, 0, 1024),
+                    sdesc_sw128(b + chunk * C::CHUNK + within, 0, 1024), idesc_kq, kk > 0 ? 1u : 0u);
+      }
+    };
+    bool ok = mbar_wait(&bar_kv, 0, &abort_flag, st, 51);
+    if (ok) ok = mbar_wait(&bar_full[0], 0, &abort_flag, st, 52);
+    if (ok) {
+      tc_fence_after();
+      issue_rows(C::S_COL, kaddr, stage0);
+      issue_rows(C::DP_COL, vaddr, stage0 + C::TILE);
+      mma_commit(&bar_s);
+    }
+    for (int i = 0; i < n_steps && ok; ++i) {
+      const int slot = i % C::NST;
+      const uint32_t qaddr = stage0 + slot * C::STAGE, doaddr = qaddr + C::TILE;
+      ok = mbar_wait(&bar_p, i & 1, &abort_flag, st, 53, 0u);
+      if (!ok) break;
+      tc_fence_after();
+      // dQ_i = dS K_j: A = dSᵀ read MN-major (queries along rows), B = K_j MN-major; 16 keys per MMA
+#pragma unroll
+      for (int kk = 0; kk < C::BK / 16; ++kk)
+        mma_bf16_ss(tbase + C::DP_COL, sdesc_sw128(dsaddr + kk * 16 * 128, C::CHUNK, 1024),
+                    sdesc_sw128(kaddr + kk * 16 * 128, C::CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+      mma_commit(&bar_dq);
+      // dV += Pᵀ dO_i: A = P from TMEM (bf16 pairs, keys on lanes), B = dO_i MN-major; 16 queries per MMA
+#pragma unroll
+      for (int kk = 0; kk < C::BQ / 16; ++kk)
+        mma_bf16_ts(tbase + C::DV_COL, tbase + C::S_COL + kk * 8, sdesc_sw128(doaddr + kk * 16 * 128, C::CHUNK, 1024),
+                    idesc_bmn, (i > 0 || kk > 0) ? 1u : 0u);
+      // dK += dSᵀ Q_i: A = dSᵀ K-major, B = Q_i MN-major
+#pragma unroll
+      for (int kk = 0; kk < C::BQ / 16; ++kk) {
+        const int kb = kk * 32, chunk = kb / 128, within = kb % 128;
+        mma_bf16_ss(tbase + C::DK_COL, sdesc_sw128(dsaddr + chunk * C::CHUNK + within, 0, 1024),
+                    sdesc_sw128(qaddr + kk * 16 * 128, C::CHUNK, 1024), idesc_bmn, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&bar_empty[slot]);  // Q_i and dO_i read
+      if (i + 1 < n_steps) {
+        const int ns = (i + 1) % C::NST;
+        const uint32_t nq = stage0 + ns * C::STAGE;
+        ok = mbar_wait(&bar_full[ns], ((i + 1) / C::NST) & 1, &abort_flag, st, 54);
+        if (!ok) break;
+        tc_fence_after();
+        issue_rows(C::S_COL, kaddr, nq);  // after dV_i, which reads P from these columns
+        ok = mbar_wait(&bar_dqfree, i & 1, &abort_flag, st, 55, 0u);
+        if (!ok) break;
+        tc_fence_after();
+        issue_rows(C::DP_COL, vaddr, nq + C::TILE);
+        mma_commit(&bar_s);
+      }
+    }
+    if (ok) mma_commit(&bar_done);
+    // TMEM is freed below only after every issued MMA has finished
+    mma_commit(&bar_drain);
+    mbar_drain_bwd(&bar_drain, 0);
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- softmax --
+    const int g = static_cast<int>(warp >> 2);  // query columns 64g .. 64g + 63
+    const uint32_t lane_base = (warp & 3u) * 32u;
+    const int r = static_cast<int>(lane_base + lane);  // key row (Sᵀ lane); query row for dQ
+    const int kr = kt * C::BK + r;
+    const uint32_t row_addr = tbase + (lane_base << 16);
+    const float* lse2h = p.lse2 + static_cast<size_t>(bh) * p.Npad;
+    const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
+    const uint32_t ds_row = smem_u32(sdS) + g * C::CHUNK + r * 128;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int i = 0; i < n_steps; ++i) {
+      const int q0 = (qt0 + i) * C::BQ;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_s, i & 1, &abort_flag, st, 60));
+      if (!ok) break;
+      tc_fence_after();
+      // P = exp2(scale log2(e) s - LSE log2(e)) for this key row and 64 queries
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(row_addr + C::S_COL + 64 * g + 32 * c, sv);
+        tmem_wait_ld_dep32(sv);
+        const float4* l4 = reinterpret_cast<const float4*>(lse2h + q0 + 64 * g + 32 * c);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 l = __ldg(l4 + u);
+          pv[32 * c + 4 * u + 0] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 0]), sl2, -l.x));
+          pv[32 * c + 4 * u + 1] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 1]), sl2, -l.y));
+          pv[32 * c + 4 * u + 2] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 2]), sl2, -l.z));
+          pv[32 * c + 4 * u + 3] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 3]), sl2, -l.w));
+        }
+      }
+      // this warp's reads of Sᵀ are done (P overwrites those columns below)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sread);
+      if (kr >= p.N) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) pv[e] = 0.f;
+      }
+      if (CAUSAL && i == 0) {
+        // diagonal tile: query q0 + 64g + e sees key kr iff 64g + e >= r
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (64 * g + e < r) pv[e] = 0.f;
+      }
+      // dS = P (dP - D), rounded to bf16, into row r of dSᵀ (swizzled 16-byte units)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dv[32];
+        tmem_ld32(row_addr + C::DP_COL + 64 * g + 32 * c, dv);
+        tmem_wait_ld_dep32(dv);
+        const float4* d4 = reinterpret_cast<const float4*>(dvh + q0 + 64 * g + 32 * c);
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 dd = __ldg(d4 + u);
+          const float* pp = &pv[32 * c + 4 * u];
+          pk[2 * u] = pack_bf16x2(pp[0] * (__uint_as_float(dv[4 * u + 0]) - dd.x),
+                                  pp[1] * (__uint_as_float(dv[4 * u + 1]) - dd.y));
+          pk[2 * u + 1] = pack_bf16x2(pp[2] * (__uint_as_float(dv[4 * u + 2]) - dd.z),
+                                      pp[3] * (__uint_as_float(dv[4 * u + 3]) - dd.w));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t unit = static_cast<uint32_t>(4 * c + u) ^ static_cast<uint32_t>(r & 7);
+          st_shared_v4(ds_row + unit * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      // P as bf16 pairs over Sᵀ, once every softmax warp has read its Sᵀ columns
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_sread, i & 1, &abort_flag, st, 61));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+        tmem_st32(row_addr + C::S_COL + 32 * g, pk);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p);
+      // dQ_i rows (queries on lanes): add into the fp32 accumulator
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_dq, i & 1, &abort_flag, st, 62));
+      if (!ok) break;
+      tc_fence_after();
+      const int qrow = q0 + r;
+      float* dqrow = p.dq_acc + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
+#pragma unroll
+      for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(row_addr + C::DP_COL + c0, v);
+        tmem_wait_ld_dep32(v);
+        if (qrow < p.N) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            red_add_v4(dqrow + c0 + 4 * u, __uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                       __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_dqfree);
+    }
+    // ------------------------------------------------------------ epilogue --
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_done, 0, &abort_flag, st, 63));
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = (static_cast<size_t>(bh) * p.N + (kr < p.N ? kr : 0)) * D;
+#pragma unroll
+      for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
+        uint32_t v[32], k[32];
+        tmem_ld32(row_addr + C::DV_COL + c0, v);
+        tmem_ld32(row_addr + C::DK_COL + c0, k);
+        tmem_wait_ld_dep32(v);
+        tmem_wait_ld_dep32(k);
+        uint32_t pv2[16], pk2[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          pv2[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          pk2[e] = pack_bf16x2(__uint_as_float(k[2 * e]) * p.scale, __uint_as_float(k[2 * e + 1]) * p.scale);
+        }
+        if (kr < p.N) {
+          uint4* dv4 = reinterpret_cast<uint4*>(p.dv + orow + c0);
+          uint4* dk4 = reinterpret_cast<uint4*>(p.dk + orow + c0);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            dv4[u] = make_uint4(pv2[4 * u], pv2[4 * u + 1], pv2[4 * u + 2], pv2[4 * u + 3]);
+            dk4[u] = make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// Prologue: per padded query row, D_i = dO_i · O_i and LSE_i log2(e) (+inf and
+// 0 past N), and zero row i of the dQ accumulator. One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                            const __nv_bfloat16* __restrict__ dout,
+                                                            const float* __restrict__ lse, float* lse2, float* dvec,
+                                                            float* dq_acc, int BH, int N, int Npad) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const uint32_t lane = lane_id();
+  if (row >= static_cast<long long>(BH) * Npad) return;
+  const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
+  if (i >= N) {
+    if (lane == 0) {
+      lse2[row] = INFINITY;
+      dvec[row] = 0.f;
+    }
+    return;
+  }
+  constexpr int PER = D / 32;  // elements per lane: 2 or 4
+  const size_t off = (static_cast<size_t>(bh) * N + i) * D + lane * PER;
+  float acc = 0.f;
+  if constexpr (PER == 4) {
+    const uint2 a = *reinterpret_cast<const uint2*>(o + off);
+    const uint2 b = *reinterpret_cast<const uint2*>(dout + off);
+    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+    const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
+    const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
+    acc = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
+    *reinterpret_cast<float4*>(dq_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + off));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + off));
+    acc = a.x * b.x + a.y * b.y;
+    *reinterpret_cast<float2*>(dq_acc + off) = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) {
+    lse2[row] = lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f;
+    dvec[row] = acc;
+  }
+}
+
+// Epilogue: dQ = scale * accumulator, rounded to bf16. n4 groups of 4 elements.
+__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq,
+                                                          long long n4, float scale) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = acc[i];
+    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  }
+}
+
+}  // namespace fa

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "merge.cuh"
 #include "quant.cuh"
@@ -374,6 +375,62 @@ fa_status dispatch_merge(const float* o_part, const float* lse_part, int n_part,
 
 }  // namespace
 
+// ------------------------------------------------------------- backward --
+inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int bwd_npad(int N) { return (N + 127) / 128 * 128; }
+
+size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+  const size_t BH = static_cast<size_t>(B) * H;
+  return round256(BH * N * d * sizeof(float)) + 2 * round256(BH * bwd_npad(N) * sizeof(float));
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, int B, int H, int N, float scale, void* workspace,
+                     cudaStream_t stream) {
+  using C = fa::BwdCfg<D>;
+  const int BH = B * H;
+  const int Npad = bwd_npad(N);
+  float* dq_acc = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         round256(static_cast<size_t>(BH) * N * D * sizeof(float)));
+  float* dvec = lse2 + round256(static_cast<size_t>(BH) * Npad * sizeof(float)) / sizeof(float);
+  CUtensorMap tmQ, tmK, tmV, tmdO;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!fa::make_tmap_3d(&tmQ, q, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmK, k, bf, 2, D, N, BH, 64, 128) ||
+      !fa::make_tmap_3d(&tmV, v, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmdO, dout, bf, 2, D, N, BH, 64, 128))
+    return FA_ERR_CUDA;
+  const long long rows = static_cast<long long>(BH) * Npad;
+  fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, dq_acc, BH, N,
+      Npad);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  auto kernel = fa::attn_bwd_kernel<D, CAUSAL>;
+  static unsigned long long smem_done = 0;
+  if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq_acc = dq_acc;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.BH = BH;
+  p.N = N;
+  p.Npad = Npad;
+  p.n_t = Npad / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, C::SMEM_BYTES, stream>>>(
+      tmQ, tmK, tmV, tmdO, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const long long n4 = static_cast<long long>(BH) * N * D / 4;
+  const long long cap = static_cast<long long>(device_sms()) * 8;
+  const long long blocks = (n4 + 255) / 256 < cap ? (n4 + 255) / 256 : cap;
+  fa::attn_bwd_dq_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                                             static_cast<uint2*>(dq), n4, scale);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -446,6 +503,34 @@ fa_status fa_fwd_partial(const void* q, const void* k, const void* v, float* o_p
   FwdArgs a{q, k, v, nullptr, nullptr, o_part, lse_part, B, H, Nq, Nk, d, causal != 0, scale, qk_dtype, descale_qk,
             n_split};
   return dispatch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return bwd_workspace_bytes(B, H, N, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || dout == nullptr || lse == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;  // d = 256: dK and dV alone fill TMEM
+  if (static_cast<long long>(B) * H * (bwd_npad(N) / 128) > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N > (1LL << 40)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return FA_ERR_ALIGNMENT;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, workspace, s)
+                  : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, workspace, s);
+  return causal ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, workspace, s)
+                : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, scale, workspace, s);
 }
 
 fa_status fa_lse_merge(const float* o_part, const float* lse_part, int n_part, int64_t rows, int d, void* o,
@@ -627,6 +712,6 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
   return FA_OK;
 }
 
-int fa_abi_version(void) { return 3; }
+int fa_abi_version(void) { return 4; }
 
 }  // extern "C"

@@ -16,6 +16,8 @@ Recipe (all on the CPU, ``torch.Generator`` seeded, then moved as needed):
   rounds up to one channel per head).
 * Outliers, reading R2: each element of Q and K independently multiplied by 20
   with probability 0.001.
+* Output gradients dO for the backward pass: fp32 standard normal from a
+  generator seeded with the given seed, cast to bf16, layout ``[B, H, N, d]``.
 * Hadamard signs: d independent fair +-1 draws (the random diagonal of the
   rotation); ``None`` means no sign flips.
 """
@@ -54,6 +56,12 @@ def qkv_decode(B: int, H: int, Nq: int, Nk: int, d: int, seed: int, dtype=torch.
     k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32).to(dtype)
     v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32).to(dtype)
     return q, k, v
+
+
+def grad_out(B: int, H: int, N: int, d: int, seed: int, dtype=torch.bfloat16) -> torch.Tensor:
+    """dLoss/dO for the backward pass: standard normal, cast to ``dtype``."""
+    g = _gen(seed)
+    return torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(dtype)
 
 
 def outlier_channels(H: int, d: int, seed: int) -> torch.Tensor:

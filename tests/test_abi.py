@@ -30,7 +30,8 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
     assert {"fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_splits", "fa_fwd_partial",
             "fa_lse_merge"} <= set(names)
-    assert lib.fa_abi_version() == 3
+    assert {"fa_bwd", "fa_bwd_workspace_bytes"} <= set(names)
+    assert lib.fa_abi_version() == 4
 
 
 def test_status_strings(lib):
@@ -180,3 +181,30 @@ def test_python_binding_rejects_cpu_tensors():
         binding.fwd_partial(q, q, q)
     with pytest.raises(binding.FaError):
         binding.lse_merge(q.float(), q.float()[..., 0])
+
+
+def test_bwd_argument_errors(lib):
+    need = lib.fa_bwd_workspace_bytes(2, 3, 300, 128)
+    # dQ accumulator (fp32, 256-byte padded) plus the per-row D and LSE over whole 128-row tiles
+    assert need == 2 * 3 * 300 * 128 * 4 + 2 * ((2 * 3 * 384 * 4 + 255) // 256 * 256)
+    assert lib.fa_bwd_workspace_bytes(2, 3, 300, 256) == 0
+    assert lib.fa_bwd_workspace_bytes(0, 3, 300, 128) == 0
+
+    def bwd(**kw):
+        ptrs = [kw.get(n, A) for n in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv")]
+        return lib.fa_bwd(*ptrs, kw.get("B", 2), 3, kw.get("N", 300), kw.get("d", 128), kw.get("causal", 0),
+                          kw.get("scale", 0.1), kw.get("ws", A), kw.get("wsb", need), None)
+
+    for name in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv", "ws"):
+        assert bwd(**{name: None}) == binding.FA_ERR_INVALID_ARG, name
+    assert bwd(B=0) == binding.FA_ERR_INVALID_ARG
+    assert bwd(N=0) == binding.FA_ERR_INVALID_ARG
+    assert bwd(scale=0.0) == binding.FA_ERR_INVALID_ARG
+    assert bwd(scale=float("nan")) == binding.FA_ERR_INVALID_ARG
+    assert bwd(d=256) == binding.FA_ERR_UNSUPPORTED
+    assert bwd(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert bwd(wsb=need - 1) == binding.FA_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "o", "do", "dq", "dk", "dv"):
+        assert bwd(**{name: MIS}) == binding.FA_ERR_ALIGNMENT, name
+    assert bwd(lse=A + 2) == binding.FA_ERR_ALIGNMENT
+    assert bwd(ws=A + 16) == binding.FA_ERR_ALIGNMENT
