@@ -18,6 +18,12 @@ split-key attention kernel (fp32 partial results per block of keys) and the LSE
 merge. It is HBM-bound (the 1.07 GB of K and V are read once per step), so its
 metric is GB/s of algorithmic traffic.
 
+``--workload bwd`` measures the backward pass on the B=4, H=16, N=2048, d=128
+workload: one step is fa_bwd non-causal then fa_bwd causal (each a prologue, the
+tcgen05 kernel and the dQ conversion), given O and LSE from the library's
+forward (computed once, outside the timed region). Metric: backward TFLOPS =
+10*B*H*N^2*d (the five N x N x d products; halved when causal) / step time.
+
 Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
 torch.distributed.run, one rank per GPU, each rank its own batch: weak scaling,
 no collective on the data path).
@@ -45,6 +51,7 @@ from io_aware_exact_17_b200 import inputs as fa_inputs  # noqa: E402
 METRIC = "attention fwd TFLOPS (4·B·H·N²·d, ½ if causal) and % of B200 BF16/FP8 peak"
 DECODE = {"B": 4, "H": 16, "Nq": 1, "Nk": 32768, "d": 128, "seed": 1005}
 DECODE_METRIC = "decode attention GB/s (algorithmic HBM bytes: K, V, Q read; O, LSE written)"
+BWD_METRIC = "attention bwd TFLOPS (10·B·H·N²·d, ½ if causal) and % of B200 BF16 peak"
 B, H, N, D = 4, 16, 2048, 128
 SEED = 1001
 WORKLOAD = f"b{B}h{H}n{N}d{D}: bf16 fwd non-causal + bf16 fwd causal + rotate/quantise Q,K + e4m3-QK fwd non-causal"
@@ -385,6 +392,77 @@ class DecodeStep:
         return self.o_h.numel() * 2 + self.lse_h.numel() * 4
 
 
+class BwdStep:
+    """The backward pass: fa_bwd non-causal, then fa_bwd causal, over the same
+    Q, K, V and dO, each with the O and LSE the library's forward returned for
+    that mask (computed once at set-up)."""
+
+    def __init__(self, seed: int):
+        import io_aware_exact_17_b200 as fa
+
+        self.fa = fa
+        q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
+        do = fa_inputs.grad_out(B, H, N, D, seed + 500)
+        dev = [t.cuda() for t in (q, k, v, do)]
+        fwd = [fa.fwd(dev[0], dev[1], dev[2], causal=c) for c in (False, True)]
+        torch.cuda.synchronize()
+        # host copies of every input, pinned, for the end-to-end steps
+        self.host_in = [t.pin_memory() for t in (q, k, v, do)]
+        for o, lse in fwd:
+            self.host_in += [o.cpu().pin_memory(), lse.cpu().pin_memory()]
+        # two device sets of the inputs (q, k, v, do, o_nc, lse_nc, o_c, lse_c) and workspaces
+        self.sets = [[t.to("cuda", non_blocking=False).clone() for t in self.host_in] for _ in range(2)]
+        nbytes = fa.bwd_workspace_bytes(B, H, N, D)
+        self.ws = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+        self.out = [None, None]
+        self.host_out = [torch.empty((B, H, N, D), dtype=torch.bfloat16).pin_memory() for _ in range(6)]
+        self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 6
+        self.groups = 2  # breakdown: bwd non-causal, bwd causal
+
+    def flush_l2(self):
+        self.flush_buf.zero_()
+
+    def _bwd(self, b, causal):
+        q, k, v, do, o_nc, lse_nc, o_c, lse_c = self.sets[b]
+        o, lse = (o_c, lse_c) if causal else (o_nc, lse_nc)
+        return self.fa.bwd(q, k, v, o, lse, do, causal=causal, workspace=self.ws[b])
+
+    def run(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.out[0] = self._bwd(0, False)
+        if ev is not None:
+            ev[1].record()
+        self.out[1] = self._bwd(0, True)
+        if ev is not None:
+            ev[2].record()
+
+    def h2d(self, b):
+        for dst, src in zip(self.sets[b], self.host_in):
+            dst.copy_(src, non_blocking=True)
+
+    def compute(self, b):
+        self.out[b] = self._bwd(b, False) + self._bwd(b, True)
+
+    def d2h(self, b):
+        for dst, src in zip(self.host_out, self.out[b]):
+            dst.copy_(src, non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host_in)
+
+    @property
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host_out)
+
+
+def flops_bwd(causal: bool) -> float:
+    """The five N x N x d products of the backward pass (S, dP, dV, dK, dQ)."""
+    return 10.0 * B * H * N * N * D * (0.5 if causal else 1.0)
+
+
 def capture_step(step):
     """The step's kernels captured once as a CUDA graph, so a timed step carries
     no host launch overhead (the quantiser kernels are ~10 us each)."""
@@ -510,6 +588,72 @@ def oracle_sample(target_s: float, seed: int):
     return fl, dt, threads, rows_n
 
 
+def oracle_bwd_sample(target_s: float, seed: int):
+    """Time the backward oracle (as it stands) on whole heads of the workload,
+    non-causal and causal alternately, for about ``target_s`` seconds.
+    Returns (flops, seconds, threads, heads)."""
+    import oracle
+
+    q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
+    do = fa_inputs.grad_out(B, H, N, D, seed + 500)
+    fl, heads = 0.0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < target_s or heads < 2:
+        b, h = divmod(heads % (B * H), H)
+        causal = heads % 2 == 1
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        oracle.attention_bwd(q[sl], k[sl], v[sl], do[sl], causal, D ** -0.5)
+        fl += flops_bwd(causal) / (B * H)
+        heads += 1
+    return fl, time.perf_counter() - t0, oracle.default_threads(), heads
+
+
+def run_bwd(args, world: int, rank: int):
+    step = BwdStep(SEED + rank)
+    graph = capture_step(step)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
+    e2e_ms = dist_max(time_e2e(step, max(8, args.steps // 2), 3, world), world)
+    ms = dist_max(statistics.mean(step_ms), world)
+    comp = [dist_max(statistics.mean(p[j] for p in per), world) for j in range(2)]
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    if rank == 0:
+        step_flops = flops_bwd(False) + flops_bwd(True)
+        achieved = flops_bwd(False) / (comp[0] * 1e-3) / 1e12
+        line = {
+            "metric": BWD_METRIC, "value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16)",
+            "config": {"workload": f"bwd b{B}h{H}n{N}d{D}: fa_bwd non-causal + fa_bwd causal", "B": B, "H": H,
+                       "N": N, "d": D, "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (512 MB write outside the timed events)"},
+            "timing": "value: CUDA-graph replay of the step; breakdown: eager calls, events per fa_bwd call",
+            "breakdown_ms": {"bwd_noncausal": comp[0], "bwd_causal": comp[1]},
+            "breakdown_tflops": {"bwd_noncausal": flops_bwd(False) / comp[0] / 1e9,
+                                 "bwd_causal": flops_bwd(True) / comp[1] / 1e9},
+            "roofline": {"kernel": "fa_bwd non-causal (prologue + attn_bwd_kernel<128,nc> + dQ conversion)",
+                         "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "peak_source": f"{peak_src} cuBLAS bf16 (burst)"},
+            "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
+                    "note": "Q, K, V, dO and both masks' O and LSE copied in, the six gradients copied out, per "
+                            "step; steps pipelined over three CUDA streams (copy in, compute, copy out)"},
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
+        }
+        if not args.no_cpu_baseline and world == 1:
+            fl, sec, cores, heads = oracle_bwd_sample(args.cpu_seconds, SEED)
+            line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                    "sample": f"{heads} whole heads (N={N}, d={D}) of the workload, non-causal and "
+                                              f"causal alternately, fp64 numpy, {sec:.1f} s"}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
 # ------------------------------------------------------------------- main --
 def main():
     ap = argparse.ArgumentParser()
@@ -519,9 +663,31 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["step", "decode"], default="step")
+    ap.add_argument("--workload", choices=["step", "decode", "bwd"], default="step")
     args = ap.parse_args()
     world, rank, local = dist_setup()
+
+    if args.impl == "reference" and args.workload == "bwd":
+        if rank == 0:
+            oracle_bwd_sample(1.0, SEED + 100)
+            runs = [oracle_bwd_sample(args.cpu_seconds / 2, SEED + i) for i in range(args.steps)]
+            fl, sec = sum(r[0] for r in runs), sum(r[1] for r in runs)
+            val = fl / sec / 1e12
+            line = {
+                "impl": "reference", "metric": BWD_METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1))",
+                "config": {"workload": f"bwd b{B}h{H}n{N}d{D}: fa_bwd non-causal + fa_bwd causal", "B": B, "H": H,
+                           "N": N, "d": D, "l2": "n/a (CPU)"},
+                "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": runs[0][2], "kind": "oracle",
+                                 "sample": f"{runs[0][3]} whole heads per step, non-causal and causal alternately, "
+                                           "fp64 numpy"},
+                "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            }
+            print(json.dumps(line), flush=True)
+        dist_done(world)
+        return
 
     if args.impl == "reference":
         if rank == 0:
@@ -551,6 +717,9 @@ def main():
     torch.cuda.set_device(local)
     if args.workload == "decode":
         run_decode(args, world, rank)
+        return
+    if args.workload == "bwd":
+        run_bwd(args, world, rank)
         return
     step = Step(SEED + rank)
     graph = capture_step(step)

@@ -16,16 +16,17 @@
 //  * one CTA per (batch·head, tile of 128 keys). Its K_j and V_j stay in
 //    shared memory, and dK_j and dV_j accumulate in TMEM over the query tiles
 //    (causal: from the diagonal tile on, heaviest key tiles launched first);
-//  * per query tile i (128 rows, Q_i and dO_i through a ring of stages loaded
-//    by TMA): Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ in TMEM, keys on the lanes;
-//  * two softmax warpgroups, 64 queries each, form P and dS = P (dP - D) for
-//    their key rows. They write P back over Sᵀ as bf16 pairs: the A operand of
-//    dV += Pᵀ dO_i, read from TMEM. They write dSᵀ to shared memory in the
-//    128-byte-swizzle layout: the K-major A operand of dK += dSᵀ Q_i and, read
-//    MN-major, the A operand of dQ_i = dS K_j;
-//  * dQ_i lands in the dP columns. The same warps add it into an fp32
-//    workspace with vector reductions while the tensor core runs dV, dK and
-//    the next Sᵀ;
+//  * per query tile i (128 rows): TMA brings Q_i, dO_i and the tile's LSE and D
+//    through a ring of stages; Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ land in TMEM
+//    with keys on the lanes, each with its own barrier;
+//  * two softmax warpgroups, 64 queries each, form P from Sᵀ (while dPᵀ is
+//    still being computed), then dS = P (dP - D). They write P and dSᵀ back
+//    over Sᵀ as bf16 pairs, the TMEM A operands of dV += Pᵀ dO_i and
+//    dK += dSᵀ Q_i, and dSᵀ to shared memory in the 128-byte-swizzle layout,
+//    read MN-major as the A operand of dQ_i = dS K_j;
+//  * dQ_i is issued first and lands in the dP columns. The softmax warps add it
+//    into an fp32 workspace with vector reductions while the tensor core runs
+//    dV, dK and the next Sᵀ; the next dPᵀ waits only for that read-out;
 //  * a prologue kernel forms D_i and the LSE in log2 units, padded per head to
 //    whole tiles (+inf and 0, so that padded queries get P = 0). An epilogue
 //    kernel scales dQ and rounds it to bf16.
@@ -47,17 +48,28 @@ struct BwdCfg {
   static constexpr int DS_TILE = BK * BQ * 2;    // dSᵀ, 128 keys x 128 queries bf16
   static constexpr int NST = D == 128 ? 2 : 3;   // Q_i / dO_i stages
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int SMEM_BYTES = 1024 + 2 * TILE + DS_TILE + NST * STAGE;
+  static constexpr int LD_BYTES = 2 * BQ * 4;    // per stage: the step's LSE log2(e), then its D
+  // Dynamic shared memory, 1024-byte aligned (the swizzled tiles need it; the
+  // kernel checks): K_j, V_j, dSᵀ, the Q_i / dO_i stages, their LSE / D, barriers.
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_DS = 2 * TILE;
+  static constexpr int OFF_STAGE = OFF_DS + DS_TILE;
+  static constexpr int OFF_LD = OFF_STAGE + NST * STAGE;
+  static constexpr int OFF_BAR = OFF_LD + NST * LD_BYTES;
+  static constexpr int N_BARS = 1 + 2 * NST + 8;
+  static constexpr int SMEM_BYTES = OFF_BAR + 8 * N_BARS + 16;  // + TMEM address and abort flag
   static constexpr int THREADS = 384;            // 8 softmax warps, MMA warp, TMA warp, 2 idle
   static constexpr int MMA_WARP = 8;
   static constexpr int TMA_WARP = 9;
-  static constexpr uint32_t S_COL = 0;           // Sᵀ, then P as bf16 pairs (64 columns)
-  static constexpr uint32_t DP_COL = 128;        // dPᵀ, then dQ_i (D columns)
+  // TMEM columns. S region: Sᵀ; then P (bf16 pairs, columns 0-63) and dSᵀ
+  // (bf16 pairs, columns 64-127). dP region: dPᵀ, then dQ_i (D columns).
+  static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t DP_COL = 128;
   static constexpr uint32_t DV_COL = 256;
   static constexpr uint32_t DK_COL = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(D == 64 || D == 128, "head dim");
-  static_assert(SMEM_BYTES + 256 <= 227 * 1024, "shared memory");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 struct BwdParams {
@@ -77,6 +89,14 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Untiled bulk copy global -> this CTA's shared memory (both addresses 16-byte
+// aligned, bytes a multiple of 16), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (the tensor core reads its shared-memory operands through it).
@@ -98,49 +118,71 @@ __global__ void __launch_bounds__(384, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = sm;
-  uint8_t* sV = sK + C::TILE;
-  uint8_t* sdS = sV + C::TILE;
-  uint8_t* sStage = sdS + C::DS_TILE;  // stage s: Q_i then dO_i
-
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[C::NST], bar_empty[C::NST];
-  __shared__ __align__(8) uint64_t bar_s, bar_sread, bar_p, bar_dq, bar_dqfree, bar_done, bar_drain;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    // the 128-byte-swizzle tiles need 1024-byte alignment: refuse, loudly
+    if (threadIdx.x == 0 && atomicCAS(&g_fa_status.code, 0u, 3u /*FA_ERR_ALIGNMENT*/) == 0u) {
+      g_fa_status.site = 70;
+      g_fa_status.block = blockIdx.x;
+    }
+    return;
+  }
+  uint8_t* sK = smem_raw;
+  uint8_t* sV = smem_raw + C::OFF_V;
+  uint8_t* sdS = smem_raw + C::OFF_DS;
+  uint8_t* sStage = smem_raw + C::OFF_STAGE;  // stage s: Q_i then dO_i
+  const float* sLD = reinterpret_cast<const float*>(smem_raw + C::OFF_LD);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + C::OFF_BAR);
+  uint64_t* bar_kv = bars;
+  uint64_t* bar_full = bars + 1;
+  uint64_t* bar_empty = bars + 1 + C::NST;
+  uint64_t* bar_S = bars + 1 + 2 * C::NST;  // Sᵀ_i in TMEM
+  uint64_t* bar_dP = bar_S + 1;             // dPᵀ_i in TMEM
+  uint64_t* bar_sread = bar_S + 2;          // every softmax warp has read Sᵀ_i
+  uint64_t* bar_p = bar_S + 3;              // P_i, dSᵀ_i written (TMEM and shared memory)
+  uint64_t* bar_dq = bar_S + 4;             // dQ_i in TMEM
+  uint64_t* bar_dqfree = bar_S + 5;         // dQ_i read out
+  uint64_t* bar_done = bar_S + 6;           // dK, dV complete
+  uint64_t* bar_drain = bar_S + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   // causal: key tile 0 (the most query tiles) first
   const int kt = static_cast<int>(blockIdx.x) / p.BH;
   const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Query tile of step i. Causal: from the diagonal tile on. Non-causal: all
+  // tiles, starting at the CTA's own key tile, so that the CTAs of one head
+  // that run at the same time add into different dQ rows.
   const int qt0 = CAUSAL ? kt : 0;
   const int n_steps = p.n_t - qt0;
+  auto q_tile = [&](int i) { return CAUSAL ? kt + i : (kt + i) % p.n_t; };
 
   if (threadIdx.x == 0) {
-    abort_flag = 0;
-    mbar_init(&bar_kv, 1);
+    *abort_flag = 0;
+    mbar_init(bar_kv, 1);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&bar_full[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_sread, 8);  // one arrival per softmax warp
-    mbar_init(&bar_p, 8);
-    mbar_init(&bar_dq, 1);
-    mbar_init(&bar_dqfree, 8);
-    mbar_init(&bar_done, 1);
-    mbar_init(&bar_drain, 1);
+    mbar_init(bar_S, 1);
+    mbar_init(bar_dP, 1);
+    mbar_init(bar_sread, 8);  // one arrival per softmax warp
+    mbar_init(bar_p, 8);
+    mbar_init(bar_dq, 1);
+    mbar_init(bar_dqfree, 8);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
   if (warp == C::MMA_WARP) {
-    tmem_alloc(&tmem_slot, C::TMEM_COLS);
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tbase = tmem_slot;
+  const uint32_t tbase = *tmem_slot;
   DevStatus* st = &g_fa_status;
 
   if (warp == C::TMA_WARP && lane == 0) {
@@ -149,34 +191,39 @@ __global__ void __launch_bounds__(384, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
-    mbar_arrive_expect_tx(&bar_kv, 2 * C::TILE);
+    mbar_arrive_expect_tx(bar_kv, 2 * C::TILE);
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sK + c * C::CHUNK, &tmK, &bar_kv, c * 64, kt * C::BK, bh);
-      tma_load_3d(sV + c * C::CHUNK, &tmV, &bar_kv, c * 64, kt * C::BK, bh);
+      tma_load_3d(sK + c * C::CHUNK, &tmK, bar_kv, c * 64, kt * C::BK, bh);
+      tma_load_3d(sV + c * C::CHUNK, &tmV, bar_kv, c * 64, kt * C::BK, bh);
     }
+    const float* lse2h = p.lse2 + static_cast<size_t>(bh) * p.Npad;
+    const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
     bool ok = true;
     int issued = 0;
     for (int i = 0; i < n_steps && ok; ++i) {
       const int slot = i % C::NST, round = i / C::NST;
-      if (round > 0) ok = mbar_wait(&bar_empty[slot], (round - 1) & 1, &abort_flag, st, 50);
+      if (round > 0) ok = mbar_wait(&bar_empty[slot], (round - 1) & 1, abort_flag, st, 50);
       if (!ok) break;
       uint8_t* dst = sStage + slot * C::STAGE;
-      const int q0 = (qt0 + i) * C::BQ;
-      mbar_arrive_expect_tx(&bar_full[slot], 2 * C::TILE);
+      uint8_t* ld = smem_raw + C::OFF_LD + slot * C::LD_BYTES;
+      const int q0 = q_tile(i) * C::BQ;
+      mbar_arrive_expect_tx(&bar_full[slot], 2 * C::TILE + C::LD_BYTES);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_3d(dst + c * C::CHUNK, &tmQ, &bar_full[slot], c * 64, q0, bh);
         tma_load_3d(dst + C::TILE + c * C::CHUNK, &tmdO, &bar_full[slot], c * 64, q0, bh);
       }
+      bulk_load(ld, lse2h + q0, C::BQ * 4, &bar_full[slot]);
+      bulk_load(ld + C::BQ * 4, dvh + q0, C::BQ * 4, &bar_full[slot]);
       ++issued;
     }
     // every load this thread issued lands before the CTA can exit
-    mbar_drain_bwd(&bar_kv, 0);
+    mbar_drain_bwd(bar_kv, 0);
     for (int i = issued - C::NST; i < issued; ++i)
       if (i >= 0) mbar_drain_bwd(&bar_full[i % C::NST], (i / C::NST) & 1);
   } else if (warp == C::MMA_WARP && lane == 0) {
     // ---------------------------------------------------------- MMA issuer --
-    constexpr uint32_t idesc_kq = idesc_make(1u, 128, 128, false);        // A, B K-major
-    constexpr uint32_t idesc_bmn = idesc_make(1u, 128, D, true);          // B MN-major
+    constexpr uint32_t idesc_kq = idesc_make(1u, 128, 128, false);            // A, B K-major
+    constexpr uint32_t idesc_bmn = idesc_make(1u, 128, D, true);              // B MN-major
     constexpr uint32_t idesc_dq = idesc_make(1u, 128, D, true) | (1u << 15);  // A and B MN-major
     const uint32_t kaddr = smem_u32(sK), vaddr = smem_u32(sV), dsaddr = smem_u32(sdS);
     const uint32_t stage0 = smem_u32(sStage);
@@ -189,57 +236,58 @@ __global__ void __launch_bounds__(384, 1)
                     sdesc_sw128(b + chunk * C::CHUNK + within, 0, 1024), idesc_kq, kk > 0 ? 1u : 0u);
       }
     };
-    bool ok = mbar_wait(&bar_kv, 0, &abort_flag, st, 51);
-    if (ok) ok = mbar_wait(&bar_full[0], 0, &abort_flag, st, 52);
+    bool ok = mbar_wait(bar_kv, 0, abort_flag, st, 51);
+    if (ok) ok = mbar_wait(&bar_full[0], 0, abort_flag, st, 52);
     if (ok) {
       tc_fence_after();
       issue_rows(C::S_COL, kaddr, stage0);
+      mma_commit(bar_S);
       issue_rows(C::DP_COL, vaddr, stage0 + C::TILE);
-      mma_commit(&bar_s);
+      mma_commit(bar_dP);
     }
     for (int i = 0; i < n_steps && ok; ++i) {
       const int slot = i % C::NST;
       const uint32_t qaddr = stage0 + slot * C::STAGE, doaddr = qaddr + C::TILE;
-      ok = mbar_wait(&bar_p, i & 1, &abort_flag, st, 53, 0u);
+      ok = mbar_wait(bar_p, i & 1, abort_flag, st, 53, 0u);
       if (!ok) break;
       tc_fence_after();
-      // dQ_i = dS K_j: A = dSᵀ read MN-major (queries along rows), B = K_j MN-major; 16 keys per MMA
+      // dQ_i = dS K_j into the dP columns (read by the softmax warps while the
+      // products below run): A = dSᵀ read MN-major, B = K_j MN-major; 16 keys per MMA
 #pragma unroll
       for (int kk = 0; kk < C::BK / 16; ++kk)
         mma_bf16_ss(tbase + C::DP_COL, sdesc_sw128(dsaddr + kk * 16 * 128, C::CHUNK, 1024),
                     sdesc_sw128(kaddr + kk * 16 * 128, C::CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
-      mma_commit(&bar_dq);
-      // dV += Pᵀ dO_i: A = P from TMEM (bf16 pairs, keys on lanes), B = dO_i MN-major; 16 queries per MMA
+      mma_commit(bar_dq);
+      // dV += Pᵀ dO_i and dK += dSᵀ Q_i: A from TMEM (bf16 pairs, keys on lanes),
+      // B = dO_i / Q_i MN-major; 16 queries per MMA
 #pragma unroll
       for (int kk = 0; kk < C::BQ / 16; ++kk)
         mma_bf16_ts(tbase + C::DV_COL, tbase + C::S_COL + kk * 8, sdesc_sw128(doaddr + kk * 16 * 128, C::CHUNK, 1024),
                     idesc_bmn, (i > 0 || kk > 0) ? 1u : 0u);
-      // dK += dSᵀ Q_i: A = dSᵀ K-major, B = Q_i MN-major
 #pragma unroll
-      for (int kk = 0; kk < C::BQ / 16; ++kk) {
-        const int kb = kk * 32, chunk = kb / 128, within = kb % 128;
-        mma_bf16_ss(tbase + C::DK_COL, sdesc_sw128(dsaddr + chunk * C::CHUNK + within, 0, 1024),
+      for (int kk = 0; kk < C::BQ / 16; ++kk)
+        mma_bf16_ts(tbase + C::DK_COL, tbase + C::S_COL + 64 + kk * 8,
                     sdesc_sw128(qaddr + kk * 16 * 128, C::CHUNK, 1024), idesc_bmn, (i > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(&bar_empty[slot]);  // Q_i and dO_i read
+      mma_commit(&bar_empty[slot]);  // Q_i, dO_i and their LSE / D read
       if (i + 1 < n_steps) {
         const int ns = (i + 1) % C::NST;
         const uint32_t nq = stage0 + ns * C::STAGE;
-        ok = mbar_wait(&bar_full[ns], ((i + 1) / C::NST) & 1, &abort_flag, st, 54);
+        ok = mbar_wait(&bar_full[ns], ((i + 1) / C::NST) & 1, abort_flag, st, 54);
         if (!ok) break;
         tc_fence_after();
-        issue_rows(C::S_COL, kaddr, nq);  // after dV_i, which reads P from these columns
-        ok = mbar_wait(&bar_dqfree, i & 1, &abort_flag, st, 55, 0u);
+        issue_rows(C::S_COL, kaddr, nq);  // after dV_i and dK_i, which read P and dS from these columns
+        mma_commit(bar_S);
+        ok = mbar_wait(bar_dqfree, i & 1, abort_flag, st, 55, 0u);
         if (!ok) break;
         tc_fence_after();
         issue_rows(C::DP_COL, vaddr, nq + C::TILE);
-        mma_commit(&bar_s);
+        mma_commit(bar_dP);
       }
     }
-    if (ok) mma_commit(&bar_done);
+    if (ok) mma_commit(bar_done);
     // TMEM is freed below only after every issued MMA has finished
-    mma_commit(&bar_drain);
-    mbar_drain_bwd(&bar_drain, 0);
+    mma_commit(bar_drain);
+    mbar_drain_bwd(bar_drain, 0);
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
     const int g = static_cast<int>(warp >> 2);  // query columns 64g .. 64g + 63
@@ -247,90 +295,13 @@ __global__ void __launch_bounds__(384, 1)
     const int r = static_cast<int>(lane_base + lane);  // key row (Sᵀ lane); query row for dQ
     const int kr = kt * C::BK + r;
     const uint32_t row_addr = tbase + (lane_base << 16);
-    const float* lse2h = p.lse2 + static_cast<size_t>(bh) * p.Npad;
-    const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
     const uint32_t ds_row = smem_u32(sdS) + g * C::CHUNK + r * 128;
     const float sl2 = p.scale_log2;
-    bool ok = true;
-    for (int i = 0; i < n_steps; ++i) {
-      const int q0 = (qt0 + i) * C::BQ;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_s, i & 1, &abort_flag, st, 60));
-      if (!ok) break;
+    // dQ_i rows (queries on lanes) added into the fp32 accumulator
+    auto dq_out = [&](int i) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, st, 62))) return false;
       tc_fence_after();
-      // P = exp2(scale log2(e) s - LSE log2(e)) for this key row and 64 queries
-      float pv[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(row_addr + C::S_COL + 64 * g + 32 * c, sv);
-        tmem_wait_ld_dep32(sv);
-        const float4* l4 = reinterpret_cast<const float4*>(lse2h + q0 + 64 * g + 32 * c);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 l = __ldg(l4 + u);
-          pv[32 * c + 4 * u + 0] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 0]), sl2, -l.x));
-          pv[32 * c + 4 * u + 1] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 1]), sl2, -l.y));
-          pv[32 * c + 4 * u + 2] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 2]), sl2, -l.z));
-          pv[32 * c + 4 * u + 3] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 3]), sl2, -l.w));
-        }
-      }
-      // this warp's reads of Sᵀ are done (P overwrites those columns below)
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_sread);
-      if (kr >= p.N) {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) pv[e] = 0.f;
-      }
-      if (CAUSAL && i == 0) {
-        // diagonal tile: query q0 + 64g + e sees key kr iff 64g + e >= r
-#pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (64 * g + e < r) pv[e] = 0.f;
-      }
-      // dS = P (dP - D), rounded to bf16, into row r of dSᵀ (swizzled 16-byte units)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t dv[32];
-        tmem_ld32(row_addr + C::DP_COL + 64 * g + 32 * c, dv);
-        tmem_wait_ld_dep32(dv);
-        const float4* d4 = reinterpret_cast<const float4*>(dvh + q0 + 64 * g + 32 * c);
-        uint32_t pk[16];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 dd = __ldg(d4 + u);
-          const float* pp = &pv[32 * c + 4 * u];
-          pk[2 * u] = pack_bf16x2(pp[0] * (__uint_as_float(dv[4 * u + 0]) - dd.x),
-                                  pp[1] * (__uint_as_float(dv[4 * u + 1]) - dd.y));
-          pk[2 * u + 1] = pack_bf16x2(pp[2] * (__uint_as_float(dv[4 * u + 2]) - dd.z),
-                                      pp[3] * (__uint_as_float(dv[4 * u + 3]) - dd.w));
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t unit = static_cast<uint32_t>(4 * c + u) ^ static_cast<uint32_t>(r & 7);
-          st_shared_v4(ds_row + unit * 16, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-      }
-      // P as bf16 pairs over Sᵀ, once every softmax warp has read its Sᵀ columns
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_sread, i & 1, &abort_flag, st, 61));
-      if (!ok) break;
-      tc_fence_after();
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-        tmem_st32(row_addr + C::S_COL + 32 * g, pk);
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_p);
-      // dQ_i rows (queries on lanes): add into the fp32 accumulator
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_dq, i & 1, &abort_flag, st, 62));
-      if (!ok) break;
-      tc_fence_after();
-      const int qrow = q0 + r;
+      const int qrow = q_tile(i) * C::BQ + r;
       float* dqrow = p.dq_acc + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
 #pragma unroll
       for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
@@ -346,10 +317,94 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_dqfree);
+      if (lane == 0) mbar_arrive(bar_dqfree);
+      return true;
+    };
+    bool ok = true;
+    for (int i = 0; i < n_steps; ++i) {
+      if (i > 0 && !(ok = dq_out(i - 1))) break;
+      const float* lse_s = sLD + (i % C::NST) * (C::LD_BYTES / 4) + 64 * g;  // this warpgroup's 64 queries
+      const float* d_s = lse_s + C::BQ;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_S, i & 1, abort_flag, st, 60));
+      if (!ok) break;
+      tc_fence_after();
+      // P = exp2(scale log2(e) s - LSE log2(e)) for this key row and 64 queries
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(row_addr + C::S_COL + 64 * g + 32 * c, sv);
+        tmem_wait_ld_dep32(sv);
+        const float4* l4 = reinterpret_cast<const float4*>(lse_s + 32 * c);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 l = l4[u];
+          pv[32 * c + 4 * u + 0] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 0]), sl2, -l.x));
+          pv[32 * c + 4 * u + 1] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 1]), sl2, -l.y));
+          pv[32 * c + 4 * u + 2] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 2]), sl2, -l.z));
+          pv[32 * c + 4 * u + 3] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 3]), sl2, -l.w));
+        }
+      }
+      // this warp's reads of Sᵀ are done (P and dS overwrite those columns below)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sread);
+      if (kr >= p.N) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) pv[e] = 0.f;
+      }
+      if (CAUSAL && i == 0) {
+        // diagonal tile: query q0 + 64g + e sees key kr iff 64g + e >= r
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (64 * g + e < r) pv[e] = 0.f;
+      }
+      // dS = P (dP - D), rounded to bf16: into row r of dSᵀ in shared memory
+      // (swizzled 16-byte units) and kept as pairs for TMEM
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dP, i & 1, abort_flag, st, 64));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dsp[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dv[32];
+        tmem_ld32(row_addr + C::DP_COL + 64 * g + 32 * c, dv);
+        tmem_wait_ld_dep32(dv);
+        const float4* d4 = reinterpret_cast<const float4*>(d_s + 32 * c);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 dd = d4[u];
+          const float* pp = &pv[32 * c + 4 * u];
+          dsp[16 * c + 2 * u] = pack_bf16x2(pp[0] * (__uint_as_float(dv[4 * u + 0]) - dd.x),
+                                            pp[1] * (__uint_as_float(dv[4 * u + 1]) - dd.y));
+          dsp[16 * c + 2 * u + 1] = pack_bf16x2(pp[2] * (__uint_as_float(dv[4 * u + 2]) - dd.z),
+                                                pp[3] * (__uint_as_float(dv[4 * u + 3]) - dd.w));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t unit = static_cast<uint32_t>(4 * c + u) ^ static_cast<uint32_t>(r & 7);
+          st_shared_v4(ds_row + unit * 16, dsp[16 * c + 4 * u], dsp[16 * c + 4 * u + 1], dsp[16 * c + 4 * u + 2],
+                       dsp[16 * c + 4 * u + 3]);
+        }
+      }
+      uint32_t pp[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) pp[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+      // P and dSᵀ as bf16 pairs over Sᵀ, once every softmax warp has read its Sᵀ columns
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_sread, i & 1, abort_flag, st, 61));
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st32(row_addr + C::S_COL + 32 * g, pp);
+      tmem_st32(row_addr + C::S_COL + 64 + 32 * g, dsp);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p);
     }
+    if (ok && n_steps > 0) ok = dq_out(n_steps - 1);
     // ------------------------------------------------------------ epilogue --
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_done, 0, &abort_flag, st, 63));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, st, 63));
     if (ok) {
       tc_fence_after();
       const size_t orow = (static_cast<size_t>(bh) * p.N + (kr < p.N ? kr : 0)) * D;
