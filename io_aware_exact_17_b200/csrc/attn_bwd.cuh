@@ -27,8 +27,8 @@
 //  * dQ_i is issued first and lands in the dP columns. The softmax warps add it
 //    into an fp32 workspace with vector reductions while the tensor core runs
 //    dV, dK and the next Sᵀ; the next dPᵀ waits only for that read-out;
-//  * a prologue kernel forms D_i and the LSE in log2 units, padded per head to
-//    whole tiles (+inf and 0, so that padded queries get P = 0). An epilogue
+//  * a prologue kernel forms D_i and -LSE in log2 units, padded per head to
+//    whole tiles (-inf and 0, so that padded queries get P = 0). An epilogue
 //    kernel scales dQ and rounds it to bf16.
 // TMEM holds Sᵀ (128 columns), dPᵀ / dQ (128), dV (d) and dK (d): d <= 128.
 #pragma once
@@ -48,7 +48,7 @@ struct BwdCfg {
   static constexpr int DS_TILE = BK * BQ * 2;    // dSᵀ, 128 keys x 128 queries bf16
   static constexpr int NST = D == 128 ? 2 : 3;   // Q_i / dO_i stages
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int LD_BYTES = 2 * BQ * 4;    // per stage: the step's LSE log2(e), then its D
+  static constexpr int LD_BYTES = 2 * BQ * 4;    // per stage: the step's -LSE log2(e), then its D
   // Dynamic shared memory, 1024-byte aligned (the swizzled tiles need it; the
   // kernel checks): K_j, V_j, dSᵀ, the Q_i / dO_i stages, their LSE / D, barriers.
   static constexpr int OFF_V = TILE;
@@ -76,7 +76,7 @@ struct BwdParams {
   __nv_bfloat16* dk;        // [BH][N][D]
   __nv_bfloat16* dv;        // [BH][N][D]
   float* dq_acc;            // [BH][N][D] fp32, zeroed by the prologue; dQ / scale
-  const float* lse2;        // [BH][Npad]: LSE * log2(e), +inf past N
+  const float* nlse2;       // [BH][Npad]: -LSE * log2(e), -inf past N
   const float* dvec;        // [BH][Npad]: D_i = dO_i · O_i, 0 past N
   int BH, N, Npad, n_t;     // n_t = Npad / 128 tiles per head
   float scale, scale_log2;  // scale, scale * log2(e)
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_load_3d(sK + c * C::CHUNK, &tmK, bar_kv, c * 64, kt * C::BK, bh);
       tma_load_3d(sV + c * C::CHUNK, &tmV, bar_kv, c * 64, kt * C::BK, bh);
     }
-    const float* lse2h = p.lse2 + static_cast<size_t>(bh) * p.Npad;
+    const float* nlse2h = p.nlse2 + static_cast<size_t>(bh) * p.Npad;
     const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
     bool ok = true;
     int issued = 0;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(384, 1)
         tma_load_3d(dst + c * C::CHUNK, &tmQ, &bar_full[slot], c * 64, q0, bh);
         tma_load_3d(dst + C::TILE + c * C::CHUNK, &tmdO, &bar_full[slot], c * 64, q0, bh);
       }
-      bulk_load(ld, lse2h + q0, C::BQ * 4, &bar_full[slot]);
+      bulk_load(ld, nlse2h + q0, C::BQ * 4, &bar_full[slot]);
       bulk_load(ld + C::BQ * 4, dvh + q0, C::BQ * 4, &bar_full[slot]);
       ++issued;
     }
@@ -296,24 +296,27 @@ __global__ void __launch_bounds__(384, 1)
     const int kr = kt * C::BK + r;
     const uint32_t row_addr = tbase + (lane_base << 16);
     const uint32_t ds_row = smem_u32(sdS) + g * C::CHUNK + r * 128;
-    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
     // dQ_i rows (queries on lanes) added into the fp32 accumulator
     auto dq_out = [&](int i) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, st, 62))) return false;
       tc_fence_after();
       const int qrow = q_tile(i) * C::BQ + r;
       float* dqrow = p.dq_acc + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
+      constexpr int NC = D / 64;  // 32-column chunks of this warpgroup's D / 2 columns
+      uint32_t v[NC][32];
 #pragma unroll
-      for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(row_addr + C::DP_COL + c0, v);
-        tmem_wait_ld_dep32(v);
-        if (qrow < p.N) {
+      for (int c = 0; c < NC; ++c) tmem_ld32(row_addr + C::DP_COL + g * (D / 2) + 32 * c, v[c]);
+#pragma unroll
+      for (int c = 0; c < NC; ++c) tmem_wait_ld_dep32(v[c]);
+      if (qrow < p.N) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            red_add_v4(dqrow + c0 + 4 * u, __uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                       __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
-        }
+            red_add_v4(dqrow + g * (D / 2) + 32 * c + 4 * u, __uint_as_float(v[c][4 * u]),
+                       __uint_as_float(v[c][4 * u + 1]), __uint_as_float(v[c][4 * u + 2]),
+                       __uint_as_float(v[c][4 * u + 3]));
       }
       tc_fence_before();
       __syncwarp();
@@ -330,19 +333,27 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       // P = exp2(scale log2(e) s - LSE log2(e)) for this key row and 64 queries
       float pv[64];
+      uint32_t sv2[2][32];
+      tmem_ld32(row_addr + C::S_COL + 64 * g, sv2[0]);
+      tmem_wait_ld_dep32(sv2[0]);
+      tmem_ld32(row_addr + C::S_COL + 64 * g + 32, sv2[1]);  // in flight during chunk 0's exps
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(row_addr + C::S_COL + 64 * g + 32 * c, sv);
-        tmem_wait_ld_dep32(sv);
+        uint32_t* sv = sv2[c];
+        if (c == 1) tmem_wait_ld_dep32(sv);
         const float4* l4 = reinterpret_cast<const float4*>(lse_s + 32 * c);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float4 l = l4[u];
-          pv[32 * c + 4 * u + 0] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 0]), sl2, -l.x));
-          pv[32 * c + 4 * u + 1] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 1]), sl2, -l.y));
-          pv[32 * c + 4 * u + 2] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 2]), sl2, -l.z));
-          pv[32 * c + 4 * u + 3] = ex2_approx(fmaf(__uint_as_float(sv[4 * u + 3]), sl2, -l.w));
+          const float4 l = l4[u];  // -LSE log2(e) of four queries
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * u + 0]), __uint_as_float(sv[4 * u + 1])), sl2x2,
+                           f2_pack(l.x, l.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * u + 2]), __uint_as_float(sv[4 * u + 3])), sl2x2,
+                           f2_pack(l.z, l.w)), x2, x3);
+          pv[32 * c + 4 * u + 0] = ex2_approx(x0);
+          pv[32 * c + 4 * u + 1] = ex2_approx(x1);
+          pv[32 * c + 4 * u + 2] = ex2_approx(x2);
+          pv[32 * c + 4 * u + 3] = ex2_approx(x3);
         }
       }
       // this warp's reads of Sᵀ are done (P and dS overwrite those columns below)
@@ -365,20 +376,28 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t dsp[32];
+      uint32_t dv2[2][32];
+      tmem_ld32(row_addr + C::DP_COL + 64 * g, dv2[0]);
+      tmem_wait_ld_dep32(dv2[0]);
+      tmem_ld32(row_addr + C::DP_COL + 64 * g + 32, dv2[1]);  // in flight during chunk 0
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t dv[32];
-        tmem_ld32(row_addr + C::DP_COL + 64 * g + 32 * c, dv);
-        tmem_wait_ld_dep32(dv);
+        uint32_t* dv = dv2[c];
+        if (c == 1) tmem_wait_ld_dep32(dv);
         const float4* d4 = reinterpret_cast<const float4*>(d_s + 32 * c);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float4 dd = d4[u];
           const float* pp = &pv[32 * c + 4 * u];
-          dsp[16 * c + 2 * u] = pack_bf16x2(pp[0] * (__uint_as_float(dv[4 * u + 0]) - dd.x),
-                                            pp[1] * (__uint_as_float(dv[4 * u + 1]) - dd.y));
-          dsp[16 * c + 2 * u + 1] = pack_bf16x2(pp[2] * (__uint_as_float(dv[4 * u + 2]) - dd.z),
-                                                pp[3] * (__uint_as_float(dv[4 * u + 3]) - dd.w));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(pp[0], pp[1]),
+                           f2_sub(f2_pack(__uint_as_float(dv[4 * u + 0]), __uint_as_float(dv[4 * u + 1])),
+                                  f2_pack(dd.x, dd.y))), a0, a1);
+          f2_unpack(f2_mul(f2_pack(pp[2], pp[3]),
+                           f2_sub(f2_pack(__uint_as_float(dv[4 * u + 2]), __uint_as_float(dv[4 * u + 3])),
+                                  f2_pack(dd.z, dd.w))), a2, a3);
+          dsp[16 * c + 2 * u] = pack_bf16x2(a0, a1);
+          dsp[16 * c + 2 * u + 1] = pack_bf16x2(a2, a3);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -442,12 +461,12 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// Prologue: per padded query row, D_i = dO_i · O_i and LSE_i log2(e) (+inf and
-// 0 past N), and zero row i of the dQ accumulator. One warp per row.
+// Prologue: per padded query row, D_i = dO_i · O_i and -LSE_i log2(e) (-inf
+// and 0 past N), and zero row i of the dQ accumulator. One warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
-                                                            const float* __restrict__ lse, float* lse2, float* dvec,
+                                                            const float* __restrict__ lse, float* nlse2, float* dvec,
                                                             float* dq_acc, int BH, int N, int Npad) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const uint32_t lane = lane_id();
@@ -455,7 +474,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
   if (i >= N) {
     if (lane == 0) {
-      lse2[row] = INFINITY;
+      nlse2[row] = -INFINITY;
       dvec[row] = 0.f;
     }
     return;
@@ -481,7 +500,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   if (lane == 0) {
-    lse2[row] = lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f;
+    nlse2[row] = lse[static_cast<size_t>(bh) * N + i] * -1.4426950408889634f;
     dvec[row] = acc;
   }
 }

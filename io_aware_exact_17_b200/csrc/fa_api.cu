@@ -392,9 +392,9 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   const int BH = B * H;
   const int Npad = bwd_npad(N);
   float* dq_acc = static_cast<float*>(workspace);
-  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+  float* nlse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                          round256(static_cast<size_t>(BH) * N * D * sizeof(float)));
-  float* dvec = lse2 + round256(static_cast<size_t>(BH) * Npad * sizeof(float)) / sizeof(float);
+  float* dvec = nlse2 + round256(static_cast<size_t>(BH) * Npad * sizeof(float)) / sizeof(float);
   CUtensorMap tmQ, tmK, tmV, tmdO;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!fa::make_tmap_3d(&tmQ, q, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmK, k, bf, 2, D, N, BH, 64, 128) ||
@@ -402,7 +402,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     return FA_ERR_CUDA;
   const long long rows = static_cast<long long>(BH) * Npad;
   fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, dq_acc, BH, N,
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH, N,
       Npad);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   auto kernel = fa::attn_bwd_kernel<D, CAUSAL>;
@@ -412,7 +412,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dq_acc = dq_acc;
-  p.lse2 = lse2;
+  p.nlse2 = nlse2;
   p.dvec = dvec;
   p.BH = BH;
   p.N = N;
