@@ -208,3 +208,12 @@ def test_bwd_argument_errors(lib):
         assert bwd(**{name: MIS}) == binding.FA_ERR_ALIGNMENT, name
     assert bwd(lse=A + 2) == binding.FA_ERR_ALIGNMENT
     assert bwd(ws=A + 16) == binding.FA_ERR_ALIGNMENT
+
+
+def test_bwd_binding_rejects_host_tensors_and_bad_shapes():
+    import torch
+
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 8)
+    with pytest.raises(binding.FaError):
+        binding.bwd(q, q, q, q, lse, q)  # host tensors: no CPU path
