@@ -88,6 +88,49 @@ def test_rotation_leaves_qkT_unchanged(use_signs):
     np.testing.assert_allclose(oracle.rotate(q, s) @ oracle.rotate(k, s).T, q @ k.T, atol=1e-12)
 
 
+def rotation_golden_holds(rotation_matrix) -> bool:
+    """True iff ``rotation_matrix(d, signs)`` reproduces every hand-derived
+    case of tests/golden/rotation_sign_order.json: signs applied first, then
+    the Hadamard (M = D H_d / sqrt(d), subsection 3, step 1), and none of the
+    values the other order (H_d D) would give."""
+    g = json.loads((GOLDEN / "rotation_sign_order.json").read_text())
+    ok = True
+    for c in g["cases"]:
+        x = np.array(c["x"], dtype=np.float64)
+        got = x @ rotation_matrix(c["d"], np.array(c["signs"], dtype=np.float64))
+        want = np.array(c["expected"]["numer"], dtype=np.float64) / np.sqrt(c["expected"]["denom_sqrt"])
+        wrong = np.array(c["wrong_order"]["numer"], dtype=np.float64) / np.sqrt(c["wrong_order"]["denom_sqrt"])
+        ok &= bool(np.allclose(got, want, rtol=0, atol=1e-15))
+        ok &= not np.allclose(got, wrong, rtol=0, atol=1e-15)
+    return bool(ok)
+
+
+def test_rotation_sign_order_golden():
+    assert rotation_golden_holds(oracle.rotation_matrix)
+    # rotate() and the quantisers go through the same matrix
+    g = json.loads((GOLDEN / "rotation_sign_order.json").read_text())
+    for c in g["cases"]:
+        x = np.array(c["x"], dtype=np.float64)
+        signs = np.array(c["signs"], dtype=np.float64)
+        want = np.array(c["expected"]["numer"], dtype=np.float64) / np.sqrt(c["expected"]["denom_sqrt"])
+        np.testing.assert_allclose(oracle.rotate(x[None], signs)[0], want, rtol=0, atol=1e-15)
+        _, ds, scaled = oracle.quantize_per_tensor(x[None], True, signs, return_scaled=True)
+        np.testing.assert_allclose(scaled[0] * ds, want, rtol=0, atol=1e-14)
+
+
+def test_signs_flip_input_coordinates_before_mixing():
+    # Flipping coordinate c of x and the sign s_c together leaves x D unchanged,
+    # so x M is unchanged; the other order would not have this property.
+    d = 64
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(d)
+    s = inputs.hadamard_signs(d, seed=4).numpy().astype(np.float64)
+    for c in (0, 17, 63):
+        x2, s2 = x.copy(), s.copy()
+        x2[c], s2[c] = -x2[c], -s2[c]
+        np.testing.assert_allclose(oracle.rotate(x2[None], s2), oracle.rotate(x[None], s), rtol=0, atol=1e-13)
+
+
 def test_rotation_spreads_a_single_coordinate():
     # An outlier on one coordinate becomes +-|x|/sqrt(d) on every coordinate
     # (subsection 3, step 2: the transform spreads large values over all coordinates).

@@ -136,3 +136,39 @@ def test_each_planted_mistake_is_caught(tmp_path, name):
     old, new = MUTANTS[name]
     assert SRC.count(old) == 1, f"mutation anchor for {name} not found exactly once"
     assert not _pins_pass(_build(tmp_path, name, SRC.replace(old, new)))
+
+
+# ------------------------------------------------- rotation sign order --
+# M = D H_d / sqrt(d) (signs first, "FlashAttention-3 (PT)", "Inovações
+# técnicas do FlashAttention-3", subsection 3, step 1). The mistaken order
+# H_d D / sqrt(d) is orthogonal and keeps Q Kᵀ too, so orthogonality and
+# invariance pins cannot catch it; the hand-derived golden values must.
+ROTATION_MUTANTS = {
+    "signs_after_hadamard": ("return s[:, None] * h", "return h * s[None, :]"),
+    "signs_ignored": ("return s[:, None] * h", "return h"),
+    "unnormalised": ("h = sylvester_hadamard(d) / np.sqrt(d)", "h = sylvester_hadamard(d)"),
+}
+
+
+def _rotation_mutant(name):
+    import inspect
+
+    src = inspect.getsource(oracle.rotation_matrix)
+    old, new = ROTATION_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    ns = {"np": np, "sylvester_hadamard": oracle.sylvester_hadamard, "_as_f64": oracle._as_f64}
+    exec(src.replace(old, new), ns)
+    return ns["rotation_matrix"]
+
+
+def test_rotation_golden_accepts_the_oracle():
+    from test_codec import rotation_golden_holds
+
+    assert rotation_golden_holds(oracle.rotation_matrix)
+
+
+@pytest.mark.parametrize("name", sorted(ROTATION_MUTANTS))
+def test_each_planted_rotation_mistake_is_caught(name):
+    from test_codec import rotation_golden_holds
+
+    assert not rotation_golden_holds(_rotation_mutant(name))
