@@ -18,7 +18,7 @@ import torch
 _PKG = Path(__file__).resolve().parent
 _lock = threading.Lock()
 _lib = None
-_workspaces: dict[int, torch.Tensor] = {}
+_workspaces: dict[tuple[int, int], torch.Tensor] = {}
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
 FA_BF16, FA_E4M3, FA_E4M3_BLOCK = 0, 1, 2
@@ -96,29 +96,78 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _descale_arg(qk_descale, B, H, Nq, Nk):
+def _tensor_arg(t, name: str, device, dtypes=None, shape=None, min_bytes: int | None = None):
+    """Check one tensor argument before its pointer reaches the library: a CUDA
+    tensor on ``device``, of one of ``dtypes``, of exactly ``shape``, contiguous
+    (a pointer to a strided view would be read or written as if it were dense),
+    and holding at least ``min_bytes`` bytes. Raises FaError otherwise."""
+    if not isinstance(t, torch.Tensor):
+        raise FaError(f"{name} must be a torch tensor")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise FaError(f"{name} must have dtype {' or '.join(str(x) for x in dtypes)} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise FaError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise FaError(f"{name} must be contiguous")
+    if min_bytes is not None and _nbytes(t) < min_bytes:
+        raise FaError(f"{name} holds {_nbytes(t)} bytes, needs at least {min_bytes}")
+    if not t.is_cuda:
+        raise FaError(f"{name} must be on a CUDA device (got {t.device})")
+    if t.device != torch.device(device):
+        raise FaError(f"{name} is on {t.device}, the other tensors on {device}")
+    return t
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _descale_arg(qk_descale, B, H, Nq, Nk, device):
     """(fa_dtype, fp32 CUDA tensor) for e4m3 inputs: a 2-element tensor [dq, dk]
     is one scale per tensor; a pair (dq_blocks [B, H, ceil(Nq/128)], dk_blocks
     [B, H, ceil(Nk/128)]) is one scale per 128-row block."""
+    f32 = (torch.float32,)
     if isinstance(qk_descale, (tuple, list)):
+        if len(qk_descale) != 2:
+            raise FaError("per-block descales must be a pair (dq_blocks, dk_blocks)")
         dq, dk = qk_descale
         nbq, nbk = -(-Nq // BLOCK_ROWS), -(-Nk // BLOCK_ROWS)
-        if dq.numel() != B * H * nbq or dk.numel() != B * H * nbk:
-            raise FaError(f"per-block descales must hold B*H*ceil(N/128) values ({B * H * nbq}, {B * H * nbk})")
-        if dq.dtype != torch.float32 or dk.dtype != torch.float32 or not (dq.is_cuda and dk.is_cuda):
-            raise FaError("per-block descales must be CUDA fp32 tensors")
+        for t, name, nb in ((dq, "dq_blocks", nbq), (dk, "dk_blocks", nbk)):
+            if not isinstance(t, torch.Tensor) or t.numel() != B * H * nb:
+                raise FaError(f"per-block descales must hold B*H*ceil(N/128) values ({B * H * nbq}, {B * H * nbk})")
+            _tensor_arg(t, name, device, f32)
         return FA_E4M3_BLOCK, torch.cat([dq.reshape(-1), dk.reshape(-1)])
-    if qk_descale is None or qk_descale.dtype != torch.float32 or qk_descale.numel() < 2:
+    if qk_descale is None:
         raise FaError("e4m3 q/k need qk_descale = CUDA fp32 tensor [dq, dk] or a pair of per-block tensors")
-    return FA_E4M3, qk_descale.contiguous()
+    _tensor_arg(qk_descale, "qk_descale", device, f32)
+    if qk_descale.numel() != 2:
+        raise FaError("qk_descale must hold exactly two values [dq, dk]")
+    return FA_E4M3, qk_descale
 
 
 def _require_cuda(*ts):
-    for t in ts:
-        if t is not None and not t.is_cuda:
-            raise FaError("tensors must be on a CUDA device")
+    """The input tensors are CUDA tensors on one device (a CUDA device must exist)."""
     if not torch.cuda.is_available():
         raise FaError("no CUDA device")
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise FaError("tensors must be on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise FaError(f"tensors must be on one device (got {dev} and {t.device})")
+
+
+def _signs_arg(signs, d: int, device):
+    """The d Hadamard signs as a contiguous fp32 tensor on ``device``."""
+    if signs is None:
+        return None
+    if not isinstance(signs, torch.Tensor) or signs.numel() != d:
+        raise FaError(f"signs must be a tensor of d = {d} values")
+    return signs.to(device=device, dtype=torch.float32).reshape(d).contiguous()
 
 
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=None, out=None, lse=None,
@@ -153,11 +202,14 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
-    if return_lse and lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _tensor_arg(out, "out", q.device, (torch.bfloat16,), (B, H, N, d))
+    if return_lse:
+        if lse is None:
+            lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        _tensor_arg(lse, "lse", q.device, (torch.float32,), (B, H, N))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    dt, desc_t = _descale_arg(qk_descale, B, H, N, N) if fp8 else (FA_BF16, None)
+    dt, desc_t = _descale_arg(qk_descale, B, H, N, N, q.device) if fp8 else (FA_BF16, None)
     desc = _ptr(desc_t)
     with torch.cuda.device(q.device):
         if n_split == 1:
@@ -174,20 +226,28 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
     return out, (lse if return_lse else None)
 
 
-_split_workspaces: dict[int, torch.Tensor] = {}
+_split_workspaces: dict[tuple[int, int], torch.Tensor] = {}
+
+
+def _stream_key(device) -> tuple[int, int]:
+    dev = torch.device(device)
+    return dev.index, torch.cuda.current_stream(dev).cuda_stream
 
 
 def _split_workspace(device, nbytes: int):
     """A device buffer of at least ``nbytes`` for the split schedules, cached per
-    device and grown when a call needs more (calls on one device share it, so
-    they must be ordered on one stream)."""
+    (device, current stream) and grown when a call needs more. Calls on one
+    stream run in order, so they can share it; calls on different streams get
+    different buffers. A buffer is allocated while its stream is current, so
+    the caching allocator reuses its memory only in that stream's order when it
+    is replaced."""
     if nbytes <= 0:
         return None
-    idx = torch.device(device).index
-    ws = _split_workspaces.get(idx)
+    key = _stream_key(device)
+    ws = _split_workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
-        _split_workspaces[idx] = ws
+        _split_workspaces[key] = ws
     return ws
 
 
@@ -226,18 +286,23 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, qk_de
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
     if out is None:
         out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
-    if return_lse and lse is None:
-        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _tensor_arg(out, "out", q.device, (torch.bfloat16,), (B, H, Nq, d))
+    if return_lse:
+        if lse is None:
+            lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+        _tensor_arg(lse, "lse", q.device, (torch.float32,), (B, H, Nq))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(q.device):
         if n_split == 0:
             n_split = int(lib.fa_fwd_splitkv_splits(B, H, Nq, Nk, d))
         need = int(lib.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, int(n_split)))
-        if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk) if fp8 else (FA_BF16, None)
+        if need > 0:
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            _tensor_arg(workspace, "workspace", q.device, min_bytes=need)
+        ws_bytes = _nbytes(workspace) if workspace is not None else 0
+        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk, q.device) if fp8 else (FA_BF16, None)
         rc = lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, Nq,
                                 Nk, d, int(bool(causal)), float(scale), dt, _ptr(desc_t), int(n_split),
                                 _ptr(workspace) if need > 0 else None, ws_bytes, _stream(q.device))
@@ -255,14 +320,18 @@ def fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, qk_de
     lib = load_library()
     B, H, Nq, Nk, d, fp8 = _qkv_kinds(q, k, v, qk_descale)
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if int(n_split) < 1:
+        raise FaError("n_split must be at least 1")
     if o_part is None:
         o_part = torch.empty((n_split, B, H, Nq, d), dtype=torch.float32, device=q.device)
     if lse_part is None:
         lse_part = torch.empty((n_split, B, H, Nq), dtype=torch.float32, device=q.device)
+    _tensor_arg(o_part, "o_part", q.device, (torch.float32,), (n_split, B, H, Nq, d))
+    _tensor_arg(lse_part, "lse_part", q.device, (torch.float32,), (n_split, B, H, Nq))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(q.device):
-        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk) if fp8 else (FA_BF16, None)
+        dt, desc_t = _descale_arg(qk_descale, B, H, Nq, Nk, q.device) if fp8 else (FA_BF16, None)
         rc = lib.fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, H, Nq, Nk, d,
                                 int(bool(causal)), float(scale), dt, _ptr(desc_t), int(n_split), _stream(q.device))
     _check(rc, "fa_fwd_partial")
@@ -284,8 +353,11 @@ def lse_merge(o_part, lse_part, out=None, lse=None, return_lse: bool = True):
     o_part, lse_part = o_part.contiguous(), lse_part.contiguous()
     if out is None:
         out = torch.empty(tuple(o_part.shape[1:]), dtype=torch.bfloat16, device=o_part.device)
-    if return_lse and lse is None:
-        lse = torch.empty(tuple(lse_part.shape[1:]), dtype=torch.float32, device=o_part.device)
+    _tensor_arg(out, "out", o_part.device, (torch.bfloat16,), tuple(o_part.shape[1:]))
+    if return_lse:
+        if lse is None:
+            lse = torch.empty(tuple(lse_part.shape[1:]), dtype=torch.float32, device=o_part.device)
+        _tensor_arg(lse, "lse", o_part.device, (torch.float32,), tuple(lse_part.shape[1:]))
     with torch.cuda.device(o_part.device):
         rc = lib.fa_lse_merge(_ptr(o_part), _ptr(lse_part), n_part, rows, d, _ptr(out),
                               _ptr(lse) if return_lse else None, _stream(o_part.device))
@@ -308,9 +380,10 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
         raise FaError("lse must be fp32 [B, H, N]")
     scale = d ** -0.5 if scale is None else scale
     q, k, v, o, dout, lse = (t.contiguous() for t in (q, k, v, o, dout, lse))
-    need = lib.fa_bwd_workspace_bytes(B, H, N, d)
+    need = int(lib.fa_bwd_workspace_bytes(B, H, N, d))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _tensor_arg(workspace, "workspace", q.device, min_bytes=need)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     with torch.cuda.device(q.device):
         rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -326,11 +399,14 @@ def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def _workspace(device) -> torch.Tensor:
-    idx = torch.device(device).index
-    ws = _workspaces.get(idx)
+    """The quantisers' 256-byte workspace (amax words and grid-barrier counter),
+    cached per (device, current stream): each call zeroes it on its stream, so
+    calls on one stream may share it and calls on two streams must not."""
+    key = _stream_key(device)
+    ws = _workspaces.get(key)
     if ws is None:
         ws = torch.empty(QUANT_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
-        _workspaces[idx] = ws
+        _workspaces[key] = ws
     return ws
 
 
@@ -351,8 +427,10 @@ def hadamard_quant(x, rotate: bool = True, signs=None, out=None, descale=None, w
         descale = torch.empty(1, dtype=torch.float32, device=x.device)
     if workspace is None:
         workspace = _workspace(x.device)
-    if signs is not None:
-        signs = signs.to(device=x.device, dtype=torch.float32).contiguous()
+    _tensor_arg(out, "out", x.device, E4M3_DTYPES, tuple(x.shape))
+    _tensor_arg(descale, "descale", x.device, (torch.float32,), min_bytes=4)
+    _tensor_arg(workspace, "workspace", x.device, min_bytes=QUANT_WORKSPACE_BYTES)
+    signs = _signs_arg(signs, d, x.device)
     with torch.cuda.device(x.device):
         rc = lib.fa_hadamard_quant(_ptr(x), _ptr(out), _ptr(descale), rows, d, int(bool(rotate)),
                                    _ptr(signs) if (rotate and signs is not None) else None, _ptr(workspace),
@@ -374,14 +452,20 @@ def hadamard_quant_multi(xs, rotate: bool = True, signs=None, outs=None, descale
         raise FaError("xs must be bf16 tensors of one shape")
     d = xs[0].shape[-1]
     rows = xs[0].numel() // d if d else 0
+    dev = xs[0].device
     if outs is None:
-        outs = [torch.empty(x.shape, dtype=torch.uint8, device=x.device) for x in xs]
+        outs = [torch.empty(x.shape, dtype=torch.uint8, device=dev) for x in xs]
     if descales is None:
-        descales = torch.empty(len(xs), dtype=torch.float32, device=xs[0].device)
+        descales = torch.empty(len(xs), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = _workspace(xs[0].device)
-    if signs is not None:
-        signs = signs.to(device=xs[0].device, dtype=torch.float32).contiguous()
+        workspace = _workspace(dev)
+    if len(outs) != len(xs):
+        raise FaError("outs must hold one tensor per input")
+    for i, o in enumerate(outs):
+        _tensor_arg(o, f"outs[{i}]", dev, E4M3_DTYPES, tuple(xs[0].shape))
+    _tensor_arg(descales, "descales", dev, (torch.float32,), min_bytes=4 * len(xs))
+    _tensor_arg(workspace, "workspace", dev, min_bytes=QUANT_WORKSPACE_BYTES)
+    signs = _signs_arg(signs, d, dev)
     n = len(xs)
     x_arr = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
     o_arr = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
@@ -409,8 +493,9 @@ def hadamard_quant_blocks(x, rotate: bool = True, signs=None, out=None, descales
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if descales is None:
         descales = torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
-    if signs is not None:
-        signs = signs.to(device=x.device, dtype=torch.float32).contiguous()
+    _tensor_arg(out, "out", x.device, E4M3_DTYPES, tuple(x.shape))
+    _tensor_arg(descales, "descales", x.device, (torch.float32,), (B, H, nb))
+    signs = _signs_arg(signs, d, x.device)
     with torch.cuda.device(x.device):
         rc = lib.fa_hadamard_quant_blocks(_ptr(x), _ptr(out), _ptr(descales), B * H, N, d, int(bool(rotate)),
                                           _ptr(signs) if (rotate and signs is not None) else None,

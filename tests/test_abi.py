@@ -217,3 +217,33 @@ def test_bwd_binding_rejects_host_tensors_and_bad_shapes():
     lse = torch.zeros(1, 1, 8)
     with pytest.raises(binding.FaError):
         binding.bwd(q, q, q, q, lse, q)  # host tensors: no CPU path
+
+
+def test_tensor_argument_checks_run_before_any_launch():
+    """Every caller-supplied tensor (outputs, workspaces, descales, signs) is
+    checked before its pointer reaches the library: dtype, exact shape,
+    contiguity, size, and that it is a CUDA tensor on the inputs' device."""
+    import torch
+
+    dev = torch.device("cuda:0")
+    ok = torch.zeros(2, 3, dtype=torch.float32)
+    with pytest.raises(binding.FaError, match="CUDA"):           # a host tensor
+        binding._tensor_arg(ok, "out", dev, (torch.float32,), (2, 3))
+    with pytest.raises(binding.FaError, match="dtype"):
+        binding._tensor_arg(ok.double(), "out", dev, (torch.float32,), (2, 3))
+    with pytest.raises(binding.FaError, match="shape"):          # a short output
+        binding._tensor_arg(torch.zeros(2, 2), "out", dev, (torch.float32,), (2, 3))
+    with pytest.raises(binding.FaError, match="contiguous"):     # a strided view
+        binding._tensor_arg(torch.zeros(3, 2).t(), "out", dev, (torch.float32,), (2, 3))
+    with pytest.raises(binding.FaError, match="bytes"):          # a short workspace
+        binding._tensor_arg(torch.zeros(255, dtype=torch.uint8), "workspace", dev, min_bytes=256)
+    with pytest.raises(binding.FaError, match="torch tensor"):
+        binding._tensor_arg([0.0], "descale", dev)
+    with pytest.raises(binding.FaError, match="signs"):
+        binding._signs_arg(torch.ones(64), 128, dev)
+    with pytest.raises(binding.FaError, match="pair"):
+        binding._descale_arg((ok,), 1, 1, 128, 128, dev)
+    with pytest.raises(binding.FaError):
+        binding._descale_arg(ok.reshape(-1)[:2], 1, 1, 128, 128, dev)   # host descale
+    with pytest.raises(binding.FaError):
+        binding._descale_arg(None, 1, 1, 128, 128, dev)
