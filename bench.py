@@ -1,28 +1,29 @@
 """Benchmark of the fused attention forward on B200.
 
-One step = one pass of the whole hot path over one batch of synthetic input of
-the B=4, H=16, N=2048, d=128 workload (Q, K, V ~ N(0,1) bf16, scale 1/sqrt(128)):
-  1. BF16 forward, non-causal;   2. BF16 forward, causal;
-  3. Hadamard rotate + e4m3 quantise of Q and K (one launch, a scale each);   4. e4m3-QK forward, non-causal.
-Metric: attention TFLOPS = sum of 4*B*H*N^2*d (halved when causal) over the
-three forward passes / step time. L2 (126 MB) is flushed between steps by
-writing a 512 MB buffer outside the timed events, since the inputs (100 MB)
-would otherwise stay resident.
+Headline (default, ``--workload fwd``): the BF16 forward, non-causal, on the
+largest single-GPU configuration of the sequence sweep, B=1, H=16, N=16384,
+d=128 (Q, K, V ~ N(0,1) bf16, scale 1/sqrt(128)). One step is one ``fa_fwd``
+launch. Metric: TFLOPS = 4*B*H*N^2*d / step time, and its fraction of the bf16
+tensor peak. The inputs (201 MB) are larger than L2 (126 MB), and L2 is also
+flushed between steps by a 512 MB write outside the timed events.
+
+The same JSON line carries the other workloads as named sub-objects, each timed
+as CUDA-graph replays of its own calls with L2 flushed between replays:
+  * ``b4h16n2048d128``: BF16 forward, non-causal and causal;
+  * ``seq_sweep_h16d128``: BF16 forward for N in 512..16384 with B*N = 16384;
+  * ``dsweep_b2n4096_causal``: BF16 causal forward for d in 64, 128, 256;
+  * ``fp8_b2h16n8192d128``: Hadamard rotate + e4m3 quantise of Q and K (one
+    launch; per tensor and per 128-row block) and the e4m3 attention;
+  * ``bwd_b4h16n2048d128``: the backward pass, non-causal and causal;
+  * ``decode_b4h16nq1nk32768d128``: one query per head over 32768 keys.
+``--no-extras`` skips them.
+
+``--workload bwd`` and ``--workload decode`` print a line of their own for the
+backward pass (10*B*H*N^2*d FLOPs, halved when causal, on B=4, H=16, N=2048,
+d=128) and for the decode problem (GB/s of algorithmic HBM bytes).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only), on a bounded
 row sample of the same workload per step.
-
-``--workload decode`` measures the decode-shaped problem instead: B=4, H=16
-single-query heads (Nq=1) over Nk=32768 keys, d=128, bf16: one step is the
-split-key attention kernel (fp32 partial results per block of keys) and the LSE
-merge. It is HBM-bound (the 1.07 GB of K and V are read once per step), so its
-metric is GB/s of algorithmic traffic.
-
-``--workload bwd`` measures the backward pass on the B=4, H=16, N=2048, d=128
-workload: one step is fa_bwd non-causal then fa_bwd causal (each a prologue, the
-tcgen05 kernel and the dQ conversion), given O and LSE from the library's
-forward (computed once, outside the timed region). Metric: backward TFLOPS =
-10*B*H*N^2*d (the five N x N x d products; halved when causal) / step time.
 
 Launch: ``python bench.py --gpus N --steps K --warmup W`` (N > 1 under
 torch.distributed.run, one rank per GPU, each rank its own batch: weak scaling,
@@ -49,21 +50,29 @@ import torch  # noqa: E402
 from io_aware_exact_17_b200 import inputs as fa_inputs  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (4·B·H·N²·d, ½ if causal) and % of B200 BF16/FP8 peak"
-DECODE = {"B": 4, "H": 16, "Nq": 1, "Nk": 32768, "d": 128, "seed": 1005}
 DECODE_METRIC = "decode attention GB/s (algorithmic HBM bytes: K, V, Q read; O, LSE written)"
 BWD_METRIC = "attention bwd TFLOPS (10·B·H·N²·d, ½ if causal) and % of B200 BF16 peak"
-B, H, N, D = 4, 16, 2048, 128
-SEED = 1001
-WORKLOAD = f"b{B}h{H}n{N}d{D}: bf16 fwd non-causal + bf16 fwd causal + rotate/quantise Q,K + e4m3-QK fwd non-causal"
+
+# The headline: the sequence sweep's largest configuration (B*N = 16384, seed 1002).
+HEADLINE = {"B": 1, "H": 16, "N": 16384, "d": 128, "causal": False, "seed": 1002}
+CFG1 = {"B": 4, "H": 16, "N": 2048, "d": 128, "seed": 1001}
+SWEEP_SEED, SWEEP_TOKENS = 1002, 16384
+FP8_CFG = {"B": 2, "H": 16, "N": 8192, "d": 128, "seed": 1003}
+DSWEEP = {"B": 2, "N": 4096, "seed": 1004}
+DECODE = {"B": 4, "H": 16, "Nq": 1, "Nk": 32768, "d": 128, "seed": 1005}
+B, H, N, D = CFG1["B"], CFG1["H"], CFG1["N"], CFG1["d"]  # the backward workload
+SEED = CFG1["seed"]
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0  # nominal dense e4m3 : bf16 tensor rate (4.5 : 2.25 PFLOP/s)
+FLUSH_BYTES = 512 * 1024 * 1024
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# bf16 non-causal attention kernel on this workload, from one ncu capture, and
-# the SHA-256 of the kernel's sources at that capture. When the sources differ
-# the figure no longer describes the kernel and `traffic` is reported as null.
+# headline kernel, from one ncu capture, and the SHA-256 of the kernel's sources
+# at that capture. When the sources differ the figure no longer describes the
+# kernel and `traffic` is reported as null.
 KERNEL_SOURCES = ("io_aware_exact_17_b200/csrc/attn_fwd.cuh", "io_aware_exact_17_b200/csrc/sm100.cuh")
-NCU_TRAFFIC_BYTES = 109134336  # 100.744192 MB read + 8.390144 MB written
-NCU_TRAFFIC_SHA256 = "1cd88edb5ead5007262af6e353d6d14f4f7c22db05befff7ab8ab3ffc1717029"
+NCU_TRAFFIC_BYTES = None
+NCU_TRAFFIC_SHA256 = None
 
 
 def kernel_sources_sha256() -> str:
@@ -81,12 +90,9 @@ def measured_traffic():
     return NCU_TRAFFIC_BYTES
 
 
-def flops_fwd(causal: bool) -> float:
-    f = 4.0 * B * H * N * N * D
+def attn_flops(b: int, h: int, n: int, d: int, causal: bool) -> float:
+    f = 4.0 * b * h * n * n * d
     return f / 2 if causal else f
-
-
-STEP_FLOPS = flops_fwd(False) + flops_fwd(True) + flops_fwd(False)
 
 
 def load_peaks():
@@ -244,18 +250,19 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- GPU step --
-class Step:
-    """All buffers of one step, allocated once; run() enqueues the step's kernels
-    on the current stream, bracketing each kernel group with CUDA events."""
+class FwdStep:
+    """One BF16 forward problem, all buffers allocated once; run() enqueues the
+    step's one kernel (fa_fwd through the public ``fwd``) on the current stream,
+    bracketed by CUDA events when given."""
 
-    def __init__(self, seed: int):
+    def __init__(self, b: int, h: int, n: int, d: int, causal: bool, seed: int):
         import io_aware_exact_17_b200 as fa
 
         self.fa = fa
-        q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
-        self.signs = fa_inputs.hadamard_signs(D, seed).cuda()
+        self.shape = (b, h, n, d)
+        self.causal = causal
+        q, k, v = fa_inputs.qkv_normal(b, h, n, d, seed)
         self.q_h, self.k_h, self.v_h = (t.pin_memory() for t in (q, k, v))
-        shp = (B, H, N, D)
         # two sets of device inputs and outputs, so that pipelined end-to-end steps
         # can copy one set while computing on the other (the timed device-only
         # steps use set 0)
@@ -263,55 +270,40 @@ class Step:
         for _ in range(2):
             self.bufs.append({
                 "q": q.cuda(), "k": k.cuda(), "v": v.cuda(),
-                "o": [torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(3)],
-                "lse": [torch.empty((B, H, N), dtype=torch.float32, device="cuda") for _ in range(3)],
+                "o": torch.empty(self.shape, dtype=torch.bfloat16, device="cuda"),
+                "lse": torch.empty((b, h, n), dtype=torch.float32, device="cuda"),
             })
-        self.q, self.k, self.v = self.bufs[0]["q"], self.bufs[0]["k"], self.bufs[0]["v"]
-        self.o, self.lse = self.bufs[0]["o"], self.bufs[0]["lse"]
-        self.q8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
-        self.k8 = torch.empty(shp, dtype=torch.uint8, device="cuda")
-        self.desc = torch.empty(2, dtype=torch.float32, device="cuda")
-        self.o_h = [torch.empty(shp, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-        self.lse_h = [torch.empty((B, H, N), dtype=torch.float32).pin_memory() for _ in range(3)]
-        self.flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-        self.launches_per_step = 4  # 3 attention kernels + 1 quantisation of Q and K
-        self.groups = 4  # breakdown: bf16 nc, bf16 causal, quantise Q+K, e4m3 nc
+        self.o_h = torch.empty(self.shape, dtype=torch.bfloat16).pin_memory()
+        self.lse_h = torch.empty((b, h, n), dtype=torch.float32).pin_memory()
+        self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 1
+        self.groups = 1
+        self.flops = attn_flops(b, h, n, d, causal)
 
     def flush_l2(self):
         self.flush_buf.zero_()
 
     def run(self, ev=None, b=0):
-        fa = self.fa
-        q, k, v, o, lse = (self.bufs[b][n] for n in ("q", "k", "v", "o", "lse"))
+        s = self.bufs[b]
         if ev is not None:
             ev[0].record()
-        fa.fwd(q, k, v, causal=False, out=o[0], lse=lse[0])
+        self.fa.fwd(s["q"], s["k"], s["v"], causal=self.causal, out=s["o"], lse=s["lse"], n_split=1)
         if ev is not None:
             ev[1].record()
-        fa.fwd(q, k, v, causal=True, out=o[1], lse=lse[1])
-        if ev is not None:
-            ev[2].record()
-        fa.hadamard_quant_multi([q, k], rotate=True, signs=self.signs, outs=[self.q8, self.k8], descales=self.desc)
-        if ev is not None:
-            ev[3].record()
-        fa.fwd(self.q8, self.k8, v, causal=False, qk_descale=self.desc, out=o[2], lse=lse[2])
-        if ev is not None:
-            ev[4].record()
 
-    # End to end, through the same public calls with host buffers: pinned
-    # host -> device copies of Q, K, V, the step, device -> host copies of every
-    # O and LSE, each part on the current stream, for buffer set b.
+    # End to end, through the same public call with host buffers: pinned
+    # host -> device copies of Q, K, V, the step, device -> host copies of O and
+    # LSE, each part on the current stream, for buffer set b.
     def h2d(self, b):
-        for n, h in (("q", self.q_h), ("k", self.k_h), ("v", self.v_h)):
-            self.bufs[b][n].copy_(h, non_blocking=True)
+        for n_, h_ in (("q", self.q_h), ("k", self.k_h), ("v", self.v_h)):
+            self.bufs[b][n_].copy_(h_, non_blocking=True)
 
     def compute(self, b):
         self.run(b=b)
 
     def d2h(self, b):
-        for i in range(3):
-            self.o_h[i].copy_(self.bufs[b]["o"][i], non_blocking=True)
-            self.lse_h[i].copy_(self.bufs[b]["lse"][i], non_blocking=True)
+        self.o_h.copy_(self.bufs[b]["o"], non_blocking=True)
+        self.lse_h.copy_(self.bufs[b]["lse"], non_blocking=True)
 
     @property
     def h2d_bytes(self):
@@ -319,7 +311,7 @@ class Step:
 
     @property
     def d2h_bytes(self):
-        return sum(t.numel() * t.element_size() for t in self.o_h + self.lse_h)
+        return self.o_h.numel() * 2 + self.lse_h.numel() * 4
 
 
 class DecodeStep:
@@ -465,7 +457,7 @@ def flops_bwd(causal: bool) -> float:
 
 def capture_step(step):
     """The step's kernels captured once as a CUDA graph, so a timed step carries
-    no host launch overhead (the quantiser kernels are ~10 us each)."""
+    no host launch overhead."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
@@ -504,6 +496,42 @@ def time_steps(step, graph, steps: int, warmup: int, world: int):
     torch.cuda.synchronize()
     per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(step.groups)] for i in range(steps)]
     return step_ms, per  # per: ms of each kernel group per eager step
+
+
+class _Flush:
+    def __init__(self):
+        self.buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def time_call(fn, reps: int, flush, warmup: int = 3) -> float:
+    """Mean ms of ``fn``'s launches: the calls captured once as a CUDA graph and
+    replayed ``reps`` times, L2 flushed between replays outside the events,
+    which are recorded on the stream the graph is replayed on."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        fn()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        flush()
+        g.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in ev:
+        flush()
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    del g
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
 
 def time_e2e(step, steps: int, warmup: int, world: int):
@@ -557,35 +585,182 @@ def time_e2e(step, steps: int, warmup: int, world: int):
     return e0.elapsed_time(e1) / steps
 
 
+# ------------------------------------------------- the other workloads --
+def _frac(x, peak):
+    return None if x is None else x / peak
+
+
+def _attn_entry(ms: float, flops: float, peak_tflops: float) -> dict:
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"ms": ms, "tflops": tf, "frac": tf / peak_tflops}
+
+
+def extras(peaks: dict, reps: int) -> dict:
+    """The other workloads of the path, each as a sub-object of the JSON line.
+    Every figure is the mean of ``reps`` CUDA-graph replays of its calls, L2
+    flushed between replays. Buffers are freed between workloads."""
+    import io_aware_exact_17_b200 as fa
+
+    flush = _Flush()
+    bf16 = peaks["bf16_tflops"]
+    out = {}
+
+    def guarded(name, fn):
+        try:
+            out[name] = fn()
+        except Exception as e:  # report, keep the headline line
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    def fwd_pair(shape, seed, masks=(False, True), views=None):
+        q, k, v = views if views is not None else (t.cuda() for t in fa_inputs.qkv_normal(*shape, seed))
+        o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(shape[:3], dtype=torch.float32, device="cuda")
+        res = {}
+        for causal in masks:
+            ms = time_call(lambda: fa.fwd(q, k, v, causal=causal, out=o, lse=lse, n_split=1), reps, flush)
+            res["causal" if causal else "noncausal"] = _attn_entry(ms, attn_flops(*shape, causal), bf16)
+        return res
+
+    c = CFG1
+    guarded(f"b{c['B']}h{c['H']}n{c['N']}d{c['d']}", lambda: fwd_pair((c["B"], c["H"], c["N"], c["d"]), c["seed"]))
+
+    def sweep():
+        flat = [t.cuda() for t in fa_inputs.qkv_normal(1, 16, SWEEP_TOKENS, 128, SWEEP_SEED)]
+        res = {}
+        for n in (512, 1024, 2048, 4096, 8192, 16384):
+            shape = (SWEEP_TOKENS // n, 16, n, 128)
+            r = fwd_pair(shape, SWEEP_SEED, views=[t.view(shape) for t in flat])
+            res[f"N={n}"] = {"B": shape[0], "noncausal_tflops": r["noncausal"]["tflops"],
+                             "causal_tflops": r["causal"]["tflops"], "noncausal_frac": r["noncausal"]["frac"]}
+        return res
+
+    guarded("seq_sweep_h16d128", sweep)
+
+    def dsweep():
+        res = {}
+        for d in (64, 128, 256):
+            shape = (DSWEEP["B"], 2048 // d, DSWEEP["N"], d)
+            r = fwd_pair(shape, DSWEEP["seed"], masks=(True,))
+            res[f"d={d}"] = {"H": shape[1], "causal_tflops": r["causal"]["tflops"], "causal_frac": r["causal"]["frac"]}
+        return res
+
+    guarded(f"dsweep_b{DSWEEP['B']}n{DSWEEP['N']}_causal", dsweep)
+
+    def fp8():
+        f = FP8_CFG
+        shape = (f["B"], f["H"], f["N"], f["d"])
+        q, k, v = (t.cuda() for t in fa_inputs.qkv_normal(*shape, f["seed"]))
+        signs = fa_inputs.hadamard_signs(f["d"], f["seed"]).cuda()
+        q8, k8 = (torch.empty(shape, dtype=torch.uint8, device="cuda") for _ in range(2))
+        desc = torch.empty(2, dtype=torch.float32, device="cuda")
+        nb = -(-f["N"] // 128)
+        dqb, dkb = (torch.empty((f["B"], f["H"], nb), dtype=torch.float32, device="cuda") for _ in range(2))
+        o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(shape[:3], dtype=torch.float32, device="cuda")
+        fl = attn_flops(*shape, False)
+        hbm = peaks["hbm_gbs"]
+        qbytes = 2 * q.numel() * 3  # Q and K: read bf16, write e4m3
+        res = {"peaks": {"fp8_tflops": FP8_OVER_BF16 * bf16, "mixed_e4m3qk_bf16pv_tflops": bf16 / 0.75,
+                         "source": "derived: measured bf16 burst x nominal e4m3:bf16 ratio 2; the e4m3-QK kernel "
+                                   "runs half its FLOPs (Q.K^T) at the e4m3 rate and half (P.V) at the bf16 rate"}}
+        ms = time_call(lambda: fa.hadamard_quant_multi([q, k], rotate=True, signs=signs, outs=[q8, k8],
+                                                       descales=desc), reps, flush)
+        res["rotate_quant_qk_per_tensor"] = {"ms": ms, "gbs": qbytes / (ms * 1e-3) / 1e9,
+                                             "frac": qbytes / (ms * 1e-3) / 1e9 / hbm,
+                                             "bytes": qbytes, "bound": "hbm"}
+        ms_a = time_call(lambda: fa.fwd(q8, k8, v, causal=False, qk_descale=desc, out=o, lse=lse, n_split=1),
+                         reps, flush)
+        tf = fl / (ms_a * 1e-3) / 1e12
+        res["attn_e4m3qk_per_tensor"] = {"ms": ms_a, "tflops": tf, "frac_fp8_peak": tf / (FP8_OVER_BF16 * bf16),
+                                         "frac_mixed_peak": tf * 0.75 / bf16}
+
+        def blocks():
+            fa.hadamard_quant_blocks(q, rotate=True, signs=signs, out=q8, descales=dqb)
+            fa.hadamard_quant_blocks(k, rotate=True, signs=signs, out=k8, descales=dkb)
+
+        ms = time_call(blocks, reps, flush)
+        res["rotate_quant_qk_per_block"] = {"ms": ms, "gbs": qbytes / (ms * 1e-3) / 1e9,
+                                            "frac": qbytes / (ms * 1e-3) / 1e9 / hbm, "bytes": qbytes,
+                                            "bound": "hbm"}
+        ms_b = time_call(lambda: fa.fwd(q8, k8, v, causal=False, qk_descale=(dqb, dkb), out=o, lse=lse,
+                                        n_split=1), reps, flush)
+        tf = fl / (ms_b * 1e-3) / 1e12
+        res["attn_e4m3qk_per_block"] = {"ms": ms_b, "tflops": tf, "frac_fp8_peak": tf / (FP8_OVER_BF16 * bf16),
+                                        "frac_mixed_peak": tf * 0.75 / bf16}
+        step_ms = res["rotate_quant_qk_per_tensor"]["ms"] + ms_a
+        res["step_quant_plus_attn"] = {"ms": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12}
+        return res
+
+    guarded(f"fp8_b{FP8_CFG['B']}h{FP8_CFG['H']}n{FP8_CFG['N']}d{FP8_CFG['d']}", fp8)
+
+    def bwd():
+        step = BwdStep(SEED)
+        res = {}
+        for causal in (False, True):
+            ms = time_call(lambda: step._bwd(0, causal), reps, flush)
+            tf = flops_bwd(causal) / (ms * 1e-3) / 1e12
+            res["causal" if causal else "noncausal"] = {"ms": ms, "tflops": tf, "frac": tf / bf16}
+        del step
+        return res
+
+    guarded(f"bwd_b{B}h{H}n{N}d{D}", bwd)
+
+    def decode():
+        step = DecodeStep(DECODE["seed"])
+        ms = time_call(lambda: step.run(), reps, flush)
+        ms_attn = time_call(lambda: step.fa.fwd_partial(step.q, step.k, step.v, n_split=step.n_split,
+                                                        o_part=step.o_part, lse_part=step.lse_part), reps, flush)
+        attn_bytes = step.kv_bytes + step.q_h.numel() * 2 + step.part_bytes
+        res = {"n_split": step.n_split, "step_ms": ms, "step_gbs": step.bytes / (ms * 1e-3) / 1e9,
+               "attn_ms": ms_attn, "attn_gbs": attn_bytes / (ms_attn * 1e-3) / 1e9,
+               "attn_frac": attn_bytes / (ms_attn * 1e-3) / 1e9 / peaks["hbm_gbs"], "bound": "hbm"}
+        del step
+        return res
+
+    c = DECODE
+    guarded(f"decode_b{c['B']}h{c['H']}nq{c['Nq']}nk{c['Nk']}d{c['d']}", decode)
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------ CPU oracle --
-def oracle_sample(target_s: float, seed: int):
-    """Time the oracle (as it stands) on a row sample of the three attention
-    passes of the step, sized for about ``target_s`` seconds. Returns
-    (flops, seconds, threads, rows_per_pass)."""
-    import numpy as np
+class OracleSampler:
+    """The oracle (as it stands) timed on random query rows of one forward
+    workload: the inputs are drawn once by the same recipe as the GPU's and
+    widened to fp64; each call times one row sample."""
 
-    import oracle
+    def __init__(self, cfg: dict):
+        import oracle
 
-    q, k, v = fa_inputs.qkv_normal(B, H, N, D, seed)
-    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
-    threads = oracle.default_threads()
-    rng = np.random.default_rng(seed)
+        self.oracle = oracle
+        self.cfg = cfg
+        b, h, n, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+        q, k, v = fa_inputs.qkv_normal(b, h, n, d, cfg["seed"])
+        self.q, self.k, self.v = (t.double().numpy() for t in (q, k, v))
+        self.threads = oracle.default_threads()
 
-    def run(rows_n):
-        rows = rng.integers(0, B * H * N, rows_n)
-        fl = 0.0
+    def run(self, rows_n: int, rng):
+        import numpy as np
+
+        c = self.cfg
+        rows = rng.integers(0, c["B"] * c["H"] * c["N"], rows_n)
         t0 = time.perf_counter()
-        for causal in (False, True, False):
-            oracle.attention(qd, kd, vd, causal, D ** -0.5, rows=rows, threads=threads)
-            i = rows % N
-            fl += float(np.sum(4.0 * D * (i + 1))) if causal else 4.0 * N * D * rows_n
-        return fl, time.perf_counter() - t0
+        self.oracle.attention(self.q, self.k, self.v, c["causal"], c["d"] ** -0.5, rows=rows, threads=self.threads)
+        dt = time.perf_counter() - t0
+        if c["causal"]:
+            fl = float(np.sum(4.0 * c["d"] * (rows % c["N"] + 1)))
+        else:
+            fl = 4.0 * c["N"] * c["d"] * rows_n
+        return fl, dt
 
-    probe_rows = max(threads * 4, 64)
-    fl, dt = run(probe_rows)
-    rows_n = int(min(B * H * N, max(probe_rows, probe_rows * target_s / max(dt, 1e-3))))
-    fl, dt = run(rows_n)
-    return fl, dt, threads, rows_n
+    def rows_for(self, seconds: float, rng) -> int:
+        probe = max(self.threads * 4, 64)
+        _, dt = self.run(probe, rng)
+        total = self.cfg["B"] * self.cfg["H"] * self.cfg["N"]
+        return int(min(total, max(probe, probe * seconds / max(dt, 1e-3))))
 
 
 def oracle_bwd_sample(target_s: float, seed: int):
@@ -608,30 +783,162 @@ def oracle_bwd_sample(target_s: float, seed: int):
     return fl, time.perf_counter() - t0, oracle.default_threads(), heads
 
 
-def time_call_graph(step, causal: bool, steps: int):
-    """ms per fa_bwd call for one mask: the call captured alone as a CUDA graph
-    and replayed, L2 flushed between replays outside the events."""
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(s):
-        step._bwd(0, causal)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=s):
-            step._bwd(0, causal)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    for _ in range(3):
-        step.flush_l2()
-        g.replay()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for e0, e1 in ev:
-        step.flush_l2()
-        e0.record()
-        g.replay()
-        e1.record()
-    torch.cuda.synchronize()
-    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+def headline_workload_name(c=HEADLINE) -> str:
+    return (f"fwd b{c['B']}h{c['H']}n{c['N']}d{c['d']} {'causal' if c['causal'] else 'non-causal'} bf16 "
+            "(the sequence sweep's largest configuration, B*N = 16384)")
+
+
+def headline_config(world: int) -> dict:
+    c = HEADLINE
+    return {"workload": headline_workload_name(), "B": c["B"], "H": c["H"], "N": c["N"], "d": c["d"],
+            "causal": c["causal"], "parallelism": f"replicas x{world}",
+            "l2": "inputs (201 MB) larger than L2, and L2 flushed between steps (512 MB write outside the timed "
+                  "events)"}
+
+
+def reference_fwd(args, world: int, rank: int):
+    """The reference arm: the oracle on the headline workload, one bounded row
+    sample per step, on the host cores (rank 0 only)."""
+    if rank == 0:
+        import numpy as np
+
+        samp = OracleSampler(HEADLINE)
+        rng = np.random.default_rng(HEADLINE["seed"])
+        per_step = max(0.5, min(args.cpu_seconds / 2, 60.0 / max(1, args.steps + args.warmup)))
+        rows_n = samp.rows_for(per_step, rng)
+        for _ in range(args.warmup):
+            samp.run(rows_n, rng)
+        runs = [samp.run(rows_n, rng) for _ in range(args.steps)]
+        fl, sec = sum(r[0] for r in runs), sum(r[1] for r in runs)
+        val = fl / sec / 1e12
+        cfg = headline_config(1)
+        cfg.pop("parallelism")
+        cfg["l2"] = "n/a (CPU)"
+        line = {
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1))", "config": cfg,
+            "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": samp.threads, "kind": "oracle",
+                             "sample": f"{rows_n} random query rows of the workload per step, exact fp64"},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+def reference_bwd(args, world: int, rank: int):
+    if rank == 0:
+        oracle_bwd_sample(1.0, SEED + 100)
+        runs = [oracle_bwd_sample(args.cpu_seconds / 2, SEED + i) for i in range(args.steps)]
+        fl, sec = sum(r[0] for r in runs), sum(r[1] for r in runs)
+        val = fl / sec / 1e12
+        line = {
+            "impl": "reference", "metric": BWD_METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": f"bwd b{B}h{H}n{N}d{D}: fa_bwd non-causal + fa_bwd causal", "B": B, "H": H,
+                       "N": N, "d": D, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": runs[0][2], "kind": "oracle",
+                             "sample": f"{runs[0][3]} whole heads per step, non-causal and causal alternately, "
+                                       "fp64 numpy"},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+def reference_decode(args, world: int, rank: int):
+    """The oracle on the whole decode problem (every query row) per step."""
+    if rank == 0:
+        import oracle
+
+        c = DECODE
+        q, k, v = fa_inputs.qkv_decode(c["B"], c["H"], c["Nq"], c["Nk"], c["d"], c["seed"])
+        qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+        n = c["B"] * c["H"]
+        nbytes = 2.0 * n * c["Nk"] * c["d"] * 2 + n * c["Nq"] * c["d"] * 2 * 2 + n * c["Nq"] * 4
+        for _ in range(args.warmup):
+            oracle.attention(qd, kd, vd, False, c["d"] ** -0.5)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.attention(qd, kd, vd, False, c["d"] ** -0.5)
+        sec = time.perf_counter() - t0
+        val = nbytes * args.steps / sec / 1e9
+        line = {
+            "impl": "reference", "metric": DECODE_METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": f"decode b{c['B']}h{c['H']} nq{c['Nq']} nk{c['Nk']} d{c['d']}",
+                       **{key: c[key] for key in ("B", "H", "Nq", "Nk", "d")}, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
+                             "sample": "every query row of the problem per step, exact fp64"},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+# ------------------------------------------------------------- GPU lines --
+def clocks_entry(clocks: dict) -> dict:
+    return {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+            "samples": clocks["samples"], "source": clocks["source"]}
+
+
+def run_fwd(args, world: int, rank: int, local: int):
+    c = HEADLINE
+    step = FwdStep(c["B"], c["H"], c["N"], c["d"], c["causal"], c["seed"] + rank)
+    graph = capture_step(step)
+    with ClockSampler(local) as clk:
+        step_ms, _ = time_steps(step, graph, args.steps, args.warmup, world)
+    del graph
+    e2e_ms = None if args.no_e2e else dist_max(time_e2e(step, max(8, args.steps // 2), 3, world), world)
+    ms = dist_max(statistics.mean(step_ms), world)
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    h2d, d2h = step.h2d_bytes, step.d2h_bytes
+    del step
+    torch.cuda.empty_cache()
+    more = extras(peaks, max(5, args.steps // 2)) if (not args.no_extras and world == 1) else {}
+    if rank == 0:
+        # one launch per step: the step time is the kernel's launch duration
+        achieved = attn_flops(c["B"], c["H"], c["N"], c["d"], c["causal"]) / (ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": world * achieved, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+            "config": headline_config(world),
+            "timing": "value: CUDA-graph replay of one fa_fwd launch per step, events on the replay stream; "
+                      "sub-objects: each workload's calls replayed the same way",
+            "roofline": {"kernel": "attn_fwd_kernel<128,2,nc,bf16>", "bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": measured_traffic(), "traffic_unit": "bytes per launch (ncu dram read + write)",
+                         "algorithmic_bytes": 8.0 * c["B"] * c["H"] * c["N"] * c["d"] + 4.0 * c["B"] * c["H"] * c["N"],
+                         "peak_source": f"{peak_src} cuBLAS bf16 (burst; the kernel is timed alone)"},
+            "gpu_launches": args.steps,
+            "clocks": clocks_entry(clocks),
+        }
+        if e2e_ms is not None:
+            line["e2e"] = {"value": world * achieved * ms / e2e_ms, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                           "d2h_bytes_per_step": d2h,
+                           "note": "fwd() with Q, K, V copied in from pinned host memory and O, LSE copied out "
+                                   "every step; steps pipelined over three CUDA streams (copy in, compute, copy "
+                                   "out) with two sets of device buffers"}
+        line.update(more)
+        if not args.no_cpu_baseline and world == 1:
+            import numpy as np
+
+            samp = OracleSampler(HEADLINE)
+            rng = np.random.default_rng(HEADLINE["seed"])
+            rows_n = samp.rows_for(args.cpu_seconds, rng)
+            fl, sec = samp.run(rows_n, rng)
+            line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": samp.threads,
+                                    "kind": "oracle",
+                                    "sample": f"{rows_n} random query rows of the workload, exact fp64, {sec:.1f} s"}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
 
 
 def run_bwd(args, world: int, rank: int):
@@ -639,7 +946,8 @@ def run_bwd(args, world: int, rank: int):
     graph = capture_step(step)
     with ClockSampler(torch.cuda.current_device()) as clk:
         step_ms, _ = time_steps(step, graph, args.steps, args.warmup, world)
-    comp = [dist_max(time_call_graph(step, c, args.steps), world) for c in (False, True)]
+    flush = _Flush()
+    comp = [dist_max(time_call(lambda: step._bwd(0, c), args.steps, flush), world) for c in (False, True)]
     e2e_ms = dist_max(time_e2e(step, max(8, args.steps // 2), 3, world), world)
     ms = dist_max(statistics.mean(step_ms), world)
     peaks, peak_src = load_peaks()
@@ -668,132 +976,13 @@ def run_bwd(args, world: int, rank: int):
                     "note": "Q, K, V, dO and both masks' O and LSE copied in, the six gradients copied out, per "
                             "step; steps pipelined over three CUDA streams (copy in, compute, copy out)"},
             "gpu_launches": step.launches_per_step * args.steps,
-            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
+            "clocks": clocks_entry(clocks),
         }
         if not args.no_cpu_baseline and world == 1:
             fl, sec, cores, heads = oracle_bwd_sample(args.cpu_seconds, SEED)
             line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                                     "sample": f"{heads} whole heads (N={N}, d={D}) of the workload, non-causal and "
                                               f"causal alternately, fp64 numpy, {sec:.1f} s"}
-        print(json.dumps(line), flush=True)
-    dist_done(world)
-
-
-# ------------------------------------------------------------------- main --
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["step", "decode", "bwd"], default="step")
-    args = ap.parse_args()
-    world, rank, local = dist_setup()
-
-    if args.impl == "reference" and args.workload == "bwd":
-        if rank == 0:
-            oracle_bwd_sample(1.0, SEED + 100)
-            runs = [oracle_bwd_sample(args.cpu_seconds / 2, SEED + i) for i in range(args.steps)]
-            fl, sec = sum(r[0] for r in runs), sum(r[1] for r in runs)
-            val = fl / sec / 1e12
-            line = {
-                "impl": "reference", "metric": BWD_METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic (seeded N(0,1))",
-                "config": {"workload": f"bwd b{B}h{H}n{N}d{D}: fa_bwd non-causal + fa_bwd causal", "B": B, "H": H,
-                           "N": N, "d": D, "l2": "n/a (CPU)"},
-                "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": runs[0][2], "kind": "oracle",
-                                 "sample": f"{runs[0][3]} whole heads per step, non-causal and causal alternately, "
-                                           "fp64 numpy"},
-                "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            }
-            print(json.dumps(line), flush=True)
-        dist_done(world)
-        return
-
-    if args.impl == "reference":
-        if rank == 0:
-            warm = [oracle_sample(2.0, SEED + 100 + i) for i in range(args.warmup)]
-            del warm
-            runs = [oracle_sample(args.cpu_seconds / 2, SEED + i) for i in range(args.steps)]
-            fl = sum(r[0] for r in runs)
-            sec = sum(r[1] for r in runs)
-            val = fl / sec / 1e12
-            line = {
-                "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic (seeded N(0,1))",
-                "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "l2": "n/a (CPU)"},
-                "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": runs[0][2], "kind": "oracle",
-                                 "sample": f"{runs[0][3]} random query rows per attention pass per step, "
-                                           "3 passes (non-causal, causal, non-causal), exact fp64"},
-                "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            }
-            print(json.dumps(line), flush=True)
-        dist_done(world)
-        return
-
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device for --impl ours")
-    torch.cuda.set_device(local)
-    if args.workload == "decode":
-        run_decode(args, world, rank)
-        return
-    if args.workload == "bwd":
-        run_bwd(args, world, rank)
-        return
-    step = Step(SEED + rank)
-    graph = capture_step(step)
-    with ClockSampler(local) as clk:
-        step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
-    e2e_ms = time_e2e(step, max(8, args.steps // 2), 3, world)
-    ms_local = statistics.mean(step_ms)
-    ms = dist_max(ms_local, world)
-    e2e_ms = dist_max(e2e_ms, world)
-    comp = [statistics.mean(p[j] for p in per) for j in range(4)]
-    comp = [dist_max(c, world) for c in comp]
-    peaks, peak_src = load_peaks()
-    clocks = clk.summary()
-
-    if rank == 0:
-        value = world * STEP_FLOPS / (ms * 1e-3) / 1e12
-        nc_ms = comp[0]
-        achieved = flops_fwd(False) / (nc_ms * 1e-3) / 1e12
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
-            "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "parallelism": f"replicas x{world}",
-                       "l2": "flushed between steps (512 MB write outside the timed events)"},
-            "timing": "value: CUDA-graph replay of the step; breakdown: eager calls, events per kernel group",
-            "breakdown_ms": {"bf16_noncausal": comp[0], "bf16_causal": comp[1], "rotate_quant_qk": comp[2],
-                             "e4m3qk_noncausal": comp[3]},
-            "breakdown_tflops": {"bf16_noncausal": flops_fwd(False) / comp[0] / 1e9,
-                                 "bf16_causal": flops_fwd(True) / comp[1] / 1e9,
-                                 "e4m3qk_noncausal": flops_fwd(False) / comp[3] / 1e9},
-            "roofline": {"kernel": "attn_fwd_kernel<128,2,nc,bf16>", "bound": "tensor", "achieved": achieved,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops"], "traffic": measured_traffic(),
-                         "traffic_unit": "bytes per launch (ncu dram read + write)",
-                         "peak_source": f"{peak_src} cuBLAS bf16 (burst)"},
-            "e2e": {"value": world * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
-                    "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
-                    "note": "steps pipelined over three CUDA streams (copy in, compute, copy out) with two sets of "
-                            "device buffers; every step copies its inputs in and its results out"},
-            "gpu_launches": step.launches_per_step * args.steps,
-            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
-        }
-        if not args.no_cpu_baseline and world == 1:
-            fl, sec, cores, rows_n = oracle_sample(args.cpu_seconds, SEED)
-            line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-                                    "sample": f"{rows_n} random query rows x 3 attention passes of the workload, "
-                                              f"exact fp64, {sec:.1f} s"}
         print(json.dumps(line), flush=True)
     dist_done(world)
 
@@ -834,11 +1023,39 @@ def run_decode(args, world: int, rank: int):
                     "note": "K/V cache resident on the device; Q in, O and LSE out per step; steps pipelined over "
                             "three CUDA streams (copy in, compute, copy out)"},
             "gpu_launches": step.launches_per_step * args.steps,
-            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                       "reasons": clocks["reasons"], "samples": clocks["samples"], "source": clocks["source"]},
+            "clocks": clocks_entry(clocks),
         }
         print(json.dumps(line), flush=True)
     dist_done(world)
+
+
+# ------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="headline only: skip the other workloads")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host copies) measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--workload", choices=["fwd", "decode", "bwd"], default="fwd")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        {"fwd": reference_fwd, "bwd": reference_bwd, "decode": reference_decode}[args.workload](args, world, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    if args.workload == "decode":
+        run_decode(args, world, rank)
+    elif args.workload == "bwd":
+        run_bwd(args, world, rank)
+    else:
+        run_fwd(args, world, rank, local)
 
 
 if __name__ == "__main__":

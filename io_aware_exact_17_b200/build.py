@@ -30,20 +30,30 @@ def sources() -> list[Path]:
         (ROOT / "include").glob("*.h"))
 
 
-def needs_build() -> bool:
-    if not LIB.exists():
+# The test build: the same sources with the test hooks compiled in (a forward
+# launch can be made to leave out one software mbarrier arrival) and a 5 ms
+# wait limit, so that a test can make a bounded wait run out and check that the
+# kernel returns with FA_ERR_TIMEOUT. Only tests load it.
+TEST_LIB = PKG / "libfa_testhooks.so"
+TEST_DEFINES = ["-DFA_TEST_HOOKS", "-DFA_WAIT_LIMIT_NS=5000000ull"]
+
+
+def needs_build_of(lib: Path) -> bool:
+    if not lib.exists():
         return True
-    t = LIB.stat().st_mtime
+    t = lib.stat().st_mtime
     return any(s.stat().st_mtime > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> Path:
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB.with_suffix(".so.tmp")
+def needs_build() -> bool:
+    return needs_build_of(LIB)
+
+
+def _compile(lib: Path, defines: list[str], verbose: bool) -> Path:
+    tmp = lib.with_suffix(".so.tmp")
     cmd = [
         _nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-        "--expt-relaxed-constexpr", "-o", str(tmp), str(CSRC / "fa_api.cu"),
+        "--expt-relaxed-constexpr", *defines, "-o", str(tmp), str(CSRC / "fa_api.cu"),
     ]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -52,10 +62,24 @@ def build(force: bool = False, verbose: bool = False) -> Path:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> Path:
+    if not force and not needs_build():
+        return LIB
+    return _compile(LIB, [], verbose)
+
+
+def build_test_hooks(force: bool = False, verbose: bool = False) -> Path:
+    """Build libfa_testhooks.so (see TEST_DEFINES); tests only."""
+    if not force and not needs_build_of(TEST_LIB):
+        return TEST_LIB
+    return _compile(TEST_LIB, TEST_DEFINES, verbose)
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
+    build_test_hooks(force="--force" in sys.argv)
     print(LIB)

@@ -749,7 +749,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
+#ifdef FA_TEST_HOOKS
+      const bool withhold = lane == 0 && warp == 0 && blockIdx.x == 0 && round == 0 && j == 1 &&
+                            atomicExch(&g_fa_test_withhold_p, 0) != 0;
+      if (lane == 0 && !withhold) mbar_arrive(&bar_p[t]);
+#else
       if (lane == 0) mbar_arrive(&bar_p[t]);  // one arrival per warp
+#endif
     }
     if (ok && n_kv_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[t], oc & 1u, &abort_flag, st, 40 + t));
     if (n_kv_t > 0) ++oc;

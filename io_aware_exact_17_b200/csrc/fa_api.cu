@@ -714,4 +714,13 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
 
 int fa_abi_version(void) { return 4; }
 
+#ifdef FA_TEST_HOOKS
+// Test build only (not declared in include/, not in the product library): arm
+// the withheld P arrival of the next forward launch on the current device.
+int fa_test_withhold_p_arrive(int on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(fa::g_fa_test_withhold_p, &v, sizeof(v)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 }  // extern "C"

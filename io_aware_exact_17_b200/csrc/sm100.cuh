@@ -30,7 +30,21 @@ __device__ DevStatus g_fa_status;  // first device-side error of any launch of t
 
 // 1 s: no legitimate wait inside one CTA comes near this (the longest kernels
 // run for milliseconds), so hitting it means a lost arrival, not slowness.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// The test build (FA_TEST_HOOKS) sets a few milliseconds, so that a test can
+// make a wait run out quickly.
+#ifndef FA_WAIT_LIMIT_NS
+#define FA_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = FA_WAIT_LIMIT_NS;
+
+#ifdef FA_TEST_HOOKS
+// Test build only (never in the product library): when nonzero, softmax warp 0
+// of CTA 0 of the next forward launch leaves out its arrival on the P barrier
+// of its first query tile at key tile 1 of its first work item, and clears the
+// word. The MMA issuer's wait for that P then runs out; it is a plain software
+// arrival, so no copy or tensor-core operation is left in flight.
+__device__ int g_fa_test_withhold_p;
+#endif
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;

@@ -10,7 +10,7 @@ import pytest
 ROOT = Path(__file__).resolve().parents[1]
 
 
-@pytest.mark.parametrize("workload", ["step", "bwd"])
+@pytest.mark.parametrize("workload", ["fwd", "bwd"])
 def test_reference_arm_prints_one_line(workload):
     out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--workload", workload,
                           "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"],
