@@ -195,7 +195,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  *             may be NULL when rows = 0.
  * out         device, e4m3 codes [rows][d], 16-byte aligned; may be NULL when rows = 0.
  * descale_out device, one fp32 (written in the second pass, after the grid-wide amax).
- * rows >= 0;  d in {64, 128, 256}.
+ * rows        0 .. 2^31 - 4097 (TMA tile coordinates are 32-bit; a larger bf16
+ *             tensor would not fit in device memory);  d in {64, 128, 256}.
  * rotate      0 = quantise only, 1 = rotate first.
  * signs       device, d fp32 values +-1 (16-byte aligned), or NULL for no sign flips.
  * workspace   device scratch of >= FA_QUANT_WORKSPACE_BYTES bytes, 16-byte aligned,

@@ -277,6 +277,10 @@ size_t plan_bytes(const Plan& pl, int B, int H, int Nq, int d) {
   return pl.n_split <= 1 ? 0 : part_bytes(B, H, Nq, d, pl.n_split);
 }
 
+// Largest row count of the quantisers: TMA tile coordinates are 32-bit (such a
+// tensor of bf16 rows would not fit in a GPU's memory anyway).
+constexpr int64_t kQuantMaxRows = (static_cast<int64_t>(1) << 31) - 4096;
+
 template <int D>
 fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t rows, int rotate, const float* signs,
                        unsigned int* amax, cudaStream_t stream) {
@@ -305,38 +309,49 @@ fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t row
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// Both quantisation passes in one cooperative launch (quant_fused_kernel) for
+// Both quantisation passes in one cooperative launch (quant_tma_kernel) for
 // the tensors of `b`: the workspace holds their amax words and the grid
-// barrier's counter, zeroed here.
+// barrier's counter, zeroed here. One CTA per SM (up to one per row block), all
+// co-resident.
 template <int D>
 fa_status launch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int rotate,
                              const float* signs, unsigned int* ws, cudaStream_t stream) {
-  using FC = fa::FusedCfg<D>;
+  using TC = fa::TmaQuantCfg<D>;
   if (cudaMemsetAsync(ws, 0, (b.n + 1) * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
-  auto kernel = rotate ? fa::quant_fused_kernel<D, true> : fa::quant_fused_kernel<D, false>;
-  // Co-resident blocks per SM and SM count, looked up once per device (this is
-  // host time in front of a ~10 us kernel).
+  if (rows == 0) {  // nothing to read: every descale is 1
+    fa::fill_f32_kernel<<<1, 32, 0, stream>>>(descale_out, b.n, 1.0f);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  auto kernel = rotate ? fa::quant_tma_kernel<D, true> : fa::quant_tma_kernel<D, false>;
+  static unsigned long long smem_set[2] = {0, 0};
+  if (!set_smem_once(kernel, TC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
+  // Co-resident CTAs per SM, looked up once per device (host time in front of
+  // a ~20 us kernel).
   static int cached_per_sm[2][64] = {};
-  static int cached_sms[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
   int& per_sm = cached_per_sm[rotate ? 1 : 0][dev];
-  int& sms = cached_sms[dev];
-  if (sms == 0 && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
   if (per_sm == 0 &&
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, fa::kFusedThreads, 0) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, TC::THREADS, TC::SMEM) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (per_sm < 1 || sms < 1) return FA_ERR_CUDA;
-  const int64_t steps = (rows + FC::RPW - 1) / FC::RPW;  // warp-steps of work per tensor
-  int64_t blocks = (steps + fa::kFusedThreads / 32 - 1) / (fa::kFusedThreads / 32);
-  const int64_t cap = static_cast<int64_t>(per_sm) * sms;  // all blocks co-resident
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  fa::QuantBatch bb = b;
-  void* args[] = {&bb, &rows, &signs, &ws, &descale_out};
+  if (per_sm < 1) return FA_ERR_CUDA;
+  const int64_t nblk = (rows + TC::RB - 1) / TC::RB;
+  int64_t blocks = static_cast<int64_t>(per_sm) * device_sms();
+  if (blocks > nblk) blocks = nblk;
+  fa::QuantMaps qm;
+  std::memset(&qm, 0, sizeof(qm));
+  for (int t = 0; t < b.n; ++t) {
+    if (!fa::make_tmap_2d(&qm.x[t], b.x[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(rows), 64,
+                          TC::BOX_ROWS))
+      return FA_ERR_CUDA;
+    qm.out[t] = b.out[t];
+  }
+  qm.n = b.n;
+  int rows_i = static_cast<int>(rows);
+  void* args[] = {&qm, &rows_i, &signs, &ws, &descale_out};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(static_cast<unsigned>(blocks)),
-                                  dim3(fa::kFusedThreads), args, 0, stream) != cudaSuccess)
+                                  dim3(TC::THREADS), args, TC::SMEM, stream) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }
@@ -550,7 +565,7 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
   if (rows > 0 && (x == nullptr || out == nullptr)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < FA_QUANT_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  if (rows > (static_cast<int64_t>(1) << 40)) return FA_ERR_INVALID_ARG;
+  if (rows > kQuantMaxRows) return FA_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(descale_out, 4))
     return FA_ERR_ALIGNMENT;
   if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
@@ -568,7 +583,7 @@ fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, floa
                                   size_t workspace_bytes, void* stream) {
   if (xs == nullptr || outs == nullptr || descales == nullptr || workspace == nullptr) return FA_ERR_INVALID_ARG;
   if (ntensors < 1 || ntensors > fa::kQuantBatch) return FA_ERR_INVALID_ARG;
-  if (rows < 0 || rows > (static_cast<int64_t>(1) << 40) || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (rows < 0 || rows > kQuantMaxRows || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < FA_QUANT_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (!aligned(descales, 4) || !aligned(workspace, 16)) return FA_ERR_ALIGNMENT;

@@ -13,12 +13,13 @@
 // Two streaming passes over the bf16 input, both HBM/L2-bound:
 //   pass 1: rotate, reduce |x'| to one block max, atomicMax into a scratch word;
 //   pass 2: rotate again, scale, convert, store the codes.
-// A tensor of up to ~60 MB stays in the 126 MB L2 between the passes, so the
-// second read mostly hits L2. quant_fused_kernel runs both passes in one
-// cooperative launch, for up to 8 tensors at once (each with its own scale);
-// quant_amax_kernel + quant_apply_kernel are the two-launch form (used where
-// the scratch is the library's own static array). quant_block_kernel (end of
-// the file) takes one scale per 128-row block of a head, in one pass.
+// Tensors of up to ~100 MB stay in the 126 MB L2 between the passes, so the
+// second read mostly hits L2. quant_tma_kernel runs both passes in one
+// cooperative launch, for up to 8 tensors at once (each with its own scale),
+// with the input staged through shared memory by TMA; quant_amax_kernel +
+// quant_apply_kernel are the two-launch form (used where the scratch is the
+// library's own static array). quant_block_kernel (end of the file) takes one
+// scale per 128-row block of a head, in one pass.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -172,16 +173,11 @@ quant_apply_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
 namespace fa {
 
 // ---------------------------------------------------------------------------
-// One-launch variant: both passes in one cooperative kernel with a grid-wide
-// barrier between them (all blocks are co-resident, which the cooperative
-// launch guarantees), 32 elements per thread (fewer cross-lane butterfly
-// stages), and the second pass re-reading the tensor while it is still in L2.
-// The butterfly stages run in the same order (index bits 0, 1, 2, ...) with
-// the same operands as hadamard_rotate, so the codes are bit-identical to the
-// two-kernel path.
+// 32 elements per thread (four interleaved 16-byte chunks of a row), for the
+// per-block kernel. The butterfly stages run in the same order (index bits 0,
+// 1, 2, ...) with the same operands as hadamard_rotate, so the codes are
+// bit-identical to the two-kernel path.
 // ---------------------------------------------------------------------------
-constexpr int kFusedThreads = 256;
-
 template <int D>
 struct FusedCfg {
   static constexpr int E = 32;          // elements per thread (four 16-byte chunks)
@@ -299,59 +295,232 @@ struct QuantBatch {
   int n;
 };
 
-// ws[0 .. n-1]: amax bits of each tensor, ws[n]: arrival counter of the grid
-// barrier; all zero at launch. descale_out[i]: tensor i's descale.
+// ---------------------------------------------------------------------------
+// Per-tensor scales in one cooperative launch, with the input staged through
+// shared memory by TMA (quant_tma_kernel).
+//
+// One CTA per SM. A producer warp streams blocks of RB rows of the tensors
+// through a ring of stages (TMA, 128-byte swizzle), far enough ahead to keep
+// HBM busy; 16 consumer warps take one stage at a time, each thread 64
+// consecutive elements of one row (a whole 128-byte swizzle column), so the
+// first six butterfly stages of the rotation stay inside the thread and only
+// log2(d / 64) stages cross lanes. Pass 1 reduces |x'| per tensor; a bounded
+// grid barrier publishes the amax words; pass 2 streams the same blocks again,
+// in reverse order so that the most recently read ones, still in L2, come
+// first, and writes the codes. The producer runs on into pass 2 while the
+// consumers wait at the barrier.
+//
+// The butterflies run over index bits 0, 1, ... in increasing order with the
+// same operations as hadamard_rotate and hadamard_rotate32, so the codes are
+// bit-identical to the two-launch kernels'. Pass 1 takes the max before the
+// 1/sqrt(d) factor and multiplies it once: fp32 rounding is monotonic, so
+// max_i fl(|v_i| c) = fl(c max_i |v_i|).
+// ---------------------------------------------------------------------------
+// descale_out[0 .. n-1] = v (the descales of empty tensors).
+__global__ void fill_f32_kernel(float* out, int n, float v) {
+  if (static_cast<int>(threadIdx.x) < n) out[threadIdx.x] = v;
+}
+
+constexpr int kTmaQuantConsumers = 512;
+constexpr int kTmaQuantStages = 3;
+
+template <int D>
+struct TmaQuantCfg {
+  static constexpr int E = 64;                           // elements per thread: one 128-byte column
+  static constexpr int TPR = D / E;                      // threads per row
+  static constexpr int RB = kTmaQuantConsumers / TPR;    // rows per stage
+  static constexpr int BOX_ROWS = RB < 256 ? RB : 256;   // TMA box height (at most 256)
+  static constexpr int COLS = D / 64;                    // 128-byte columns per row
+  static constexpr int STAGE = RB * D * 2;               // bytes per stage (64 KB)
+  static constexpr int CONSUMER_WARPS = kTmaQuantConsumers / 32;
+  static constexpr int THREADS = kTmaQuantConsumers + 32;  // + the producer warp
+  static constexpr int SMEM = 1024 + kTmaQuantStages * STAGE;
+  static_assert(D == 64 || D == 128 || D == 256, "head dim");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct QuantMaps {
+  CUtensorMap x[kQuantBatch];  // tensor t as [rows][D] bf16, box (64, BOX_ROWS), 128-byte swizzle
+  uint8_t* out[kQuantBatch];
+  int n;
+};
+
+// In place: 64 consecutive elements e0 .. e0+63 of a row (w[i] = elements
+// e0+2i, e0+2i+1) become the same elements of (x * signs) H_D, without the
+// 1/sqrt(D) factor. The TPR threads of the row (lanes 8 apart, part p = e0 / 64
+// = bits 3.. of the lane) must call together.
 template <int D, bool ROT>
-__global__ void __launch_bounds__(kFusedThreads, 3)
-quant_fused_kernel(const QuantBatch b, int64_t rows, const float* __restrict__ signs, unsigned int* ws,
-                   float* descale_out) {
-  DevStatus* st = &g_fa_status;
-  using C = FusedCfg<D>;
-  const int lane = threadIdx.x & 31;
-  const int lr = lane % C::L, sub = lane / C::L;
-  const int64_t warp_g = (static_cast<int64_t>(blockIdx.x) * kFusedThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kFusedThreads) >> 5;
-  __shared__ float warp_max[kFusedThreads / 32];
-  __shared__ unsigned int amax_sh[kQuantBatch];
-  // pass 1: amax of each rotated tensor
-#pragma unroll 1
-  for (int t = 0; t < b.n; ++t) {
-    const __nv_bfloat16* x = b.x[t];
-    float m = 0.f;
-    for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
-      const int64_t row = w * C::RPW + sub;
-      float v[32];
-      if (row < rows) {
-        load_bf16x32<D>(x + row * D, lr, v);
-      } else {
+__device__ __forceinline__ void rotate64(uint64_t (&w)[32], int p, const float* sgn) {
+  if (!ROT) return;
+  if (sgn != nullptr) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.f;
-      }
-      if (ROT) hadamard_rotate32<D>(v, lr, signs);
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) m = fmax3(m, fabsf(v[e]), fabsf(v[e + 1]));
+    for (int i = 0; i < 32; i += 2) {
+      const float4 s4 = *reinterpret_cast<const float4*>(sgn + 64 * p + 2 * i);
+      w[i] = f2_mul(w[i], f2_pack(s4.x, s4.y));
+      w[i + 1] = f2_mul(w[i + 1], f2_pack(s4.z, s4.w));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) warp_max[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float bm = warp_max[0];
-#pragma unroll
-      for (int i = 1; i < kFusedThreads / 32; ++i) bm = fmaxf(bm, warp_max[i]);
-      atomicMax(&ws[t], __float_as_uint(bm));
-    }
-    __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    // Grid-wide barrier: every block is resident (cooperative launch). The wait
-    // is bounded; if it runs out the status word records it and the block goes on.
+  // index bit 0: inside each pair
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float a, b;
+    f2_unpack(w[i], a, b);
+    w[i] = f2_pack(a + b, a - b);
+  }
+  // index bits 1 .. 5: pair i with pair i + h
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & h) == 0) {
+        const uint64_t a = w[i], b = w[i + h];
+        w[i] = f2_add(a, b);
+        w[i + h] = f2_sub(a, b);
+      }
+    }
+  }
+  // index bits 6 ..: across the TPR lanes of the row (lower part: v + other,
+  // upper part: other - v, each one fma with +-1, i.e. one rounding)
+#pragma unroll
+  for (int m = 1; m < D / 64; m <<= 1) {
+    const float sg = (p & m) != 0 ? -1.0f : 1.0f;
+    const uint64_t sgn2 = f2_pack(sg, sg);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float a, b;
+      f2_unpack(w[i], a, b);
+      const float oa = __shfl_xor_sync(0xffffffffu, a, 8 * m);
+      const float ob = __shfl_xor_sync(0xffffffffu, b, 8 * m);
+      w[i] = f2_fma(w[i], sgn2, f2_pack(oa, ob));
+    }
+  }
+}
+
+// ws[0 .. n-1]: amax bits of each tensor, ws[n]: arrival counter of the grid
+// barrier; all zero at launch. descale_out[t]: tensor t's descale.
+template <int D, bool ROT>
+__global__ void __launch_bounds__(TmaQuantCfg<D>::THREADS, 1)
+quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __restrict__ signs, unsigned int* ws,
+                 float* descale_out) {
+  using C = TmaQuantCfg<D>;
+  constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kTmaQuantStages], empty[kTmaQuantStages];
+  __shared__ __align__(16) float sgn[D];
+  __shared__ unsigned int amax_cta[kQuantBatch];
+  __shared__ float amax_all[kQuantBatch];
+  __shared__ volatile int abort_flag;
+  DevStatus* st = &g_fa_status;
+  const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
+  const int nblk = (rows + C::RB - 1) / C::RB;  // row blocks per tensor
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int per = c < nblk ? (nblk - 1 - c) / G + 1 : 0;  // this CTA's blocks per tensor
+  const int K = per * qm.n;                               // this CTA's steps per pass
+  // Step k of pass 1: tensor k / per, row block c + (k % per) * G. Pass 2 takes
+  // the same steps in reverse; stream position s = 0 .. 2K-1 covers both.
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < kTmaQuantStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], C::CONSUMER_WARPS);
+    }
+    for (int t = 0; t < kQuantBatch; ++t) amax_cta[t] = 0u;
+    fence_mbar_init();
+  }
+  if (ROT && tid < D) sgn[tid] = signs != nullptr ? signs[tid] : 1.0f;
+  __syncthreads();
+
+  if (warp == C::CONSUMER_WARPS) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      for (int t = 0; t < qm.n; ++t) tma_prefetch_desc(&qm.x[t]);
+      bool ok = true;
+      int s = 0;
+      for (; s < 2 * K && ok; ++s) {
+        const int k = s < K ? s : 2 * K - 1 - s;
+        const int t = k / per, b = c + (k % per) * G;
+        const int stage = s % kTmaQuantStages, round = s / kTmaQuantStages;
+        if (round > 0) ok = mbar_wait(&empty[stage], (round - 1) & 1, &abort_flag, st, 61);
+        if (!ok) break;
+        uint8_t* dst = smem + stage * C::STAGE;
+        mbar_arrive_expect_tx(&full[stage], C::STAGE);
+#pragma unroll
+        for (int col = 0; col < C::COLS; ++col)
+#pragma unroll
+          for (int r0 = 0; r0 < C::RB; r0 += C::BOX_ROWS)
+            tma_load_2d(dst + col * (C::RB * 128) + r0 * 128, &qm.x[t], &full[stage], col * 64, b * C::RB + r0);
+      }
+      // every issued load lands before the CTA can exit
+      for (int q = s - kTmaQuantStages; q < s; ++q)
+        if (q >= 0) {
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[q % kTmaQuantStages], (q / kTmaQuantStages) & 1))
+            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers --
+  // Lane bits 0-2: row (low bits), bits 3 .. 2+log2(TPR): the row's 64-element
+  // part p, higher bits: row (high bits). The 8 lanes of a shared-memory phase
+  // (one 16-byte load each) then read the same chunk j of 8 consecutive rows,
+  // whose swizzled positions j ^ (row & 7) are 8 different bank groups.
+  constexpr int LT = C::TPR == 1 ? 0 : (C::TPR == 2 ? 1 : 2);  // log2(TPR)
+  const int p = (lane >> 3) & (C::TPR - 1);
+  const int rr = warp * (32 / C::TPR) + (lane & 7) + 8 * (lane >> (3 + LT));  // row within the block
+  const uint8_t* my_col = smem + p * (C::RB * 128) + rr * 128;
+  const float* sg = (ROT && signs != nullptr) ? sgn : nullptr;
+  auto load_row = [&](int stage, uint64_t (&w)[32]) {
+    const uint8_t* base = my_col + stage * C::STAGE;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (rr & 7)) << 4));
+      w[4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
+      w[4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+      w[4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
+      w[4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+    }
+  };
+  bool ok = true;
+  float m = 0.f;
+  for (int s = 0; s < K; ++s) {
+    const int stage = s % kTmaQuantStages;
+    ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 62));
+    if (!ok) break;
+    uint64_t w[32];
+    load_row(stage, w);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    rotate64<D, ROT>(w, p, sg);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float a, b;
+      f2_unpack(w[i], a, b);
+      m = fmax3(m, fabsf(a), fabsf(b));
+    }
+    if (s % per == per - 1) {  // last block of tensor s / per
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) atomicMax(&amax_cta[s / per], __float_as_uint(m));
+      m = 0.f;
+    }
+  }
+  named_barrier_sync(1, kTmaQuantConsumers);
+  if (tid == 0) {
+    for (int t = 0; t < qm.n; ++t) {
+      const float cm = __uint_as_float(amax_cta[t]);
+      atomicMax(&ws[t], __float_as_uint(ROT ? cm * inv_sqrt_d : cm));
+    }
+    // Grid-wide barrier: every CTA is resident (cooperative launch). The wait
+    // is bounded; if it runs out the status word records it and the CTA goes on.
     __threadfence();
-    atomicAdd(&ws[b.n], 1u);
+    atomicAdd(&ws[qm.n], 1u);
     const unsigned long long t0 = globaltimer_ns();
     unsigned int arrived;
     for (;;) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + b.n) : "memory");
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + qm.n) : "memory");
       if (arrived >= gridDim.x) break;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         if (atomicCAS(&st->code, 0u, 5u) == 0u) {
@@ -362,42 +531,43 @@ quant_fused_kernel(const QuantBatch b, int64_t rows, const float* __restrict__ s
       }
       __nanosleep(64);
     }
-    for (int t = 0; t < b.n; ++t) {
+    for (int t = 0; t < qm.n; ++t) {
       unsigned int a;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(ws + t) : "memory");
-      amax_sh[t] = a;
+      amax_all[t] = __uint_as_float(a);
+      if (blockIdx.x == 0) descale_out[t] = __uint_as_float(a) > 0.f ? __uint_as_float(a) / 448.0f : 1.0f;
     }
   }
-  __syncthreads();
-  // pass 2: quantise (each tensor is re-read, mostly from L2)
-#pragma unroll 1
-  for (int t = 0; t < b.n; ++t) {
-    const __nv_bfloat16* x = b.x[t];
-    uint8_t* out = b.out[t];
-    const float amax = __uint_as_float(amax_sh[t]);
-    const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
-    if (blockIdx.x == 0 && threadIdx.x == 0) descale_out[t] = amax > 0.f ? amax / 448.0f : 1.0f;
-    for (int64_t w = warp_g; w * C::RPW < rows; w += nwarps) {
-      const int64_t row = w * C::RPW + sub;
-      float v[32];
-      if (row < rows) {
-        load_bf16x32<D>(x + row * D, lr, v);
-      } else {
+  named_barrier_sync(1, kTmaQuantConsumers);
+  if (!ok) return;
+  const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
+  for (int s = K; s < 2 * K; ++s) {
+    const int k = 2 * K - 1 - s;
+    const int t = k / per, b = c + (k % per) * G;
+    const int stage = s % kTmaQuantStages;
+    ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 63));
+    if (!ok) break;
+    uint64_t w[32];
+    load_row(stage, w);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    rotate64<D, ROT>(w, p, sg);
+    const float amax = amax_all[t];
+    const float sc = amax > 0.f ? 448.0f / amax : 1.0f;
+    const uint64_t sc2 = f2_pack(sc, sc);
+    uint32_t q[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.f;
-      }
-      if (ROT) hadamard_rotate32<D>(v, lr, signs);
-      uint32_t q[8];
+    for (int i = 0; i < 16; ++i) {
+      float a0, b0, a1, b1;
+      f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i], isd) : w[2 * i], sc2), a0, b0);
+      f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i + 1], isd) : w[2 * i + 1], sc2), a1, b1);
+      q[i] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
+    }
+    const int row = b * C::RB + rr;
+    if (row < rows) {
+      uint4* dst = reinterpret_cast<uint4*>(qm.out[t] + static_cast<int64_t>(row) * D + 64 * p);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        q[i] = static_cast<uint32_t>(pack_e4m3x2(v[4 * i] * scale, v[4 * i + 1] * scale)) |
-               (static_cast<uint32_t>(pack_e4m3x2(v[4 * i + 2] * scale, v[4 * i + 3] * scale)) << 16);
-      if (row < rows) {
-        // chunk c of the row (8 codes, 8 bytes) goes to out[row*D + 8c]
-        uint2* dst = reinterpret_cast<uint2*>(out + row * D);
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
-      }
+      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
     }
   }
 }

@@ -39,4 +39,21 @@ inline bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType
   return r == CUDA_SUCCESS;
 }
 
+// A 2-D row-major tensor [dim1][dim0] (dim0 contiguous), tiled in boxes of
+// box0 x box1 with the 128-byte swizzle (box0 * esize must be 128 bytes or
+// less). Out-of-range elements of a box read as zero. Returns false on failure.
+inline bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int esize, uint64_t dim0,
+                         uint64_t dim1, uint32_t box0, uint32_t box1) {
+  auto enc = get_encode_tiled();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {dim0, dim1};
+  cuuint64_t strides[1] = {dim0 * static_cast<uint64_t>(esize)};
+  cuuint32_t box[2] = {box0, box1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fa

@@ -52,7 +52,7 @@ def _quant_check(x, rotate, signs):
 
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("rotate", [False, True])
-@pytest.mark.parametrize("rows", [1, 7, 1000, 33333])
+@pytest.mark.parametrize("rows", [1, 7, 1000, 33333, 150001])
 def test_quant_matches_oracle(d, rotate, rows):
     g = torch.Generator().manual_seed(rows + d)
     x = torch.randn(rows, d, generator=g).to(torch.bfloat16)
@@ -61,7 +61,7 @@ def test_quant_matches_oracle(d, rotate, rows):
         _quant_check(x, True, inputs.hadamard_signs(d, seed=rows))
 
 
-@pytest.mark.parametrize("n", [1, 2, 3])
+@pytest.mark.parametrize("n", [1, 2, 3, 8])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_quant_multi_equals_one_call_per_tensor(n, rotate):
     # tensors of very different ranges, one launch, one scale each
