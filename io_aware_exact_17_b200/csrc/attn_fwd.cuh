@@ -130,11 +130,6 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
-#ifndef FA_EXP_POLY_EVERY
-#define FA_EXP_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FA_EXP_POLY_EVERY;  // 1 pair in kPolyEvery uses the polynomial (0: none)
-
 #ifndef FA_MMA_WAIT_SLEEP_NS
 #define FA_MMA_WAIT_SLEEP_NS 0
 #endif
@@ -146,9 +141,8 @@ constexpr uint32_t kMmaWaitSleepNs = FA_MMA_WAIT_SLEEP_NS;
 // Exponentials of one 32-key chunk of a row of S: p = 2^(x*s - m), packed to
 // bf16 pairs into pk[0..15]; accumulates the fp32 weights, with ROUND also the
 // bf16-rounded ones, into the packed-pair sums and (WITH_MAX) the raw-score max
-// into mx[0..3]. With EMU (a tile with no masked key) one pair in kPolyEvery goes
-// to the FMA-pipe polynomial.
-template <bool EMU, bool WITH_MAX, bool ROUND = true>
+// into mx[0..3].
+template <bool WITH_MAX, bool ROUND = true>
 __device__ __forceinline__ void exp_chunk32(const uint32_t* s, uint32_t* pk, uint64_t s2, uint64_t nm2,
                                             uint64_t* acc_e, uint64_t* acc_r, float* mx) {
 #pragma unroll
@@ -156,12 +150,8 @@ __device__ __forceinline__ void exp_chunk32(const uint32_t* s, uint32_t* pk, uin
     float t0, t1, p0, p1;
     if (WITH_MAX) mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
     f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), s2, nm2), t0, t1);
-    if (EMU && kPolyEvery > 0 && ((c >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-      exp2_poly_x2(t0, t1, p0, p1);
-    } else {
-      p0 = ex2_approx(t0);
-      p1 = ex2_approx(t1);
-    }
+    p0 = ex2_approx(t0);
+    p1 = ex2_approx(t1);
     const uint32_t q = pack_bf16x2(p0, p1);
     const int a = (c >> 1) & 1;
     acc_e[a] = f2_add(acc_e[a], f2_pack(p0, p1));
@@ -185,11 +175,11 @@ __device__ __forceinline__ void mask_chunk32(uint32_t* s, int kbase, int kmax) {
 // and the sum that normalises O.
 //
 // The normalising sum is the sum of the bf16-rounded weights P holds when some
-// key of the tile is masked (EMU false: the row's last tile, which holds every
+// key of the tile is masked (FULL false: the row's last tile, which holds every
 // key of a row with few keys), else the fp32 sum: over a full tile of 128 keys
 // the rounding errors of P average out to about 2^-9 / sqrt(128) of the sum, and
 // skipping the rounded sum saves three of the eight instructions per key pair.
-template <bool EMU>
+template <bool FULL>
 __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_log2, float m_ref,
                                             int kbase, int kmax, bool masked, float& sum_e, float& sum_r) {
   const uint64_t s2 = f2_pack(s_log2, s_log2);
@@ -202,7 +192,7 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_lo
   for (int ch = 0; ch < 4; ++ch) {
     if (ch < 3) tmem_ld32(tS + 32 * (ch + 1), &s[32 * (ch + 1)]);
     if (masked) mask_chunk32(&s[32 * ch], kbase + 32 * ch, kmax);
-    exp_chunk32<EMU, false, !EMU>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
+    exp_chunk32<false, !FULL>(&s[32 * ch], &s[16 * ch], s2, nm2, acc_e, acc_r, mx);
     if (ch < 3) tmem_wait_ld_dep32(&s[32 * (ch + 1)]);
   }
   float e0, e1, e2, e3, r0, r1, r2, r3;
@@ -211,7 +201,7 @@ __device__ __forceinline__ void softmax_row(uint32_t tS, uint32_t* s, float s_lo
   f2_unpack(acc_r[0], r0, r1);
   f2_unpack(acc_r[1], r2, r3);
   sum_e = (e0 + e1) + (e2 + e3);
-  sum_r = EMU ? sum_e : (r0 + r1) + (r2 + r3);
+  sum_r = FULL ? sum_e : (r0 + r1) + (r2 + r3);
 }
 
 // `masked` must be warp-uniform: both paths issue tcgen05.ld.
@@ -298,13 +288,13 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
       // later tiles hold only later keys, so it stays empty)
       m_ref = a == -INFINITY ? 0.f : a * s_log2;
       const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
-      exp_chunk32<false, false>(s, s, s2, nm2, acc_e, acc_r, mx);
+      exp_chunk32<false>(s, s, s2, nm2, acc_e, acc_r, mx);
     } else {
       uint32_t keep[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) keep[c] = s[c];
       const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
-      exp_chunk32<false, true>(s, s, s2, nm2, acc_e, acc_r, mx);
+      exp_chunk32<true>(s, s, s2, nm2, acc_e, acc_r, mx);
       const float mx_s = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * s_log2;
       const bool grow = mx_s > m_ref + 8.0f;
       if (__any_sync(0xffffffffu, grow)) {
@@ -313,7 +303,7 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
         m_ref = m_new;
         acc_e[0] = acc_e[1] = acc_r[0] = acc_r[1] = 0ull;
         const uint64_t nm2b = f2_pack(-m_ref, -m_ref);
-        exp_chunk32<false, false>(keep, s, s2, nm2b, acc_e, acc_r, mx);
+        exp_chunk32<false>(keep, s, s2, nm2b, acc_e, acc_r, mx);
         // rescale this warp's O rows (PV of the previous tile has completed)
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {

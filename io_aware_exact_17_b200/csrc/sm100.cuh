@@ -332,32 +332,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe, for two lanes at once: x = n + f with n = round(x) and
-// |f| <= 1/2 (Cody-Waite split via the 1.5*2^23 rounding constant), 2^f from a
-// degree-3 polynomial fitted for minimax relative error on [-1/2, 1/2]
-// (max relative error 7.5e-5 after fp32 evaluation), and 2^n added to the
-// exponent field. x is clamped below at -126, so the result is never zero:
-// callers use it only where no key is masked.
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f, c2 = 0.24261054396629333f,
-                  c3 = 0.05517132207751274f;
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));            // low bits hold round(x)
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));          // round(x) as float
-  const uint64_t f = f2_add(x, n ^ 0x8000000080000000ull);          // x - round(x)
-  uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
-  p = f2_fma(p, f, f2_pack(c1, c1));
-  p = f2_fma(p, f, f2_pack(c0, c0));
-  float t0, t1, p0, p1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(p, p0, p1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 

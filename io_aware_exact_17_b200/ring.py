@@ -67,9 +67,12 @@ def _default_merge(o_parts, lse_parts):
     return binding.lse_merge(o_parts, lse_parts)
 
 
-def _run_blocks(q, blocks, chunk_at, partial_fn, merge_fn):
+def _run_blocks(q, blocks, chunk_at, partial_fn, merge_fn, step_done=None):
     """Shared by the distributed and the single-device rings: partial results of
-    ``q`` over each block's chunk, then the merge."""
+    ``q`` over each block's chunk, then the merge. ``chunk_at(s)`` gives step s's
+    key/value chunk (the distributed ring also posts the exchange of the next
+    one there); ``step_done(s)``, if given, runs after step s's compute (the
+    distributed ring waits for that exchange)."""
     B, H, L, d = q.shape
     n = len(blocks)
     o_parts = torch.zeros((n, B, H, L, d), dtype=torch.float32, device=q.device)
@@ -80,6 +83,8 @@ def _run_blocks(q, blocks, chunk_at, partial_fn, merge_fn):
             o, lse = partial_fn(q, k_c, v_c, kind == DIAGONAL)
             o_parts[s].copy_(o)
             lse_parts[s].copy_(lse)
+        if step_done is not None:
+            step_done(s)
     return merge_fn(o_parts, lse_parts)
 
 
@@ -122,20 +127,13 @@ def ring_attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
         state["reqs"] = reqs
         return cur[0], cur[1]
 
-    B, H, L, d = q.shape
-    o_parts = torch.zeros((world, B, H, L, d), dtype=torch.float32, device=q.device)
-    lse_parts = torch.full((world, B, H, L), float("-inf"), dtype=torch.float32, device=q.device)
-    for s, (c, kind) in enumerate(blocks):
-        k_c, v_c = chunk_at(s)
-        if kind != SKIP:
-            o, lse = partial_fn(q, k_c, v_c, kind == DIAGONAL)
-            o_parts[s].copy_(o)
-            lse_parts[s].copy_(lse)
+    def step_done(s):
         for r in state["reqs"]:
             r.wait()
         if s + 1 < world:
             state["cur"] = state["next"]
-    return merge_fn(o_parts, lse_parts)
+
+    return _run_blocks(q, blocks, chunk_at, partial_fn, merge_fn, step_done)
 
 
 def ring_attention_local(q_chunks, k_chunks, v_chunks, causal: bool = False, scale: Optional[float] = None,
