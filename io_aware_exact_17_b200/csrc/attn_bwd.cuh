@@ -24,9 +24,10 @@
 //    over Sᵀ as bf16 pairs, the TMEM A operands of dV += Pᵀ dO_i and
 //    dK += dSᵀ Q_i, and dSᵀ to shared memory in the 128-byte-swizzle layout,
 //    read MN-major as the A operand of dQ_i = dS K_j;
-//  * dQ_i is issued first and lands in the dP columns. The softmax warps add it
-//    into an fp32 workspace with vector reductions while the tensor core runs
-//    dV, dK and the next Sᵀ; the next dPᵀ waits only for that read-out;
+//  * dQ_i is issued first and lands in the dP columns. The softmax warps read it
+//    out (the next dPᵀ waits only for that), stage it in shared memory and add
+//    it into an fp32 workspace with TMA reduce-adds, 32 x 32 tiles, while the
+//    tensor core runs dV, dK and the next Sᵀ;
 //  * a prologue kernel forms D_i and -LSE in log2 units, padded per head to
 //    whole tiles (-inf and 0, so that padded queries get P = 0). An epilogue
 //    kernel scales dQ and rounds it to bf16.
@@ -75,18 +76,27 @@ struct BwdCfg {
 struct BwdParams {
   __nv_bfloat16* dk;        // [BH][N][D]
   __nv_bfloat16* dv;        // [BH][N][D]
-  float* dq_acc;            // [BH][N][D] fp32, zeroed by the prologue; dQ / scale
   const float* nlse2;       // [BH][Npad]: -LSE * log2(e), -inf past N
   const float* dvec;        // [BH][Npad]: D_i = dO_i · O_i, 0 past N
   int BH, N, Npad, n_t;     // n_t = Npad / 128 tiles per head
   float scale, scale_log2;  // scale, scale * log2(e)
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
+// Element-wise add of a shared-memory tile into global memory through a tensor
+// map (the TMA's reduction; out-of-range elements of the box are not written),
+// tracked by this thread's bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the bulk operations of this thread have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until the bulk operations of this thread have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -116,7 +126,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
@@ -297,30 +307,48 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t row_addr = tbase + (lane_base << 16);
     const uint32_t ds_row = smem_u32(sdS) + g * C::CHUNK + r * 128;
     const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
-    // dQ_i rows (queries on lanes) added into the fp32 accumulator
+    // This warp's 4 KB of the dSᵀ tile (key rows 32 (warp & 3) .., column half g)
+    // doubles as its staging area for dQ: the dQ MMA that read dSᵀ has completed
+    // when dQ is read out, and the warp writes its dSᵀ rows again only after its
+    // staged dQ has been read by the TMA (below).
+    uint8_t* stage_dq = sdS + g * C::CHUNK + (warp & 3u) * 4096;
+    // dQ_i rows (queries on lanes) added into the fp32 accumulator: TMEM ->
+    // registers (then the columns are free for the next dPᵀ) -> shared memory,
+    // 32 rows x 32 columns at a time in the 128-byte-swizzle layout -> one TMA
+    // reduce-add per tile by lane 0 (rows past N are clipped by the map).
     auto dq_out = [&](int i) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, st, 62))) return false;
       tc_fence_after();
-      const int qrow = q_tile(i) * C::BQ + r;
-      float* dqrow = p.dq_acc + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
       constexpr int NC = D / 64;  // 32-column chunks of this warpgroup's D / 2 columns
       uint32_t v[NC][32];
 #pragma unroll
       for (int c = 0; c < NC; ++c) tmem_ld32(row_addr + C::DP_COL + g * (D / 2) + 32 * c, v[c]);
 #pragma unroll
       for (int c = 0; c < NC; ++c) tmem_wait_ld_dep32(v[c]);
-      if (qrow < p.N) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            red_add_v4(dqrow + g * (D / 2) + 32 * c + 4 * u, __uint_as_float(v[c][4 * u]),
-                       __uint_as_float(v[c][4 * u + 1]), __uint_as_float(v[c][4 * u + 2]),
-                       __uint_as_float(v[c][4 * u + 3]));
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_dqfree);
+      const uint32_t row_st = smem_u32(stage_dq) + lane * 128;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        if (c > 0) {
+          if (lane == 0) bulk_wait_read_all();  // the previous tile has left the staging area
+          __syncwarp();
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(row_st + ((static_cast<uint32_t>(u) ^ (lane & 7u)) << 4), v[c][4 * u], v[c][4 * u + 1],
+                       v[c][4 * u + 2], v[c][4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int y = q_tile(i) * C::BQ + static_cast<int>(lane_base);  // first query row of the tile
+        if (lane == 0 && y < p.N) {  // rows past N are padding (and are clipped by the map)
+          tma_reduce_add_3d(&tmdQ, stage_dq, g * (D / 2) + 32 * c, y, bh);
+          bulk_commit();
+        }
+      }
+      if (lane == 0) bulk_wait_read_all();  // before this warp writes its dSᵀ rows again
+      __syncwarp();
       return true;
     };
     bool ok = true;
@@ -451,6 +479,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // the dQ reductions have completed before the CTA exits
   }
 
   tc_fence_before();

@@ -410,11 +410,13 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   float* nlse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                          round256(static_cast<size_t>(BH) * N * D * sizeof(float)));
   float* dvec = nlse2 + round256(static_cast<size_t>(BH) * Npad * sizeof(float)) / sizeof(float);
-  CUtensorMap tmQ, tmK, tmV, tmdO;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmdQ;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!fa::make_tmap_3d(&tmQ, q, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmK, k, bf, 2, D, N, BH, 64, 128) ||
       !fa::make_tmap_3d(&tmV, v, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmdO, dout, bf, 2, D, N, BH, 64, 128))
     return FA_ERR_CUDA;
+  // the fp32 dQ accumulator, reduced into in tiles of 32 rows x 32 columns
+  if (!fa::make_tmap_3d(&tmdQ, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, 32, 32)) return FA_ERR_CUDA;
   const long long rows = static_cast<long long>(BH) * Npad;
   fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH, N,
@@ -426,7 +428,6 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   fa::BwdParams p;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dq_acc = dq_acc;
   p.nlse2 = nlse2;
   p.dvec = dvec;
   p.BH = BH;
@@ -436,7 +437,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, C::SMEM_BYTES, stream>>>(
-      tmQ, tmK, tmV, tmdO, p);
+      tmQ, tmK, tmV, tmdO, tmdQ, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const long long n4 = static_cast<long long>(BH) * N * D / 4;
   const long long cap = static_cast<long long>(device_sms()) * 8;
