@@ -108,11 +108,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (the tensor core reads its shared-memory operands through it).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Bounded wait used only while tearing down after an abort.
 __device__ __forceinline__ void mbar_drain_bwd(uint64_t* bar, uint32_t parity) {
@@ -339,7 +334,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int u = 0; u < 8; ++u)
           st_shared_v4(row_st + ((static_cast<uint32_t>(u) ^ (lane & 7u)) << 4), v[c][4 * u], v[c][4 * u + 1],
                        v[c][4 * u + 2], v[c][4 * u + 3]);
-        fence_proxy_async_smem();
+        fence_proxy_async_shared();
         __syncwarp();
         const int y = q_tile(i) * C::BQ + static_cast<int>(lane_base);  // first query row of the tile
         if (lane == 0 && y < p.N) {  // rows past N are padding (and are clipped by the map)
@@ -444,7 +439,7 @@ __global__ void __launch_bounds__(384, 1)
       tmem_st32(row_addr + C::S_COL + 32 * g, pp);
       tmem_st32(row_addr + C::S_COL + 64 + 32 * g, dsp);
       tmem_wait_st();
-      fence_proxy_async_smem();
+      fence_proxy_async_shared();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p);

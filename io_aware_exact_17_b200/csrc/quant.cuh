@@ -483,6 +483,14 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
       w[4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
     }
   };
+  // The stage is handed back to the producer, whose next TMA write to it goes
+  // through the async proxy: this thread's shared-memory reads of it are
+  // ordered before that write by a proxy fence ahead of the warp's arrival.
+  auto release_stage = [&](int stage) {
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+  };
   bool ok = true;
   float m = 0.f;
   for (int s = 0; s < K; ++s) {
@@ -491,8 +499,7 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
     if (!ok) break;
     uint64_t w[32];
     load_row(stage, w);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
+    release_stage(stage);
     rotate64<D, ROT>(w, p, sg);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -549,8 +556,7 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
     if (!ok) break;
     uint64_t w[32];
     load_row(stage, w);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
+    release_stage(stage);
     rotate64<D, ROT>(w, p, sg);
     const float amax = amax_all[t];
     const float sc = amax > 0.f ? 448.0f / amax : 1.0f;

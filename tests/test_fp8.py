@@ -61,6 +61,28 @@ def test_quant_matches_oracle(d, rotate, rows):
         _quant_check(x, True, inputs.hadamard_signs(d, seed=rows))
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("rotate", [False, True])
+def test_quant_is_repeatable_at_scale(d, rotate):
+    # The quantiser streams every row block through a shared-memory ring twice;
+    # a race between a stage's readers and its refill would show up as codes
+    # that change from launch to launch. 20 launches on 32 M elements must agree
+    # bit for bit (the arithmetic is deterministic), and the first with the oracle.
+    rows = (32 << 20) // d
+    g = torch.Generator().manual_seed(d + 7)
+    x = torch.randn(rows, d, generator=g).to(torch.bfloat16)
+    signs = inputs.hadamard_signs(d, seed=d) if rotate else None
+    codes0, ds0 = _quant_check(x, rotate, signs)
+    xc = x.cuda()
+    sc = signs.cuda() if signs is not None else None
+    first, _ = fa.hadamard_quant(xc, rotate=rotate, signs=sc)
+    for _ in range(20):
+        again, ds = fa.hadamard_quant(xc, rotate=rotate, signs=sc)
+        assert torch.equal(again, first) and float(ds.item()) == ds0
+    assert np.array_equal(first.cpu().numpy().reshape(-1, d), codes0)
+    assert fa.device_status()[0] == 0
+
+
 @pytest.mark.parametrize("n", [1, 2, 3, 8])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_quant_multi_equals_one_call_per_tensor(n, rotate):
