@@ -179,6 +179,36 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 #define FA_QUANT_WORKSPACE_BYTES 256
 
 /*
+ * fa_fwd_fp8_qrot — e4m3 attention forward with Q rotated and quantised inside
+ * the attention kernel: Q is given in bf16, and each 128-row query tile is
+ * rotated and quantised to e4m3 with its own scale in shared memory, right
+ * after it is loaded and before its first Q Kᵀ. K is given as e4m3 codes with
+ * one descale per 128-row block (fa_hadamard_quant_blocks, with the same
+ * rotation). The result is that of fa_fwd with qk_dtype = FA_E4M3_BLOCK on Q
+ * quantised by fa_hadamard_quant_blocks, without the separate pass over Q.
+ *
+ * Defined by: "FlashAttention-3 (PT)", section "Inovações técnicas",
+ * subsection 3 ("Baixa precisão (FP8)"), steps 1-4, with one scale per block of
+ * 128 rows; the attention itself as for fa_fwd.
+ *
+ * q          device, bf16 [B][H][N][d], 16-byte aligned.
+ * k8         device, e4m3 codes [B][H][N][d] (uint8), 16-byte aligned.
+ * v          device, bf16 [B][H][N][d], 16-byte aligned.
+ * o, lse     as fa_fwd (lse may be NULL).
+ * d          128 only (FA_ERR_UNSUPPORTED otherwise).
+ * dk_blocks  device, fp32 [B][H][ceil(N/128)]: K's block descales.
+ * rotate     1: x' = x diag(signs) H_128 / sqrt(128) before quantising (as K was);
+ *            0: quantise only.
+ * signs      device, 128 fp32 values +-1 (16-byte aligned), or NULL for none.
+ * dq_blocks_out  device, fp32 [B][H][ceil(N/128)] receiving each query
+ *            block's descale (amax / 448), or NULL.
+ * Errors: as fa_fwd.
+ */
+fa_status fa_fwd_fp8_qrot(const void* q, const void* k8, const void* v, void* o, float* lse, int B, int H, int N,
+                          int d, int causal, float scale, const float* dk_blocks, int rotate, const float* signs,
+                          float* dq_blocks_out, void* stream);
+
+/*
  * fa_hadamard_quant — rotate (optionally) and quantise one tensor to e4m3 with a
  * single scale.
  *
@@ -286,8 +316,9 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
 
-/* ABI version of this header: 4 (1, plus the split-key, partial and merge calls in 2,
- * plus per-block e4m3 scales in 3, plus the backward pass in 4). */
+/* ABI version of this header: 5 (1, plus the split-key, partial and merge calls in 2,
+ * plus per-block e4m3 scales in 3, plus the backward pass in 4, plus
+ * fa_fwd_fp8_qrot in 5). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -46,14 +46,22 @@ namespace fa {
 #define FA_REG_OTHER 88
 #endif
 
-template <int D, int NQ, bool QK_FP8>
+// QROT: Q arrives in bf16 and each query tile is rotated and quantised to e4m3
+// (one scale per tile) by its softmax warpgroup in shared memory, in place,
+// before its first Q Kᵀ; K is e4m3 with one scale per 128-key tile.
+template <int D, int NQ, bool QK_FP8, bool QROT = false>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per tile (TMEM lanes)
   static constexpr int BN = 128;  // keys per K/V tile
   static constexpr int EQK = QK_FP8 ? 1 : 2;
-  static constexpr int QK_CHUNKS = D * EQK / 128;  // 128-byte swizzle columns per Q/K row
+  static constexpr int QK_CHUNKS = D * EQK / 128;  // 128-byte swizzle columns per Q/K row (MMA operands)
   static constexpr int V_CHUNKS = D * 2 / 128;
-  static constexpr int Q_TILE = BM * D * EQK;
+  // Q as loaded: bf16 under QROT (converted in place: the e4m3 tile is the
+  // first BM * D bytes of the slot), else the MMA's own element type
+  static constexpr int Q_LOAD_CHUNKS = QROT ? D * 2 / 128 : QK_CHUNKS;
+  static constexpr int Q_LOAD_ELEMS = QROT ? 64 : 128 / EQK;  // elements per 128-byte column
+  static constexpr int Q_TILE = BM * D * (QROT ? 2 : EQK);
+  static_assert(!QROT || (QK_FP8 && D == 128), "Q is rotated and quantised in the kernel for e4m3, d = 128");
   static constexpr int K_TILE = BN * D * EQK;
   static constexpr int V_TILE = BN * D * 2;
   static constexpr int SLOT = V_TILE;  // a ring slot holds one K or one V tile
@@ -97,6 +105,12 @@ struct FwdParams {
   const float* dq_block;
   const float* dk_block;
   int nbq, nbk;
+  // QROT: the d Hadamard signs of the rotation (null: none) and whether to
+  // rotate at all; dq_out (may be null) receives each query tile's descale at
+  // dq_out[bh * nbq + query tile]
+  const float* qrot_signs;
+  int qrot_rotate;
+  float* dq_out;
   int BH;                    // batch * heads
   int Nq, Nk;                // query rows and keys per head
   int causal_off;            // Nk - Nq: key j is visible to query i iff j <= i + causal_off (causal)
@@ -230,6 +244,90 @@ __device__ __forceinline__ float row_max_tmem(uint32_t tS, uint32_t* s, int kbas
     }
   }
   return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
+}
+
+// In-kernel rotate-and-quantise of one query tile (QROT). Thread r of the
+// tile's warpgroup owns row r: it reads the row's 128 bf16 values from the
+// tile as the TMA left it (two 64-element columns, 128-byte swizzle), applies
+// the signs and the 7 butterfly stages of H_128 in registers (index bits 0, 1,
+// ... in increasing order with the same operations as the standalone
+// quantisers, so the rotated values are the same bits), then the warpgroup
+// takes the tile's amax through `red` and named barrier `bar_id`; the codes
+// e4m3(x' / sqrt(128) * 448 / amax) go to the row's first 128 bytes in the
+// swizzled K-major layout of an e4m3 operand. Every thread has read its row
+// before the barrier, so the in-place writes (row r's codes over the first
+// half of row r's bf16 values) never meet a read. Rows past the end of the
+// sequence hold zeros (TMA fill) and do not change the amax. Returns the
+// tile's descale amax / 448 (1 when the tile is zero): "FlashAttention-3 (PT)",
+// section "Inovações técnicas", subsection 3, steps 1-3, one scale per block of
+// 128 rows.
+__device__ __forceinline__ float qrot_tile(uint8_t* tile, int r, const float* signs, bool rotate, float* red,
+                                           uint32_t wq, uint32_t lane, uint32_t bar_id) {
+  constexpr float inv_sqrt_d = 0.08838834764831845f;  // 1 / sqrt(128)
+  uint64_t w[64];  // w[i] = elements 2i, 2i+1 of the row
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 u = *reinterpret_cast<const uint4*>(tile + c * (128 * 128) + r * 128 + ((j ^ (r & 7)) << 4));
+      w[32 * c + 4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
+      w[32 * c + 4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+      w[32 * c + 4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
+      w[32 * c + 4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+    }
+  if (rotate) {
+    if (signs != nullptr) {
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(signs + 2 * i));
+        w[i] = f2_mul(w[i], f2_pack(s4.x, s4.y));
+        w[i + 1] = f2_mul(w[i + 1], f2_pack(s4.z, s4.w));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {  // index bit 0: inside each pair
+      float a, b;
+      f2_unpack(w[i], a, b);
+      w[i] = f2_pack(a + b, a - b);
+    }
+#pragma unroll
+    for (int h = 1; h < 64; h <<= 1)  // index bits 1 .. 6: pair i with pair i + h
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if ((i & h) == 0) {
+          const uint64_t a = w[i], b = w[i + h];
+          w[i] = f2_add(a, b);
+          w[i + h] = f2_sub(a, b);
+        }
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    float a, b;
+    f2_unpack(w[i], a, b);
+    m = fmax3(m, fabsf(a), fabsf(b));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[wq] = m;
+  named_barrier_sync(bar_id, 128);
+  float amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  if (rotate) amax *= inv_sqrt_d;  // fp32 rounding is monotonic: max fl(|v| c) = fl(c max |v|)
+  const float sc = amax > 0.f ? 448.0f / amax : 1.0f;
+  const uint64_t sc2 = f2_pack(sc, sc), isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // 16 codes (elements 16j .. 16j+15) per 16-byte chunk
+    uint32_t q[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float a0, b0, a1, b1;
+      f2_unpack(f2_mul(rotate ? f2_mul(w[8 * j + 2 * k], isd) : w[8 * j + 2 * k], sc2), a0, b0);
+      f2_unpack(f2_mul(rotate ? f2_mul(w[8 * j + 2 * k + 1], isd) : w[8 * j + 2 * k + 1], sc2), a1, b1);
+      q[k] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
+    }
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+  }
+  return amax > 0.f ? amax / 448.0f : 1.0f;
 }
 
 // Softmax warps of a DEC CTA (see attn_fwd_kernel): warp w, lane r holds query
@@ -434,12 +532,13 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
 // their maxima and sums (the same combination as for blocks of a split). A thread
 // thus takes 32 exponentials per key tile instead of 128, which shortens the
 // serial softmax -> P V -> S chain that bounds a CTA with one query tile.
-template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC>
-__global__ void __launch_bounds__(FwdCfg<D, NQ, QK_FP8>::THREADS, 1)
+template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC, bool QROT = false>
+__global__ void __launch_bounds__(FwdCfg<D, NQ, QK_FP8, QROT>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D, NQ, QK_FP8>;
+  using C = FwdCfg<D, NQ, QK_FP8, QROT>;
   static_assert(!DEC || NQ == 1, "the decode layout uses one query tile");
+  static_assert(!QROT || (!PARTIAL && !DEC && NQ == 2), "in-kernel Q quantisation: square launches only");
   static_assert(!DEC || C::NSLOT * C::SLOT >= 3 * 32 * D * 4, "decode merge buffer lives in the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -450,6 +549,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // bar_qfree: the S MMAs that read the current item's Q tiles are done (the
   // producer may load the next item's Q)
   __shared__ __align__(8) uint64_t bar_q, bar_qfree, bar_drain, bar_s[NQ], bar_p[NQ], bar_o[NQ];
+  // QROT: query tile t is in e4m3 (its warpgroup has converted it)
+  __shared__ __align__(8) uint64_t bar_qready[NQ];
+  __shared__ float qrot_red[NQ][4];  // per-warp maxima of each tile
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
@@ -504,6 +606,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], 4);  // one arrival per softmax warp of the tile
       mbar_init(&bar_o[t], 1);
+      mbar_init(&bar_qready[t], 4);
     }
     fence_mbar_init();
   }
@@ -542,8 +645,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_3d(sQ + c * (C::BM * 128) + w * 32 * 128, &tmQ, &bar_q, c * (128 / C::EQK), q0, bh);
       } else {
         for (int t = 0; t < NQ; ++t)
-          for (int c = 0; c < C::QK_CHUNKS; ++c)
-            tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * (128 / C::EQK), q0 + t * C::BM,
+          for (int c = 0; c < C::Q_LOAD_CHUNKS; ++c)
+            tma_load_3d(sQ + t * C::Q_TILE + c * (C::BM * 128), &tmQ, &bar_q, c * C::Q_LOAD_ELEMS, q0 + t * C::BM,
                         bh);
       }
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -583,7 +686,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const FwdItem w = item_at(it);
       const int n_kv = w.n_kv;
       auto n_kv_at = [&](int t) { return t == 0 ? w.n_kv0 : w.n_kv1; };
-      ok = mbar_wait(&bar_q, iter & 1, &abort_flag, st, 20);
+      if constexpr (!QROT) ok = mbar_wait(&bar_q, iter & 1, &abort_flag, st, 20);
       for (int j = 0; j <= n_kv && ok; ++j) {
         const int kpos = pos + 2 * j, vpos = pos + 2 * j - 1;
         const int kslot = kpos % C::NSLOT, vslot = (vpos + C::NSLOT) % C::NSLOT;
@@ -611,6 +714,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (j == n_kv_t) mma_commit(&bar_o[t]);
           }
           if (j < n_kv_t) {
+            if constexpr (QROT) {
+              if (j == 0) {  // this tile's Q, converted to e4m3 by its warpgroup
+                ok = mbar_wait(&bar_qready[t], iter & 1, &abort_flag, st, 24 + t);
+                if (!ok) break;
+                tc_fence_after();
+              }
+            }
             // S_t = Q_t K_jᵀ, both K-major, 32 bytes of the reduction dim per MMA.
             const uint32_t kaddr = ring + kslot * C::SLOT;
             const uint32_t qt = qaddr + t * C::Q_TILE;
@@ -665,7 +775,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // key tile, when scales are per block) of the key tile
     float s_q = p.scale_log2;
     const float* dkb = nullptr;
-    if constexpr (QK_FP8) {
+    if constexpr (QROT) {
+      // this warpgroup's Q tile, bf16 from the TMA, to e4m3 in place
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_q, round & 1, &abort_flag, st, 35));
+      if (!ok) break;
+      const float dq = qrot_tile(sQ + t * C::Q_TILE, r, p.qrot_rotate ? p.qrot_signs : nullptr, p.qrot_rotate != 0,
+                                 qrot_red[t], warp & 3u, lane, 2 + t);
+      fence_proxy_async_shared();  // the tensor core reads the codes through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_qready[t]);
+      if (p.dq_out != nullptr && r == 0 && q0 + t * C::BM < p.Nq)
+        p.dq_out[static_cast<size_t>(bh) * p.nbq + (q0 + t * C::BM) / C::BM] = dq;
+      s_q *= dq;
+      dkb = p.dk_block + static_cast<size_t>(bh) * p.nbk + kt0;
+    } else if constexpr (QK_FP8) {
       if (p.dq_block != nullptr) {
         if (q0 + t * C::BM < p.Nq) s_q *= __ldg(p.dq_block + static_cast<size_t>(bh) * p.nbq + (q0 + t * C::BM) / C::BM);
         dkb = p.dk_block + static_cast<size_t>(bh) * p.nbk + kt0;

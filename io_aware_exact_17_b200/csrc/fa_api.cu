@@ -48,6 +48,12 @@ struct FwdArgs {
   fa_dtype qk_dtype;
   const float* descale_qk;
   int n_split;
+  // in-kernel rotate-and-quantise of bf16 Q (fa_fwd_fp8_qrot): descale_qk then
+  // holds the key-block descales only
+  bool qrot = false;
+  int qrot_rotate = 0;
+  const float* qrot_signs = nullptr;
+  float* dq_out = nullptr;
 };
 
 constexpr int kKeyTile = 128;  // keys per K/V tile (FwdCfg::BN)
@@ -72,17 +78,19 @@ constexpr bool kPersistent = FA_PERSISTENT != 0;
 #endif
 constexpr bool kPersistCausal = FA_PERSIST_CAUSAL != 0;
 
-template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC>
+template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC, bool QROT = false>
 fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
-  using C = FwdCfg<D, NQ, QK_FP8>;
+  using C = FwdCfg<D, NQ, QK_FP8, QROT>;
   const int BH = a.B * a.H;
   CUtensorMap tmQ, tmK, tmV;
   const CUtensorMapDataType qk_type = QK_FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!fa::make_tmap_3d(&tmQ, a.q, qk_type, C::EQK, D, a.Nq, BH, 128 / C::EQK, DEC ? kDecodeMaxQ : C::BM) ||
-      !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
+  const bool q_ok = QROT ? fa::make_tmap_3d(&tmQ, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nq, BH, 64, C::BM)
+                         : fa::make_tmap_3d(&tmQ, a.q, qk_type, C::EQK, D, a.Nq, BH, 128 / C::EQK,
+                                            DEC ? kDecodeMaxQ : C::BM);
+  if (!q_ok || !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
       !fa::make_tmap_3d(&tmV, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nk, BH, 64, C::BN))
     return FA_ERR_CUDA;
-  auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8, PARTIAL, DEC>;
+  auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8, PARTIAL, DEC, QROT>;
   static unsigned long long smem_done = 0;
   if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
   if constexpr (C::SPLIT_REGS) {
@@ -109,7 +117,12 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   p.dk_block = nullptr;
   p.nbq = (a.Nq + 127) / 128;
   p.nbk = (a.Nk + 127) / 128;
-  if (a.qk_dtype == FA_E4M3_BLOCK) {
+  p.qrot_signs = a.qrot_signs;
+  p.qrot_rotate = a.qrot_rotate;
+  p.dq_out = a.dq_out;
+  if (QROT) {
+    p.dk_block = a.descale_qk;  // key blocks only: the query blocks' are computed in the kernel
+  } else if (a.qk_dtype == FA_E4M3_BLOCK) {
     // one descale per 128-row block: the query blocks of every head, then the key blocks
     p.dq_block = a.descale_qk;
     p.dk_block = a.descale_qk + static_cast<size_t>(BH) * p.nbq;
@@ -356,6 +369,27 @@ fa_status launch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_
   return FA_OK;
 }
 
+// One scale per 128-row block of a head (quant_block_tma_kernel): one pass,
+// persistent CTAs (one per SM) over the stages of RB rows of each head.
+template <int D>
+fa_status launch_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int rotate,
+                              const float* signs, cudaStream_t stream) {
+  using TC = fa::TmaQuantCfg<D>;
+  auto kernel = rotate ? fa::quant_block_tma_kernel<D, true> : fa::quant_block_tma_kernel<D, false>;
+  static unsigned long long smem_set[2] = {0, 0};
+  if (!set_smem_once(kernel, TC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
+  CUtensorMap tm;
+  if (!fa::make_tmap_3d(&tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(N),
+                        static_cast<uint64_t>(BH), 64, TC::BOX_ROWS))
+    return FA_ERR_CUDA;
+  const long long units = static_cast<long long>(BH) * ((N + TC::RB - 1) / TC::RB);
+  long long grid = device_sms();
+  if (grid > units) grid = units;
+  kernel<<<static_cast<unsigned>(grid), TC::THREADS, TC::SMEM, stream>>>(tm, static_cast<uint8_t*>(out), BH, N,
+                                                                          signs, descales);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status dispatch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int d, int rotate,
                                const float* signs, unsigned int* ws, cudaStream_t s) {
   switch (d) {
@@ -458,6 +492,27 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
   FwdArgs a{q, k, v, o, lse, nullptr, nullptr, B, H, N, N, d, causal != 0, scale, qk_dtype, descale_qk, 1};
   return dispatch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_fp8_qrot(const void* q, const void* k8, const void* v, void* o, float* lse, int B, int H, int N,
+                          int d, int causal, float scale, const float* dk_blocks, int rotate, const float* signs,
+                          float* dq_blocks_out, void* stream) {
+  const fa_status chk = check_fwd_args(q, k8, v, B, H, N, N, d, causal, scale, FA_E4M3_BLOCK, dk_blocks, 1);
+  if (chk != FA_OK) return chk;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (o == nullptr || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (!aligned(o, 16)) return FA_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return FA_ERR_ALIGNMENT;
+  if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
+  if (dq_blocks_out != nullptr && !aligned(dq_blocks_out, 4)) return FA_ERR_ALIGNMENT;
+  FwdArgs a{q, k8, v, o, lse, nullptr, nullptr, B, H, N, N, d, causal != 0, scale, FA_E4M3_BLOCK, dk_blocks, 1};
+  a.qrot = true;
+  a.qrot_rotate = rotate;
+  a.qrot_signs = rotate ? signs : nullptr;
+  a.dq_out = dq_blocks_out;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, 2, true, true, false, false, true>(a, s)
+                : launch_fwd<128, 2, false, true, false, false, true>(a, s);
 }
 
 int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d) {
@@ -606,31 +661,17 @@ fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, in
   if (x == nullptr || out == nullptr || descales == nullptr) return FA_ERR_INVALID_ARG;
   if (BH < 1 || N < 1 || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  const long long nb = (static_cast<long long>(N) + fa::kBlockRows - 1) / fa::kBlockRows;
+  const long long nb = (static_cast<long long>(N) + 127) / 128;  // 128-row scale blocks per head
   if (nb * BH > 0x7fffffffLL || static_cast<long long>(BH) * N > (1LL << 40)) return FA_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(out, 16) || !aligned(descales, 4)) return FA_ERR_ALIGNMENT;
   if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
   const float* sg = rotate ? signs : nullptr;
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  uint8_t* ob = static_cast<uint8_t*>(out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned grid = static_cast<unsigned>(nb * BH);
-  const int nbi = static_cast<int>(nb);
   switch (d) {
-    case 64:
-      if (rotate) fa::quant_block_kernel<64, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
-      else fa::quant_block_kernel<64, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
-      break;
-    case 128:
-      if (rotate) fa::quant_block_kernel<128, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
-      else fa::quant_block_kernel<128, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
-      break;
-    default:
-      if (rotate) fa::quant_block_kernel<256, true><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, sg, descales);
-      else fa::quant_block_kernel<256, false><<<grid, fa::kBlockThreads, 0, s>>>(xb, ob, N, nbi, nullptr, descales);
-      break;
+    case 64: return launch_quant_blocks<64>(x, out, descales, BH, N, rotate, sg, s);
+    case 128: return launch_quant_blocks<128>(x, out, descales, BH, N, rotate, sg, s);
+    default: return launch_quant_blocks<256>(x, out, descales, BH, N, rotate, sg, s);
   }
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"
@@ -728,7 +769,7 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
   return FA_OK;
 }
 
-int fa_abi_version(void) { return 4; }
+int fa_abi_version(void) { return 5; }
 
 #ifdef FA_TEST_HOOKS
 // Test build only (not declared in include/, not in the product library): arm

@@ -18,8 +18,8 @@
 // cooperative launch, for up to 8 tensors at once (each with its own scale),
 // with the input staged through shared memory by TMA; quant_amax_kernel +
 // quant_apply_kernel are the two-launch form (used where the scratch is the
-// library's own static array). quant_block_kernel (end of the file) takes one
-// scale per 128-row block of a head, in one pass.
+// library's own static array). quant_block_tma_kernel (end of the file) takes
+// one scale per 128-row block of a head, in one pass.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -172,120 +172,6 @@ quant_apply_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
 
 namespace fa {
 
-// ---------------------------------------------------------------------------
-// 32 elements per thread (four interleaved 16-byte chunks of a row), for the
-// per-block kernel. The butterfly stages run in the same order (index bits 0,
-// 1, 2, ...) with the same operands as hadamard_rotate, so the codes are
-// bit-identical to the two-kernel path.
-// ---------------------------------------------------------------------------
-template <int D>
-struct FusedCfg {
-  static constexpr int E = 32;          // elements per thread (four 16-byte chunks)
-  static constexpr int L = D / E;       // threads per row
-  static constexpr int RPW = 32 / L;    // rows per warp per step
-  static_assert(D == 64 || D == 128 || D == 256, "head dim");
-};
-
-// Thread lr of a row holds the four 16-byte chunks lr, lr+L, lr+2L, lr+3L (8
-// elements each) of the row: v[8*q + i] is element 8*(lr + L*q) + i. A warp's
-// load instruction q then covers L consecutive chunks of each of its rows.
-template <int D>
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* row, int lr, float (&v)[32]) {
-  constexpr int L = D / 32;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + lr + L * q);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
-      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-}
-
-// In place: (v * signs) H_D / sqrt(D) for the elements this thread holds (the
-// layout of load_bf16x32). Butterflies run over index bits 0, 1, 2 (inside a
-// chunk), then the log2(L) bits of the chunk's lane (warp shuffles), then the two
-// bits of q (inside the thread): the same stage order as hadamard_rotate.
-// Every lane of the warp must call.
-template <int D>
-__device__ __forceinline__ void hadamard_rotate32(float (&v)[32], int lr, const float* signs) {
-  constexpr int L = D / 32;
-  // Stages over index bits 1 and up pair neighbouring elements (v[2i], v[2i+1])
-  // with another such pair, so they run as packed f32x2 operations: the same
-  // two IEEE additions (or subtractions, multiplications) per instruction, hence
-  // the same results as the scalar form.
-  uint64_t w[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = f2_pack(v[2 * i], v[2 * i + 1]);
-  if (signs != nullptr) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q)));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(signs + 8 * (lr + L * q) + 4));
-      w[4 * q + 0] = f2_mul(w[4 * q + 0], f2_pack(s0.x, s0.y));
-      w[4 * q + 1] = f2_mul(w[4 * q + 1], f2_pack(s0.z, s0.w));
-      w[4 * q + 2] = f2_mul(w[4 * q + 2], f2_pack(s1.x, s1.y));
-      w[4 * q + 3] = f2_mul(w[4 * q + 3], f2_pack(s1.z, s1.w));
-    }
-  }
-  // index bit 0: inside each pair (scalar)
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float a, b;
-    f2_unpack(w[i], a, b);
-    w[i] = f2_pack(a + b, a - b);
-  }
-  // index bits 1, 2: pair i with pair i + h/2 inside each 8-element chunk
-#pragma unroll
-  for (int h = 1; h < 4; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((i & h) == 0) {
-        const uint64_t a = w[i], b = w[i + h];
-        w[i] = f2_add(a, b);
-        w[i + h] = f2_sub(a, b);
-      }
-    }
-  }
-  // index bits 3 .. 2+log2(L): across the L lanes of the row. Lower lane:
-  // v + other; upper lane: other - v; both as one fma with +-1 (exact: the same
-  // single rounding as the add or subtract).
-#pragma unroll
-  for (int m = 1; m < L; m <<= 1) {
-    const float sg = (lr & m) != 0 ? -1.0f : 1.0f;
-    const uint64_t sgn = f2_pack(sg, sg);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float a, b;
-      f2_unpack(w[i], a, b);
-      const float oa = __shfl_xor_sync(0xffffffffu, a, m);
-      const float ob = __shfl_xor_sync(0xffffffffu, b, m);
-      w[i] = f2_fma(w[i], sgn, f2_pack(oa, ob));
-    }
-  }
-  // the two bits of q: pair i with pair i + 4 and i + 8
-#pragma unroll
-  for (int h = 4; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((i & h) == 0) {
-        const uint64_t a = w[i], b = w[i + h];
-        w[i] = f2_add(a, b);
-        w[i + h] = f2_sub(a, b);
-      }
-    }
-  }
-  constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
-  const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    w[i] = f2_mul(w[i], isd);
-    f2_unpack(w[i], v[2 * i], v[2 * i + 1]);
-  }
-}
-
 // Up to kQuantBatch tensors of one shape, rotated and quantised in one launch,
 // each with its own scale.
 constexpr int kQuantBatch = 8;
@@ -311,8 +197,8 @@ struct QuantBatch {
 // consumers wait at the barrier.
 //
 // The butterflies run over index bits 0, 1, ... in increasing order with the
-// same operations as hadamard_rotate and hadamard_rotate32, so the codes are
-// bit-identical to the two-launch kernels'. Pass 1 takes the max before the
+// same operations as hadamard_rotate, so the codes are bit-identical to the
+// two-launch kernels'. Pass 1 takes the max before the
 // 1/sqrt(d) factor and multiplies it once: fp32 rounding is monotonic, so
 // max_i fl(|v_i| c) = fl(c max_i |v_i|).
 // ---------------------------------------------------------------------------
@@ -396,8 +282,68 @@ __device__ __forceinline__ void rotate64(uint64_t (&w)[32], int p, const float* 
   }
 }
 
+// Consumer side shared by the TMA-staged quantisers: the thread's row within a
+// stage and its 64-element part of the row, and the reads of that part.
+// Lane bits 0-2: row (low bits), bits 3 .. 2+log2(TPR): the row's part p,
+// higher bits: row (high bits). The 8 lanes of a shared-memory phase (one
+// 16-byte load each) then read the same chunk j of 8 consecutive rows, whose
+// swizzled positions j ^ (row & 7) are 8 different bank groups.
+template <int D>
+struct TmaQuantLane {
+  using C = TmaQuantCfg<D>;
+  static constexpr int LT = C::TPR == 1 ? 0 : (C::TPR == 2 ? 1 : 2);  // log2(TPR)
+  int p, rr;
+  __device__ __forceinline__ TmaQuantLane(int warp, int lane)
+      : p((lane >> 3) & (C::TPR - 1)), rr(warp * (32 / C::TPR) + (lane & 7) + 8 * (lane >> (3 + LT))) {}
+  __device__ __forceinline__ void load(const uint8_t* stage_base, uint64_t (&w)[32]) const {
+    const uint8_t* base = stage_base + p * (C::RB * 128) + rr * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (rr & 7)) << 4));
+      w[4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
+      w[4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+      w[4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
+      w[4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+    }
+  }
+};
+
+// max |v| over the thread's 64 values
+__device__ __forceinline__ float absmax64(const uint64_t (&w)[32]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float a, b;
+    f2_unpack(w[i], a, b);
+    m = fmax3(m, fabsf(a), fabsf(b));
+  }
+  return m;
+}
+
+// Codes of the thread's 64 values: e4m3(v [/ sqrt(D)] * sc), stored to dst
+// (64 bytes, 16-byte aligned).
+template <int D, bool ROT>
+__device__ __forceinline__ void store_codes64(const uint64_t (&w)[32], float sc, uint8_t* dst) {
+  constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
+  const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d), sc2 = f2_pack(sc, sc);
+  uint32_t q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float a0, b0, a1, b1;
+    f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i], isd) : w[2 * i], sc2), a0, b0);
+    f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i + 1], isd) : w[2 * i + 1], sc2), a1, b1);
+    q[i] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+}
+
 // ws[0 .. n-1]: amax bits of each tensor, ws[n]: arrival counter of the grid
-// barrier; all zero at launch. descale_out[t]: tensor t's descale.
+// barrier (one round per tensor); all zero at launch. descale_out[t]: tensor
+// t's descale. The tensors are taken one after the other (pass 1, barrier,
+// pass 2 of tensor 0, then of tensor 1, ...), so that pass 2 re-reads a tensor
+// while it is still in L2 even when all of them together are larger.
 template <int D, bool ROT>
 __global__ void __launch_bounds__(TmaQuantCfg<D>::THREADS, 1)
 quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __restrict__ signs, unsigned int* ws,
@@ -408,24 +354,24 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full[kTmaQuantStages], empty[kTmaQuantStages];
   __shared__ __align__(16) float sgn[D];
-  __shared__ unsigned int amax_cta[kQuantBatch];
-  __shared__ float amax_all[kQuantBatch];
+  __shared__ unsigned int amax_cta;
+  __shared__ float amax_t;
   __shared__ volatile int abort_flag;
   DevStatus* st = &g_fa_status;
   const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
   const int nblk = (rows + C::RB - 1) / C::RB;  // row blocks per tensor
   const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const int per = c < nblk ? (nblk - 1 - c) / G + 1 : 0;  // this CTA's blocks per tensor
-  const int K = per * qm.n;                               // this CTA's steps per pass
-  // Step k of pass 1: tensor k / per, row block c + (k % per) * G. Pass 2 takes
-  // the same steps in reverse; stream position s = 0 .. 2K-1 covers both.
+  // Stream position s = 2 per t + i: tensor t, pass 1 for i < per (block
+  // c + i G), pass 2 for i >= per (the same blocks in reverse).
+  auto block_of = [&](int i) { return c + (i < per ? i : 2 * per - 1 - i) * G; };
   if (tid == 0) {
     abort_flag = 0;
     for (int i = 0; i < kTmaQuantStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::CONSUMER_WARPS);
     }
-    for (int t = 0; t < kQuantBatch; ++t) amax_cta[t] = 0u;
+    amax_cta = 0u;
     fence_mbar_init();
   }
   if (ROT && tid < D) sgn[tid] = signs != nullptr ? signs[tid] : 1.0f;
@@ -437,9 +383,8 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
       for (int t = 0; t < qm.n; ++t) tma_prefetch_desc(&qm.x[t]);
       bool ok = true;
       int s = 0;
-      for (; s < 2 * K && ok; ++s) {
-        const int k = s < K ? s : 2 * K - 1 - s;
-        const int t = k / per, b = c + (k % per) * G;
+      for (; s < 2 * per * qm.n && ok; ++s) {
+        const int t = s / (2 * per), b = block_of(s % (2 * per));
         const int stage = s % kTmaQuantStages, round = s / kTmaQuantStages;
         if (round > 0) ok = mbar_wait(&empty[stage], (round - 1) & 1, &abort_flag, st, 61);
         if (!ok) break;
@@ -463,26 +408,8 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
   }
 
   // -------------------------------------------------------------- consumers --
-  // Lane bits 0-2: row (low bits), bits 3 .. 2+log2(TPR): the row's 64-element
-  // part p, higher bits: row (high bits). The 8 lanes of a shared-memory phase
-  // (one 16-byte load each) then read the same chunk j of 8 consecutive rows,
-  // whose swizzled positions j ^ (row & 7) are 8 different bank groups.
-  constexpr int LT = C::TPR == 1 ? 0 : (C::TPR == 2 ? 1 : 2);  // log2(TPR)
-  const int p = (lane >> 3) & (C::TPR - 1);
-  const int rr = warp * (32 / C::TPR) + (lane & 7) + 8 * (lane >> (3 + LT));  // row within the block
-  const uint8_t* my_col = smem + p * (C::RB * 128) + rr * 128;
+  const TmaQuantLane<D> ln(warp, lane);
   const float* sg = (ROT && signs != nullptr) ? sgn : nullptr;
-  auto load_row = [&](int stage, uint64_t (&w)[32]) {
-    const uint8_t* base = my_col + stage * C::STAGE;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (rr & 7)) << 4));
-      w[4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
-      w[4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-      w[4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
-      w[4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
-    }
-  };
   // The stage is handed back to the producer, whose next TMA write to it goes
   // through the async proxy: this thread's shared-memory reads of it are
   // ordered before that write by a proxy fence ahead of the warp's arrival.
@@ -492,88 +419,174 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
     if (lane == 0) mbar_arrive(&empty[stage]);
   };
   bool ok = true;
-  float m = 0.f;
-  for (int s = 0; s < K; ++s) {
-    const int stage = s % kTmaQuantStages;
-    ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 62));
-    if (!ok) break;
-    uint64_t w[32];
-    load_row(stage, w);
-    release_stage(stage);
-    rotate64<D, ROT>(w, p, sg);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float a, b;
-      f2_unpack(w[i], a, b);
-      m = fmax3(m, fabsf(a), fabsf(b));
+  int s = 0;
+  for (int t = 0; t < qm.n; ++t) {
+    // pass 1: amax of the rotated tensor
+    float m = 0.f;
+    for (int i = 0; i < per && ok; ++i, ++s) {
+      const int stage = s % kTmaQuantStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 62));
+      if (!ok) break;
+      uint64_t w[32];
+      ln.load(smem + stage * C::STAGE, w);
+      release_stage(stage);
+      rotate64<D, ROT>(w, ln.p, sg);
+      m = fmaxf(m, absmax64(w));
     }
-    if (s % per == per - 1) {  // last block of tensor s / per
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) atomicMax(&amax_cta[s / per], __float_as_uint(m));
-      m = 0.f;
-    }
-  }
-  named_barrier_sync(1, kTmaQuantConsumers);
-  if (tid == 0) {
-    for (int t = 0; t < qm.n; ++t) {
-      const float cm = __uint_as_float(amax_cta[t]);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) atomicMax(&amax_cta, __float_as_uint(m));
+    named_barrier_sync(1, kTmaQuantConsumers);
+    if (tid == 0) {
+      const float cm = __uint_as_float(amax_cta);
+      amax_cta = 0u;  // for the next tensor (every consumer has passed its atomicMax)
       atomicMax(&ws[t], __float_as_uint(ROT ? cm * inv_sqrt_d : cm));
-    }
-    // Grid-wide barrier: every CTA is resident (cooperative launch). The wait
-    // is bounded; if it runs out the status word records it and the CTA goes on.
-    __threadfence();
-    atomicAdd(&ws[qm.n], 1u);
-    const unsigned long long t0 = globaltimer_ns();
-    unsigned int arrived;
-    for (;;) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + qm.n) : "memory");
-      if (arrived >= gridDim.x) break;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        if (atomicCAS(&st->code, 0u, 5u) == 0u) {
-          st->site = 60;
-          st->block = blockIdx.x;
+      // Grid-wide barrier, round t: every CTA is resident (cooperative launch).
+      // The wait is bounded; if it runs out the status word records it and the
+      // CTA goes on.
+      __threadfence();
+      atomicAdd(&ws[qm.n], 1u);
+      const unsigned int target = static_cast<unsigned int>(G) * static_cast<unsigned int>(t + 1);
+      const unsigned long long t0 = globaltimer_ns();
+      unsigned int arrived;
+      for (;;) {
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(arrived) : "l"(ws + qm.n) : "memory");
+        if (arrived >= target) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          if (atomicCAS(&st->code, 0u, 5u) == 0u) {
+            st->site = 60;
+            st->block = blockIdx.x;
+          }
+          break;
         }
-        break;
+        __nanosleep(64);
       }
-      __nanosleep(64);
-    }
-    for (int t = 0; t < qm.n; ++t) {
       unsigned int a;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(ws + t) : "memory");
-      amax_all[t] = __uint_as_float(a);
+      amax_t = __uint_as_float(a);
       if (blockIdx.x == 0) descale_out[t] = __uint_as_float(a) > 0.f ? __uint_as_float(a) / 448.0f : 1.0f;
     }
-  }
-  named_barrier_sync(1, kTmaQuantConsumers);
-  if (!ok) return;
-  const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
-  for (int s = K; s < 2 * K; ++s) {
-    const int k = 2 * K - 1 - s;
-    const int t = k / per, b = c + (k % per) * G;
-    const int stage = s % kTmaQuantStages;
-    ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 63));
-    if (!ok) break;
-    uint64_t w[32];
-    load_row(stage, w);
-    release_stage(stage);
-    rotate64<D, ROT>(w, p, sg);
-    const float amax = amax_all[t];
+    named_barrier_sync(1, kTmaQuantConsumers);
+    const float amax = amax_t;
     const float sc = amax > 0.f ? 448.0f / amax : 1.0f;
-    const uint64_t sc2 = f2_pack(sc, sc);
-    uint32_t q[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float a0, b0, a1, b1;
-      f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i], isd) : w[2 * i], sc2), a0, b0);
-      f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i + 1], isd) : w[2 * i + 1], sc2), a1, b1);
-      q[i] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
+    // pass 2: the codes, the same blocks in reverse order
+    for (int i = per; i < 2 * per && ok; ++i, ++s) {
+      const int stage = s % kTmaQuantStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 63));
+      if (!ok) break;
+      uint64_t w[32];
+      ln.load(smem + stage * C::STAGE, w);
+      release_stage(stage);
+      rotate64<D, ROT>(w, ln.p, sg);
+      const int row = block_of(i) * C::RB + ln.rr;
+      if (row < rows) store_codes64<D, ROT>(w, sc, qm.out[t] + static_cast<int64_t>(row) * D + 64 * ln.p);
     }
-    const int row = b * C::RB + rr;
-    if (row < rows) {
-      uint4* dst = reinterpret_cast<uint4*>(qm.out[t] + static_cast<int64_t>(row) * D + 64 * p);
+    // amax_t is read again only after the next round's first named barrier
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-block scales, staged by TMA (quant_block_tma_kernel): one pass, no grid
+// barrier, since every scale depends on one block of 128 rows of one head. The
+// stages are RB rows of one head (2-D tiles of a [BH][N][D] map, rows past N
+// zero-filled); the 128 * TPR threads of each 128-row block reduce its amax
+// through shared memory and a named barrier of their own, then write its codes
+// and descale. Same rotation and rounding as quant_tma_kernel.
+// ---------------------------------------------------------------------------
+template <int D, bool ROT>
+__global__ void __launch_bounds__(TmaQuantCfg<D>::THREADS, 1)
+quant_block_tma_kernel(const __grid_constant__ CUtensorMap tmx, uint8_t* __restrict__ out, int BH, int N,
+                       const float* __restrict__ signs, float* __restrict__ descales) {
+  using C = TmaQuantCfg<D>;
+  constexpr int BLK = 128;                         // rows per scale block
+  constexpr int NBPS = C::RB / BLK;                // blocks per stage
+  constexpr int WPB = C::CONSUMER_WARPS / NBPS;    // warps per block
+  static_assert(C::RB % BLK == 0, "stage rows");
+  constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kTmaQuantStages], empty[kTmaQuantStages];
+  __shared__ __align__(16) float sgn[D];
+  __shared__ float red[2][C::CONSUMER_WARPS];  // per-warp maxima, double-buffered by step
+  __shared__ volatile int abort_flag;
+  DevStatus* st = &g_fa_status;
+  const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
+  const int nsph = (N + C::RB - 1) / C::RB;  // stages per head
+  const int nb = (N + BLK - 1) / BLK;         // scale blocks per head
+  const long long units = static_cast<long long>(BH) * nsph;
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int K = c < units ? static_cast<int>((units - 1 - c) / G + 1) : 0;  // this CTA's stages
+  // step i: unit u = c + i G, head u / nsph, stage u % nsph
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < kTmaQuantStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], C::CONSUMER_WARPS);
+    }
+    fence_mbar_init();
+  }
+  if (ROT && tid < D) sgn[tid] = signs != nullptr ? signs[tid] : 1.0f;
+  __syncthreads();
+
+  if (warp == C::CONSUMER_WARPS) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmx);
+      bool ok = true;
+      int i = 0;
+      for (; i < K && ok; ++i) {
+        const long long u = c + static_cast<long long>(i) * G;
+        const int bh = static_cast<int>(u / nsph), sr = static_cast<int>(u % nsph) * C::RB;
+        const int stage = i % kTmaQuantStages, round = i / kTmaQuantStages;
+        if (round > 0) ok = mbar_wait(&empty[stage], (round - 1) & 1, &abort_flag, st, 64);
+        if (!ok) break;
+        uint8_t* dst = smem + stage * C::STAGE;
+        mbar_arrive_expect_tx(&full[stage], C::STAGE);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+        for (int col = 0; col < C::COLS; ++col)
+#pragma unroll
+          for (int r0 = 0; r0 < C::RB; r0 += C::BOX_ROWS)
+            tma_load_3d(dst + col * (C::RB * 128) + r0 * 128, &tmx, &full[stage], col * 64, sr + r0, bh);
+      }
+      for (int q = i - kTmaQuantStages; q < i; ++q)
+        if (q >= 0) {
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[q % kTmaQuantStages], (q / kTmaQuantStages) & 1))
+            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+    }
+    return;
+  }
+
+  const TmaQuantLane<D> ln(warp, lane);
+  const float* sg = (ROT && signs != nullptr) ? sgn : nullptr;
+  const int blk = ln.rr / BLK;  // this thread's block within a stage
+  for (int i = 0; i < K; ++i) {
+    const int stage = i % kTmaQuantStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], (i / kTmaQuantStages) & 1, &abort_flag, st, 65))) break;
+    uint64_t w[32];
+    ln.load(smem + stage * C::STAGE, w);
+    fence_proxy_async_shared();  // reads ordered before the producer's next TMA write of the stage
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    rotate64<D, ROT>(w, ln.p, sg);
+    float m = absmax64(w);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[i & 1][warp] = m;
+    named_barrier_sync(2 + blk, WPB * 32);
+    float amax = red[i & 1][blk * WPB];
+#pragma unroll
+    for (int k = 1; k < WPB; ++k) amax = fmaxf(amax, red[i & 1][blk * WPB + k]);
+    if (ROT) amax *= inv_sqrt_d;
+    const long long u = c + static_cast<long long>(i) * G;
+    const int bh = static_cast<int>(u / nsph), r0 = static_cast<int>(u % nsph) * C::RB + blk * BLK;
+    if (r0 < N) {  // a block with rows in this head
+      if (ln.rr % BLK == 0 && ln.p == 0) descales[static_cast<long long>(bh) * nb + r0 / BLK] =
+          amax > 0.f ? amax / 448.0f : 1.0f;
+      const int row = r0 + ln.rr % BLK;
+      if (row < N)
+        store_codes64<D, ROT>(w, amax > 0.f ? 448.0f / amax : 1.0f,
+                              out + (static_cast<long long>(bh) * N + row) * D + 64 * ln.p);
     }
   }
 }
@@ -581,72 +594,5 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
 }  // namespace fa
 
 namespace fa {
-
-// ---------------------------------------------------------------------------
-// Per-block scales: one CTA per block of 128 consecutive rows of a head. The
-// block's rotated values stay in registers between its amax and its codes, so
-// the input is read once, with no second pass and no grid-wide barrier (every
-// scale depends on one CTA's data only). The rotation is hadamard_rotate32's.
-// ---------------------------------------------------------------------------
-constexpr int kBlockRows = 128;
-constexpr int kBlockThreads = 256;
-
-template <int D, bool ROT>
-__global__ void __launch_bounds__(kBlockThreads)
-quant_block_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ out, int N, int nb,
-                   const float* __restrict__ signs, float* __restrict__ descales) {
-  using C = FusedCfg<D>;
-  constexpr int WARPS = kBlockThreads / 32;
-  constexpr int STEPS = kBlockRows / (WARPS * C::RPW);  // rows of a warp / rows per warp-step
-  static_assert(STEPS * WARPS * C::RPW == kBlockRows, "block rows");
-  const int bh = blockIdx.x / nb, blk = blockIdx.x % nb;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lr = lane % C::L, sub = lane / C::L;
-  const int row0 = blk * kBlockRows;
-  const __nv_bfloat16* xh = x + static_cast<int64_t>(bh) * N * D;
-  uint8_t* oh = out + static_cast<int64_t>(bh) * N * D;
-  float v[STEPS][32];
-  float m = 0.f;
-#pragma unroll
-  for (int s = 0; s < STEPS; ++s) {
-    const int row = row0 + (s * WARPS + warp) * C::RPW + sub;
-    if (row < N) {
-      load_bf16x32<D>(xh + static_cast<int64_t>(row) * D, lr, v[s]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[s][e] = 0.f;
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < STEPS; ++s) {
-    if (ROT) hadamard_rotate32<D>(v[s], lr, signs);
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) m = fmax3(m, fabsf(v[s][e]), fabsf(v[s][e + 1]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float warp_max[WARPS];
-  if (lane == 0) warp_max[warp] = m;
-  __syncthreads();
-  float amax = warp_max[0];
-#pragma unroll
-  for (int i = 1; i < WARPS; ++i) amax = fmaxf(amax, warp_max[i]);
-  const float scale = amax > 0.f ? 448.0f / amax : 1.0f;
-  if (threadIdx.x == 0) descales[blockIdx.x] = amax > 0.f ? amax / 448.0f : 1.0f;
-#pragma unroll
-  for (int s = 0; s < STEPS; ++s) {
-    const int row = row0 + (s * WARPS + warp) * C::RPW + sub;
-    uint32_t q[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      q[i] = static_cast<uint32_t>(pack_e4m3x2(v[s][4 * i] * scale, v[s][4 * i + 1] * scale)) |
-             (static_cast<uint32_t>(pack_e4m3x2(v[s][4 * i + 2] * scale, v[s][4 * i + 3] * scale)) << 16);
-    if (row < N) {
-      uint2* dst = reinterpret_cast<uint2*>(oh + static_cast<int64_t>(row) * D);
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) dst[lr + C::L * qq] = make_uint2(q[2 * qq], q[2 * qq + 1]);
-    }
-  }
-}
 
 }  // namespace fa

@@ -30,8 +30,8 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
     assert {"fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_splits", "fa_fwd_partial",
             "fa_lse_merge"} <= set(names)
-    assert {"fa_bwd", "fa_bwd_workspace_bytes"} <= set(names)
-    assert lib.fa_abi_version() == 4
+    assert {"fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8_qrot"} <= set(names)
+    assert lib.fa_abi_version() == 5
 
 
 def test_status_strings(lib):
