@@ -13,14 +13,17 @@ as CUDA-graph replays of its own calls with L2 flushed between replays:
   * ``seq_sweep_h16d128``: BF16 forward for N in 512..16384 with B*N = 16384;
   * ``dsweep_b2n4096_causal``: BF16 causal forward for d in 64, 128, 256;
   * ``fp8_b2h16n8192d128``: Hadamard rotate + e4m3 quantise of Q and K (one
-    launch; per tensor and per 128-row block) and the e4m3 attention;
+    launch; per tensor and per 128-row block) and the e4m3 attention, and the
+    step with Q rotated and quantised inside the attention kernel;
   * ``bwd_b4h16n2048d128``: the backward pass, non-causal and causal;
   * ``decode_b4h16nq1nk32768d128``: one query per head over 32768 keys.
 ``--no-extras`` skips them.
 
-``--workload bwd`` and ``--workload decode`` print a line of their own for the
-backward pass (10*B*H*N^2*d FLOPs, halved when causal, on B=4, H=16, N=2048,
-d=128) and for the decode problem (GB/s of algorithmic HBM bytes).
+``--workload bwd``, ``--workload decode`` and ``--workload fp8`` print a line of
+their own for the backward pass (10*B*H*N^2*d FLOPs, halved when causal, on
+B=4, H=16, N=2048, d=128), the decode problem (GB/s of algorithmic HBM bytes)
+and the FP8 step (rotate + quantise Q and K, then the e4m3-QK attention, on
+B=2, H=16, N=8192, d=128).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only), on a bounded
 row sample of the same workload per step.
@@ -450,6 +453,73 @@ class BwdStep:
         return sum(t.numel() * t.element_size() for t in self.host_out)
 
 
+class Fp8Step:
+    """The FP8 workload (B=2, H=16, N=8192, d=128): one launch rotating and
+    quantising Q and K with a scale each (Hadamard signs drawn by the input
+    generator), then the e4m3-QK attention, non-causal."""
+
+    def __init__(self, seed: int):
+        import io_aware_exact_17_b200 as fa
+
+        self.fa = fa
+        f = FP8_CFG
+        self.shape = (f["B"], f["H"], f["N"], f["d"])
+        q, k, v = fa_inputs.qkv_normal(*self.shape, seed)
+        self.signs = fa_inputs.hadamard_signs(f["d"], seed).cuda()
+        self.q_h, self.k_h, self.v_h = (t.pin_memory() for t in (q, k, v))
+        self.bufs = []
+        for _ in range(2):
+            self.bufs.append({
+                "q": q.cuda(), "k": k.cuda(), "v": v.cuda(),
+                "q8": torch.empty(self.shape, dtype=torch.uint8, device="cuda"),
+                "k8": torch.empty(self.shape, dtype=torch.uint8, device="cuda"),
+                "desc": torch.empty(2, dtype=torch.float32, device="cuda"),
+                "o": torch.empty(self.shape, dtype=torch.bfloat16, device="cuda"),
+                "lse": torch.empty(self.shape[:3], dtype=torch.float32, device="cuda"),
+            })
+        self.o_h = torch.empty(self.shape, dtype=torch.bfloat16).pin_memory()
+        self.lse_h = torch.empty(self.shape[:3], dtype=torch.float32).pin_memory()
+        self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 2
+        self.groups = 2  # breakdown: rotate + quantise Q, K; attention
+        self.flops = attn_flops(*self.shape, False)
+
+    def flush_l2(self):
+        self.flush_buf.zero_()
+
+    def run(self, ev=None, b=0):
+        s = self.bufs[b]
+        if ev is not None:
+            ev[0].record()
+        self.fa.hadamard_quant_multi([s["q"], s["k"]], rotate=True, signs=self.signs, outs=[s["q8"], s["k8"]],
+                                     descales=s["desc"])
+        if ev is not None:
+            ev[1].record()
+        self.fa.fwd(s["q8"], s["k8"], s["v"], causal=False, qk_descale=s["desc"], out=s["o"], lse=s["lse"],
+                    n_split=1)
+        if ev is not None:
+            ev[2].record()
+
+    def h2d(self, b):
+        for n_, h_ in (("q", self.q_h), ("k", self.k_h), ("v", self.v_h)):
+            self.bufs[b][n_].copy_(h_, non_blocking=True)
+
+    def compute(self, b):
+        self.run(b=b)
+
+    def d2h(self, b):
+        self.o_h.copy_(self.bufs[b]["o"], non_blocking=True)
+        self.lse_h.copy_(self.bufs[b]["lse"], non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.q_h, self.k_h, self.v_h))
+
+    @property
+    def d2h_bytes(self):
+        return self.o_h.numel() * 2 + self.lse_h.numel() * 4
+
+
 def flops_bwd(causal: bool) -> float:
     """The five N x N x d products of the backward pass (S, dP, dV, dK, dQ)."""
     return 10.0 * B * H * N * N * D * (0.5 if causal else 1.0)
@@ -691,6 +761,26 @@ def extras(peaks: dict, reps: int) -> dict:
                                         "frac_mixed_peak": tf * 0.75 / bf16}
         step_ms = res["rotate_quant_qk_per_tensor"]["ms"] + ms_a
         res["step_quant_plus_attn"] = {"ms": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12}
+        # Q rotated and quantised inside the attention kernel: the step is the
+        # per-block quantisation of K and the attention, with no pass over Q
+        kbytes = k.numel() * 3
+        ms_k = time_call(lambda: fa.hadamard_quant_blocks(k, rotate=True, signs=signs, out=k8, descales=dkb), reps,
+                         flush)
+        res["rotate_quant_k_per_block"] = {"ms": ms_k, "gbs": kbytes / (ms_k * 1e-3) / 1e9,
+                                           "frac": kbytes / (ms_k * 1e-3) / 1e9 / hbm, "bytes": kbytes,
+                                           "bound": "hbm"}
+        ms_f = time_call(lambda: fa.fwd_fp8_qrot(q, k8, v, dkb, signs=signs, out=o, lse=lse), reps, flush)
+        tf = fl / (ms_f * 1e-3) / 1e12
+        res["attn_e4m3qk_q_quantised_in_kernel"] = {"ms": ms_f, "tflops": tf,
+                                                     "frac_fp8_peak": tf / (FP8_OVER_BF16 * bf16),
+                                                     "frac_mixed_peak": tf * 0.75 / bf16}
+
+        def fused_step():
+            fa.hadamard_quant_blocks(k, rotate=True, signs=signs, out=k8, descales=dkb)
+            fa.fwd_fp8_qrot(q, k8, v, dkb, signs=signs, out=o, lse=lse)
+
+        ms_s = time_call(fused_step, reps, flush)
+        res["step_quant_k_plus_attn_q_in_kernel"] = {"ms": ms_s, "tflops": fl / (ms_s * 1e-3) / 1e12}
         return res
 
     guarded(f"fp8_b{FP8_CFG['B']}h{FP8_CFG['H']}n{FP8_CFG['N']}d{FP8_CFG['d']}", fp8)
@@ -987,6 +1077,52 @@ def run_bwd(args, world: int, rank: int):
     dist_done(world)
 
 
+def run_fp8(args, world: int, rank: int):
+    step = Fp8Step(FP8_CFG["seed"] + rank)
+    graph = capture_step(step)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms, per = time_steps(step, graph, args.steps, args.warmup, world)
+    e2e_ms = None if args.no_e2e else dist_max(time_e2e(step, max(8, args.steps // 2), 3, world), world)
+    ms = dist_max(statistics.mean(step_ms), world)
+    comp = [dist_max(statistics.mean(p[j] for p in per), world) for j in range(2)]
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    if rank == 0:
+        f = FP8_CFG
+        bf16 = peaks["bf16_tflops"]
+        mixed = bf16 / 0.75  # Q.K^T at the e4m3 rate (2x), P.V at the bf16 rate
+        achieved = step.flops / (comp[1] * 1e-3) / 1e12
+        qbytes = 2 * step.q_h.numel() * 3
+        line = {
+            "metric": METRIC, "value": world * step.flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (Q, K) / bf16 (P, V)",
+            "data": "synthetic (seeded N(0,1) bf16)",
+            "config": {"workload": f"fp8 b{f['B']}h{f['H']}n{f['N']}d{f['d']}: rotate + quantise Q, K (one launch, a "
+                                   "scale each) + e4m3-QK attention, non-causal", "B": f["B"], "H": f["H"],
+                       "N": f["N"], "d": f["d"], "parallelism": f"replicas x{world}",
+                       "l2": "inputs (201 MB) larger than L2, and L2 flushed between steps"},
+            "timing": "value: CUDA-graph replay of the step; breakdown: eager calls, events per kernel",
+            "breakdown_ms": {"rotate_quant_qk": comp[0], "attn_e4m3qk": comp[1]},
+            "roofline": {"kernel": "attn_fwd_kernel<128,2,nc,e4m3-QK>", "bound": "tensor", "achieved": achieved,
+                         "peak": mixed, "unit": "TFLOP/s", "frac": achieved / mixed, "traffic": None,
+                         "peak_source": f"derived from the {peak_src} cuBLAS bf16 burst peak: Q.K^T at 2x (nominal "
+                                        "e4m3:bf16), P.V at 1x"},
+            "quantiser": {"kernel": "quant_tma_kernel<128, rotate>", "bound": "hbm", "bytes": qbytes,
+                          "achieved_gbs": qbytes / (comp[0] * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                          "frac": qbytes / (comp[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": clocks_entry(clocks),
+        }
+        if e2e_ms is not None:
+            line["e2e"] = {"value": world * step.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                           "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
+                           "note": "bf16 Q, K, V copied in, O and LSE copied out per step; steps pipelined over three "
+                                   "CUDA streams"}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
 def run_decode(args, world: int, rank: int):
     step = DecodeStep(DECODE["seed"] + rank)
     graph = capture_step(step)
@@ -1040,11 +1176,17 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="headline only: skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host copies) measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--workload", choices=["fwd", "decode", "bwd"], default="fwd")
+    ap.add_argument("--workload", choices=["fwd", "decode", "bwd", "fp8"], default="fwd")
     args = ap.parse_args()
     world, rank, local = dist_setup()
 
     if args.impl == "reference":
+        if args.workload == "fp8":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the FP8 workload has no oracle arm of its own; "
+                                  "its parity is checked by the tests"}), flush=True)
+            dist_done(world)
+            return
         {"fwd": reference_fwd, "bwd": reference_bwd, "decode": reference_decode}[args.workload](args, world, rank)
         return
     if not torch.cuda.is_available():
@@ -1054,6 +1196,8 @@ def main():
         run_decode(args, world, rank)
     elif args.workload == "bwd":
         run_bwd(args, world, rank)
+    elif args.workload == "fp8":
+        run_fp8(args, world, rank)
     else:
         run_fwd(args, world, rank, local)
 

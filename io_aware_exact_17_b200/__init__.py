@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     bwd_workspace_bytes,
     device_status,
     fwd,
+    fwd_fp8_qrot,
     fwd_partial,
     fwd_splitkv,
     hadamard_quant,
@@ -25,5 +26,5 @@ from .binding import (  # noqa: F401
     splitkv_splits,
 )
 
-__all__ = ["fwd", "bwd", "bwd_workspace_bytes", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
+__all__ = ["fwd", "fwd_fp8_qrot", "bwd", "bwd_workspace_bytes", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
            "hadamard_quant_blocks", "hadamard_quant_multi", "device_status", "load_library", "library_path", "FaError"]

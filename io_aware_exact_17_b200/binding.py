@@ -78,6 +78,8 @@ def load_library():
         lib.fa_bwd_workspace_bytes.restype = sz
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
         lib.fa_bwd.restype = i
+        lib.fa_fwd_fp8_qrot.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, i, vp, vp, vp]
+        lib.fa_fwd_fp8_qrot.restype = i
         _lib = lib
         return lib
 
@@ -224,6 +226,46 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, qk_descale=No
                                     _ptr(ws) if need > 0 else None, need, _stream(q.device))
             _check(rc, "fa_fwd_splitkv")
     return out, (lse if return_lse else None)
+
+
+def fwd_fp8_qrot(q, k8, v, dk_blocks, causal: bool = False, scale: float | None = None, rotate: bool = True,
+                 signs=None, out=None, lse=None, return_lse: bool = True, return_dq: bool = False):
+    """e4m3 attention with Q rotated and quantised inside the attention kernel
+    (``fa_fwd_fp8_qrot``): ``q`` bf16 ``[B, H, N, 128]``; ``k8`` the e4m3 codes
+    of K with one descale per 128-row block, ``dk_blocks`` fp32 ``[B, H,
+    ceil(N/128)]`` (as ``hadamard_quant_blocks(k, rotate, signs)`` gives); ``v``
+    bf16. Each 128-row query tile is rotated with the same ``signs`` (if
+    ``rotate``) and quantised with its own scale in shared memory. Returns ``(O,
+    LSE)`` and, with ``return_dq``, also the query-block descales the kernel
+    computed, fp32 ``[B, H, ceil(N/128)]``."""
+    _require_cuda(q, k8, v, dk_blocks)
+    lib = load_library()
+    if q.dim() != 4 or q.dtype != torch.bfloat16 or v.dtype != torch.bfloat16 or tuple(v.shape) != tuple(q.shape):
+        raise FaError("q and v must be bf16 [B, H, N, d] of one shape")
+    B, H, N, d = q.shape
+    dev = q.device
+    _tensor_arg(k8, "k8", dev, E4M3_DTYPES, (B, H, N, d))
+    nb = -(-N // BLOCK_ROWS)
+    _tensor_arg(dk_blocks, "dk_blocks", dev, (torch.float32,), (B, H, nb))
+    q, v = q.contiguous(), v.contiguous()
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    _tensor_arg(out, "out", dev, (torch.bfloat16,), (B, H, N, d))
+    if return_lse:
+        if lse is None:
+            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        _tensor_arg(lse, "lse", dev, (torch.float32,), (B, H, N))
+    dq = torch.empty((B, H, nb), dtype=torch.float32, device=dev) if return_dq else None
+    signs = _signs_arg(signs, d, dev) if rotate else None
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(dev):
+        rc = lib.fa_fwd_fp8_qrot(_ptr(q), _ptr(k8), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None, B, H, N,
+                                 d, int(bool(causal)), float(scale), _ptr(dk_blocks), int(bool(rotate)), _ptr(signs),
+                                 _ptr(dq), _stream(dev))
+    _check(rc, "fa_fwd_fp8_qrot")
+    res = (out, lse if return_lse else None)
+    return res + (dq,) if return_dq else res
 
 
 _split_workspaces: dict[tuple[int, int], torch.Tensor] = {}

@@ -247,3 +247,24 @@ def test_tensor_argument_checks_run_before_any_launch():
         binding._descale_arg(ok.reshape(-1)[:2], 1, 1, 128, 128, dev)   # host descale
     with pytest.raises(binding.FaError):
         binding._descale_arg(None, 1, 1, 128, 128, dev)
+
+
+def test_fused_q_argument_errors(lib):
+    def call(**kw):
+        return lib.fa_fwd_fp8_qrot(kw.get("q", A), kw.get("k", A), kw.get("v", A), kw.get("o", A), kw.get("lse", A),
+                                   1, 2, kw.get("N", 300), kw.get("d", 128), kw.get("causal", 0), kw.get("scale", 0.1),
+                                   kw.get("dk", A), kw.get("rotate", 1), kw.get("signs", None), kw.get("dq", None),
+                                   None)
+    lib.fa_fwd_fp8_qrot.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_void_p,
+                                                                                   ctypes.c_int] + [ctypes.c_void_p] * 3
+    lib.fa_fwd_fp8_qrot.restype = ctypes.c_int
+    for name in ("q", "k", "v", "o", "dk"):
+        assert call(**{name: None}) == binding.FA_ERR_INVALID_ARG, name
+    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(d=256) == binding.FA_ERR_UNSUPPORTED
+    assert call(rotate=2) == binding.FA_ERR_INVALID_ARG
+    assert call(N=0) == binding.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == binding.FA_ERR_INVALID_ARG
+    assert call(q=MIS) == binding.FA_ERR_ALIGNMENT
+    assert call(signs=A + 4) == binding.FA_ERR_ALIGNMENT
+    assert call(dq=A + 2) == binding.FA_ERR_ALIGNMENT

@@ -55,12 +55,25 @@ def _check_block_codes(x, rotate, signs):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("N", [1, 127, 128, 300])
+@pytest.mark.parametrize("N", [1, 127, 128, 300, 1000])
 @pytest.mark.parametrize("rotate", [False, True])
 def test_block_quant_matches_oracle(d, N, rotate):
     q, _, _ = inputs.qkv_normal(2, 3, N, d, 90 + N + d)
     signs = inputs.hadamard_signs(d, 90) if rotate else None
     _check_block_codes(q, rotate, signs)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_block_quant_many_stages_per_cta_and_repeatable(d):
+    # 2 x 16 heads of 4096 rows: every CTA streams many stages of several heads
+    q, _, _ = inputs.qkv_normal(2, 16, 4096, d, 95 + d)
+    signs = inputs.hadamard_signs(d, 95)
+    codes, ds = _check_block_codes(q, True, signs)
+    qc, sg = q.cuda(), signs.cuda()
+    for _ in range(10):
+        c2, d2 = fa.hadamard_quant_blocks(qc, rotate=True, signs=sg)
+        assert np.array_equal(c2.cpu().numpy(), codes) and np.array_equal(d2.cpu().double().numpy(), ds)
+    _status_ok()
 
 
 def test_block_quant_blocks_of_different_ranges_and_a_zero_block():
