@@ -16,6 +16,9 @@
 //    of a tile therefore never waits for its own product to come back; it waits
 //    only for the S that was computed while it worked on the previous one;
 //  * TMEM: S_0 (2 x 64 columns), S_1 (2 x 64), O_0 (128), O_1 (128) = 512;
+//  * P_t(j) is signalled on a barrier of its own S buffer (bar_p[t][j & 1]):
+//    the softmax may finish P_t(j+1) before the MMA warp has taken P_t(j), so
+//    one barrier for both would run two phases ahead of its waiter;
 //  * a rescale of O (the reference max grew by more than 2^8) needs O's product
 //    of the previous step to be complete: that is the commit of S_t(j+1) (issued
 //    after it), or for a tile's last step a commit issued right after its last
@@ -137,7 +140,7 @@ attn_fwd_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __shared__ __align__(8) uint64_t bar_full[C::NSLOT], bar_empty[C::NSLOT];
   // bar_s[t][b]: S_t landed in buffer b; bar_pvq[t]: the tile's last but one
   // P V has completed; bar_qfree: the item's S MMAs (readers of sQ) are done
-  __shared__ __align__(8) uint64_t bar_q, bar_qfree, bar_drain, bar_s[NQ][2], bar_p[NQ], bar_o[NQ], bar_pvq[NQ];
+  __shared__ __align__(8) uint64_t bar_q, bar_qfree, bar_drain, bar_s[NQ][2], bar_p[NQ][2], bar_o[NQ], bar_pvq[NQ];
   // QROT: query tile t is in e4m3 (its warpgroup has converted it)
   __shared__ __align__(8) uint64_t bar_qready[NQ];
   __shared__ float qrot_red[NQ][4];  // per-warp maxima of each tile
@@ -184,7 +187,8 @@ attn_fwd_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&bar_s[t][0], 1);
       mbar_init(&bar_s[t][1], 1);
-      mbar_init(&bar_p[t], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&bar_p[t][0], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&bar_p[t][1], 4);
       mbar_init(&bar_o[t], 1);
       mbar_init(&bar_pvq[t], 1);
       mbar_init(&bar_qready[t], 4);
@@ -248,7 +252,7 @@ attn_fwd_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t ring = smem_u32(sRing);
       const uint32_t qaddr = smem_u32(sQ);
       int pos = 0, iter = 0;
-      uint32_t pc0 = 0u, pc1 = 0u;  // P-barrier phases waited, per query tile
+      uint32_t pc[2][2] = {{0u, 0u}, {0u, 0u}};  // P-barrier phases waited, per query tile and buffer
       bool ok = true;
       for (int it = next_item(0); it < p.n_items && ok; it = next_item(iter + 1), ++iter) {
         const FwdItem w = item_at(it);
@@ -267,9 +271,10 @@ attn_fwd_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int n_t = n_kv_at(t);
             const int jv = s - 2;  // the step whose P V runs now
             if (jv >= 0 && jv < n_t) {
-              const uint32_t ph = (t == 0 ? pc0 : pc1) & 1u;
-              if (t == 0) ++pc0; else ++pc1;
-              ok = mbar_wait(&bar_p[t], ph, &abort_flag, st, 123 + t, kMmaWaitSleepNs);
+              uint32_t& cnt = t == 0 ? (jv & 1 ? pc[0][1] : pc[0][0]) : (jv & 1 ? pc[1][1] : pc[1][0]);
+              const uint32_t ph = cnt & 1u;
+              ++cnt;
+              ok = mbar_wait(&bar_p[t][jv & 1], ph, &abort_flag, st, 123 + t, kMmaWaitSleepNs);
               if (!ok) break;
               tc_fence_after();
               // O_t += P_t(jv) V_jv: A = P (bf16 pairs over S buffer jv & 1), B = V (MN-major)
@@ -419,7 +424,7 @@ attn_fwd_db_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_p[t]);
+        if (lane == 0) mbar_arrive(&bar_p[t][b]);
       }
       if (n_t >= 2 && ok) {  // keep bar_pvq's phase in step (the wait is immediate here)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvq[t], qc & 1u, &abort_flag, st, 136 + t));
