@@ -224,10 +224,6 @@ fa_status launch_fwd_db(const FwdArgs& a, cudaStream_t stream) {
 
 template <int D, int NQ, bool QK_FP8, bool DEC>
 fa_status launch_fwd_cd(const FwdArgs& a, cudaStream_t s) {
-  if constexpr (D == 128 && NQ == 2 && !DEC) {
-    if (kFwdDb && a.o_part == nullptr && a.Nq == a.Nk)
-      return a.causal ? launch_fwd_db<true, QK_FP8>(a, s) : launch_fwd_db<false, QK_FP8>(a, s);
-  }
   if (a.o_part != nullptr)
     return a.causal ? launch_fwd<D, NQ, true, QK_FP8, true, DEC>(a, s)
                     : launch_fwd<D, NQ, false, QK_FP8, true, DEC>(a, s);
@@ -244,6 +240,12 @@ fa_status launch_fwd_c(const FwdArgs& a, cudaStream_t s) {
 
 // Kernel choice by head dimension, dtype and query length.
 fa_status dispatch_fwd(const FwdArgs& a, cudaStream_t s) {
+  // d = 128 square launches (any N): attn_fwd_db_kernel
+  if (kFwdDb && a.d == 128 && a.o_part == nullptr && a.Nq == a.Nk) {
+    if (a.qk_dtype == FA_BF16)
+      return a.causal ? launch_fwd_db<true, false>(a, s) : launch_fwd_db<false, false>(a, s);
+    return a.causal ? launch_fwd_db<true, true>(a, s) : launch_fwd_db<false, true>(a, s);
+  }
   const bool two = nq_for(a.d, a.Nq) == 2;
   if (a.qk_dtype == FA_BF16) {
     switch (a.d) {
