@@ -11,7 +11,6 @@
 #include "../../include/fa.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
-#include "attn_fwd_db.cuh"
 #include "merge.cuh"
 #include "quant.cuh"
 #include "tmap.h"
@@ -159,69 +158,6 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-#ifndef FA_FWD_DB
-#define FA_FWD_DB 1
-#endif
-// d = 128 square launches run attn_fwd_db_kernel (64-key steps, S double-buffered).
-constexpr bool kFwdDb = FA_FWD_DB != 0;
-
-template <bool CAUSAL, bool QK_FP8, bool QROT = false>
-fa_status launch_fwd_db(const FwdArgs& a, cudaStream_t stream) {
-  using C = fa::DbCfg<QK_FP8, QROT>;
-  constexpr int D = C::D;
-  const int BH = a.B * a.H;
-  CUtensorMap tmQ, tmK, tmV;
-  const CUtensorMapDataType qk_type = QK_FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const bool q_ok = QROT ? fa::make_tmap_3d(&tmQ, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nq, BH, 64, C::BM)
-                         : fa::make_tmap_3d(&tmQ, a.q, qk_type, C::EQK, D, a.Nq, BH, 128 / C::EQK, C::BM);
-  if (!q_ok || !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
-      !fa::make_tmap_3d(&tmV, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nk, BH, 64, C::BN))
-    return FA_ERR_CUDA;
-  auto kernel = fa::attn_fwd_db_kernel<CAUSAL, QK_FP8, QROT>;
-  static unsigned long long smem_done = 0;
-  if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
-  // the register split needs the block launched at REG_LAUNCH registers per thread
-  static int checked = 0;  // 0 = not yet, 1 = ok, 2 = bad
-  if (checked == 0) {
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
-    checked = attr.numRegs >= C::REG_LAUNCH ? 1 : 2;
-  }
-  if (checked != 1) return FA_ERR_UNSUPPORTED;
-  FwdParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.o = static_cast<__nv_bfloat16*>(a.o);
-  p.lse = a.lse;
-  p.descale_qk = a.descale_qk;
-  p.nbq = (a.Nq + 127) / 128;
-  p.nbk = (a.Nk + 127) / 128;
-  p.qrot_signs = a.qrot_signs;
-  p.qrot_rotate = a.qrot_rotate;
-  p.dq_out = a.dq_out;
-  if (QROT) {
-    p.dk_block = a.descale_qk;  // key blocks only: the query blocks' are computed in the kernel
-  } else if (a.qk_dtype == FA_E4M3_BLOCK) {
-    p.dq_block = a.descale_qk;
-    p.dk_block = a.descale_qk + static_cast<size_t>(BH) * p.nbq;
-  }
-  p.BH = BH;
-  p.Nq = a.Nq;
-  p.Nk = a.Nk;
-  p.causal_off = a.Nk - a.Nq;
-  p.n_qb = (a.Nq + C::NQ * C::BM - 1) / (C::NQ * C::BM);
-  p.n_split = 1;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
-  const long long items = static_cast<long long>(p.n_qb) * BH;
-  if (items < 1) return FA_OK;
-  p.n_items = static_cast<int>(items);
-  p.snake = CAUSAL ? 1 : 0;
-  long long grid = items;
-  const long long sms = device_sms();
-  if (grid > sms) grid = sms;
-  kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
 template <int D, int NQ, bool QK_FP8, bool DEC>
 fa_status launch_fwd_cd(const FwdArgs& a, cudaStream_t s) {
   if (a.o_part != nullptr)
@@ -240,12 +176,6 @@ fa_status launch_fwd_c(const FwdArgs& a, cudaStream_t s) {
 
 // Kernel choice by head dimension, dtype and query length.
 fa_status dispatch_fwd(const FwdArgs& a, cudaStream_t s) {
-  // d = 128 square launches (any N): attn_fwd_db_kernel
-  if (kFwdDb && a.d == 128 && a.o_part == nullptr && a.Nq == a.Nk) {
-    if (a.qk_dtype == FA_BF16)
-      return a.causal ? launch_fwd_db<true, false>(a, s) : launch_fwd_db<false, false>(a, s);
-    return a.causal ? launch_fwd_db<true, true>(a, s) : launch_fwd_db<false, true>(a, s);
-  }
   const bool two = nq_for(a.d, a.Nq) == 2;
   if (a.qk_dtype == FA_BF16) {
     switch (a.d) {
@@ -581,8 +511,6 @@ fa_status fa_fwd_fp8_qrot(const void* q, const void* k8, const void* v, void* o,
   a.qrot_signs = rotate ? signs : nullptr;
   a.dq_out = dq_blocks_out;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (kFwdDb)
-    return causal ? launch_fwd_db<true, true, true>(a, s) : launch_fwd_db<false, true, true>(a, s);
   return causal ? launch_fwd<128, 2, true, true, false, false, true>(a, s)
                 : launch_fwd<128, 2, false, true, false, false, true>(a, s);
 }

@@ -4,10 +4,13 @@ quantised with its own scale in shared memory ("FlashAttention-3 (PT)",
 section "Inovações técnicas", subsection 3, steps 1-3, one scale per block of
 128 rows), so the FP8 step needs no separate pass over Q.
 
-* Bit for bit the same O, LSE and query-block descales as quantising Q first
-  with fa_hadamard_quant_blocks and running the FA_E4M3_BLOCK attention: the
+* Bit for bit the same query-block descales as quantising Q first with
+  fa_hadamard_quant_blocks and running the FA_E4M3_BLOCK attention (the
   in-kernel rotation takes the same butterfly stages in the same order, so the
-  codes are the same.
+  codes are the same), and, where both run two query tiles per CTA (N > 128),
+  bit for bit the same O and LSE. For N <= 128 the FA_E4M3_BLOCK launch takes
+  one query tile per CTA, which sums in another order, so O and LSE are
+  compared there within the bf16 tolerance.
 * The query-block descales against the oracle's per-block quantiser, and the
   output against oracle attention on the oracle's dequantised Q and K.
 * The relative RMSE at the FP8 workload's shape against exact attention.
@@ -45,8 +48,12 @@ def test_fused_q_equals_quantise_then_attend(N, causal, rotate, use_signs):
     o, lse, dq_fused = fa.fwd_fp8_qrot(q, k8, v, dk, causal=causal, rotate=rotate, signs=signs, return_dq=True)
     _status_ok()
     assert torch.equal(dq_fused, dq)
-    assert torch.equal(o, o_ref)
-    assert torch.equal(lse, lse_ref)
+    if N > 128:
+        assert torch.equal(o, o_ref)
+        assert torch.equal(lse, lse_ref)
+    else:
+        assert max_abs(to_np(o), to_np(o_ref)) <= BF16_O_ATOL
+        assert max_abs(to_np(lse), to_np(lse_ref)) <= BF16_LSE_ATOL
 
 
 @pytest.mark.parametrize("causal", [False, True])
