@@ -187,14 +187,14 @@ struct QuantBatch {
 //
 // One CTA per SM. A producer warp streams blocks of RB rows of the tensors
 // through a ring of stages (TMA, 128-byte swizzle), far enough ahead to keep
-// HBM busy; 16 consumer warps take one stage at a time, each thread 64
-// consecutive elements of one row (a whole 128-byte swizzle column), so the
-// first six butterfly stages of the rotation stay inside the thread and only
-// log2(d / 64) stages cross lanes. Pass 1 reduces |x'| per tensor; a bounded
-// grid barrier publishes the amax words; pass 2 streams the same blocks again,
-// in reverse order so that the most recently read ones, still in L2, come
-// first, and writes the codes. The producer runs on into pass 2 while the
-// consumers wait at the barrier.
+// HBM busy; 8 consumer warps take one stage at a time, each thread a whole row
+// (d <= 128) or half a row (d = 256), so the butterfly stages of the rotation
+// stay inside the thread (one cross-lane stage at d = 256) and a warp's sign
+// loads are broadcasts. Pass 1 reduces |x'| per tensor; a bounded grid barrier
+// publishes the amax words; pass 2 streams the same blocks again, in reverse
+// order so that the most recently read ones, still in L2, come first, and
+// writes the codes. The producer runs on into pass 2 while the consumers wait
+// at the barrier.
 //
 // The butterflies run over index bits 0, 1, ... in increasing order with the
 // same operations as hadamard_rotate, so the codes are bit-identical to the
@@ -207,17 +207,18 @@ __global__ void fill_f32_kernel(float* out, int n, float v) {
   if (static_cast<int>(threadIdx.x) < n) out[threadIdx.x] = v;
 }
 
-constexpr int kTmaQuantConsumers = 512;
+constexpr int kTmaQuantConsumers = 256;
 constexpr int kTmaQuantStages = 3;
 
 template <int D>
 struct TmaQuantCfg {
-  static constexpr int E = 64;                           // elements per thread: one 128-byte column
+  static constexpr int E = D < 128 ? D : 128;            // elements per thread
+  static constexpr int W = E / 2;                        // packed pairs per thread
   static constexpr int TPR = D / E;                      // threads per row
   static constexpr int RB = kTmaQuantConsumers / TPR;    // rows per stage
   static constexpr int BOX_ROWS = RB < 256 ? RB : 256;   // TMA box height (at most 256)
   static constexpr int COLS = D / 64;                    // 128-byte columns per row
-  static constexpr int STAGE = RB * D * 2;               // bytes per stage (64 KB)
+  static constexpr int STAGE = RB * D * 2;               // bytes per stage
   static constexpr int CONSUMER_WARPS = kTmaQuantConsumers / 32;
   static constexpr int THREADS = kTmaQuantConsumers + 32;  // + the producer warp
   static constexpr int SMEM = 1024 + kTmaQuantStages * STAGE;
@@ -231,33 +232,34 @@ struct QuantMaps {
   int n;
 };
 
-// In place: 64 consecutive elements e0 .. e0+63 of a row (w[i] = elements
-// e0+2i, e0+2i+1) become the same elements of (x * signs) H_D, without the
-// 1/sqrt(D) factor. The TPR threads of the row (lanes 8 apart, part p = e0 / 64
-// = bits 3.. of the lane) must call together.
+// In place: the thread's E consecutive elements e0 .. e0+E-1 of a row (w[i] =
+// elements e0+2i, e0+2i+1) become the same elements of (x * signs) H_D,
+// without the 1/sqrt(D) factor. At d = 256 the two threads of a row (lanes 8
+// apart, part p = e0 / 128 = bit 3 of the lane) must call together.
 template <int D, bool ROT>
-__device__ __forceinline__ void rotate64(uint64_t (&w)[32], int p, const float* sgn) {
+__device__ __forceinline__ void rotate_part(uint64_t (&w)[TmaQuantCfg<D>::W], int p, const float* sgn) {
+  constexpr int E = TmaQuantCfg<D>::E, W = TmaQuantCfg<D>::W;
   if (!ROT) return;
   if (sgn != nullptr) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float4 s4 = *reinterpret_cast<const float4*>(sgn + 64 * p + 2 * i);
+    for (int i = 0; i < W; i += 2) {
+      const float4 s4 = *reinterpret_cast<const float4*>(sgn + E * p + 2 * i);
       w[i] = f2_mul(w[i], f2_pack(s4.x, s4.y));
       w[i + 1] = f2_mul(w[i + 1], f2_pack(s4.z, s4.w));
     }
   }
   // index bit 0: inside each pair
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < W; ++i) {
     float a, b;
     f2_unpack(w[i], a, b);
     w[i] = f2_pack(a + b, a - b);
   }
-  // index bits 1 .. 5: pair i with pair i + h
+  // index bits 1 .. log2(E) - 1: pair i with pair i + h
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
+  for (int h = 1; h < W; h <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < W; ++i) {
       if ((i & h) == 0) {
         const uint64_t a = w[i], b = w[i + h];
         w[i] = f2_add(a, b);
@@ -265,14 +267,14 @@ __device__ __forceinline__ void rotate64(uint64_t (&w)[32], int p, const float* 
       }
     }
   }
-  // index bits 6 ..: across the TPR lanes of the row (lower part: v + other,
-  // upper part: other - v, each one fma with +-1, i.e. one rounding)
+  // index bits log2(E) ..: across the TPR lanes of the row (lower part: v +
+  // other, upper part: other - v, each one fma with +-1, i.e. one rounding)
 #pragma unroll
-  for (int m = 1; m < D / 64; m <<= 1) {
+  for (int m = 1; m < D / E; m <<= 1) {
     const float sg = (p & m) != 0 ? -1.0f : 1.0f;
     const uint64_t sgn2 = f2_pack(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < W; ++i) {
       float a, b;
       f2_unpack(w[i], a, b);
       const float oa = __shfl_xor_sync(0xffffffffu, a, 8 * m);
@@ -283,36 +285,41 @@ __device__ __forceinline__ void rotate64(uint64_t (&w)[32], int p, const float* 
 }
 
 // Consumer side shared by the TMA-staged quantisers: the thread's row within a
-// stage and its 64-element part of the row, and the reads of that part.
-// Lane bits 0-2: row (low bits), bits 3 .. 2+log2(TPR): the row's part p,
+// stage and its part of the row (E elements: p = 0 unless d = 256), and the
+// reads of that part. Lane bits 0-2: row (low bits), then (d = 256) the part,
 // higher bits: row (high bits). The 8 lanes of a shared-memory phase (one
-// 16-byte load each) then read the same chunk j of 8 consecutive rows, whose
-// swizzled positions j ^ (row & 7) are 8 different bank groups.
+// 16-byte load each) read the same chunk j of one column of 8 consecutive
+// rows, whose swizzled positions j ^ (row & 7) are 8 different bank groups.
 template <int D>
 struct TmaQuantLane {
   using C = TmaQuantCfg<D>;
-  static constexpr int LT = C::TPR == 1 ? 0 : (C::TPR == 2 ? 1 : 2);  // log2(TPR)
+  static constexpr int LT = C::TPR == 1 ? 0 : 1;  // log2(TPR)
   int p, rr;
   __device__ __forceinline__ TmaQuantLane(int warp, int lane)
       : p((lane >> 3) & (C::TPR - 1)), rr(warp * (32 / C::TPR) + (lane & 7) + 8 * (lane >> (3 + LT))) {}
-  __device__ __forceinline__ void load(const uint8_t* stage_base, uint64_t (&w)[32]) const {
-    const uint8_t* base = stage_base + p * (C::RB * 128) + rr * 128;
+  __device__ __forceinline__ void load(const uint8_t* stage_base, uint64_t (&w)[C::W]) const {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (rr & 7)) << 4));
-      w[4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
-      w[4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-      w[4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
-      w[4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+    for (int cc = 0; cc < C::E / 64; ++cc) {
+      const uint8_t* base = stage_base + (p * (C::E / 64) + cc) * (C::RB * 128) + rr * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (rr & 7)) << 4));
+        uint64_t* o = &w[32 * cc + 4 * j];
+        o[0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
+        o[1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+        o[2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
+        o[3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+      }
     }
   }
 };
 
-// max |v| over the thread's 64 values
-__device__ __forceinline__ float absmax64(const uint64_t (&w)[32]) {
+// max |v| over the thread's values
+template <int W>
+__device__ __forceinline__ float absmax_part(const uint64_t (&w)[W]) {
   float m = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < W; ++i) {
     float a, b;
     f2_unpack(w[i], a, b);
     m = fmax3(m, fabsf(a), fabsf(b));
@@ -320,23 +327,26 @@ __device__ __forceinline__ float absmax64(const uint64_t (&w)[32]) {
   return m;
 }
 
-// Codes of the thread's 64 values: e4m3(v [/ sqrt(D)] * sc), stored to dst
-// (64 bytes, 16-byte aligned).
+// Codes of the thread's E values: e4m3(v [/ sqrt(D)] * sc), stored to dst (E
+// bytes, 16-byte aligned).
 template <int D, bool ROT>
-__device__ __forceinline__ void store_codes64(const uint64_t (&w)[32], float sc, uint8_t* dst) {
+__device__ __forceinline__ void store_codes_part(const uint64_t (&w)[TmaQuantCfg<D>::W], float sc, uint8_t* dst) {
+  constexpr int E = TmaQuantCfg<D>::E;
   constexpr float inv_sqrt_d = D == 64 ? 0.125f : (D == 128 ? 0.08838834764831845f : 0.0625f);
   const uint64_t isd = f2_pack(inv_sqrt_d, inv_sqrt_d), sc2 = f2_pack(sc, sc);
-  uint32_t q[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float a0, b0, a1, b1;
-    f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i], isd) : w[2 * i], sc2), a0, b0);
-    f2_unpack(f2_mul(ROT ? f2_mul(w[2 * i + 1], isd) : w[2 * i + 1], sc2), a1, b1);
-    q[i] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
-  }
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+  for (int c = 0; c < E / 16; ++c) {  // 16 codes per store
+    uint32_t q[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float a0, b0, a1, b1;
+      f2_unpack(f2_mul(ROT ? f2_mul(w[8 * c + 2 * k], isd) : w[8 * c + 2 * k], sc2), a0, b0);
+      f2_unpack(f2_mul(ROT ? f2_mul(w[8 * c + 2 * k + 1], isd) : w[8 * c + 2 * k + 1], sc2), a1, b1);
+      q[k] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
+    }
+    d4[c] = make_uint4(q[0], q[1], q[2], q[3]);
+  }
 }
 
 // ws[0 .. n-1]: amax bits of each tensor, ws[n]: arrival counter of the grid
@@ -427,11 +437,11 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
       const int stage = s % kTmaQuantStages;
       ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 62));
       if (!ok) break;
-      uint64_t w[32];
+      uint64_t w[C::W];
       ln.load(smem + stage * C::STAGE, w);
       release_stage(stage);
-      rotate64<D, ROT>(w, ln.p, sg);
-      m = fmaxf(m, absmax64(w));
+      rotate_part<D, ROT>(w, ln.p, sg);
+      m = fmaxf(m, absmax_part(w));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -474,12 +484,12 @@ quant_tma_kernel(const __grid_constant__ QuantMaps qm, int rows, const float* __
       const int stage = s % kTmaQuantStages;
       ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (s / kTmaQuantStages) & 1, &abort_flag, st, 63));
       if (!ok) break;
-      uint64_t w[32];
+      uint64_t w[C::W];
       ln.load(smem + stage * C::STAGE, w);
       release_stage(stage);
-      rotate64<D, ROT>(w, ln.p, sg);
+      rotate_part<D, ROT>(w, ln.p, sg);
       const int row = block_of(i) * C::RB + ln.rr;
-      if (row < rows) store_codes64<D, ROT>(w, sc, qm.out[t] + static_cast<int64_t>(row) * D + 64 * ln.p);
+      if (row < rows) store_codes_part<D, ROT>(w, sc, qm.out[t] + static_cast<int64_t>(row) * D + C::E * ln.p);
     }
     // amax_t is read again only after the next round's first named barrier
   }
@@ -563,13 +573,13 @@ quant_block_tma_kernel(const __grid_constant__ CUtensorMap tmx, uint8_t* __restr
   for (int i = 0; i < K; ++i) {
     const int stage = i % kTmaQuantStages;
     if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], (i / kTmaQuantStages) & 1, &abort_flag, st, 65))) break;
-    uint64_t w[32];
+    uint64_t w[C::W];
     ln.load(smem + stage * C::STAGE, w);
     fence_proxy_async_shared();  // reads ordered before the producer's next TMA write of the stage
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
-    rotate64<D, ROT>(w, ln.p, sg);
-    float m = absmax64(w);
+    rotate_part<D, ROT>(w, ln.p, sg);
+    float m = absmax_part(w);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) red[i & 1][warp] = m;
@@ -585,8 +595,8 @@ quant_block_tma_kernel(const __grid_constant__ CUtensorMap tmx, uint8_t* __restr
           amax > 0.f ? amax / 448.0f : 1.0f;
       const int row = r0 + ln.rr % BLK;
       if (row < N)
-        store_codes64<D, ROT>(w, amax > 0.f ? 448.0f / amax : 1.0f,
-                              out + (static_cast<long long>(bh) * N + row) * D + 64 * ln.p);
+        store_codes_part<D, ROT>(w, amax > 0.f ? 448.0f / amax : 1.0f,
+                                 out + (static_cast<long long>(bh) * N + row) * D + C::E * ln.p);
     }
   }
 }
