@@ -1,5 +1,6 @@
 """bench.py's reference arm on CPU: the oracle timed per step, one JSON line with
-the contract's keys, for the default (forward) step and the backward workload."""
+the contract's keys, for the default (forward) step, the backward and the
+decode workloads; the FP8 workload has no oracle arm and says so."""
 import json
 import subprocess
 import sys
@@ -24,3 +25,17 @@ def test_reference_arm_prints_one_line(workload):
         assert key in line, key
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert ("bwd" in line["config"]["workload"]) == (workload == "bwd")
+
+
+def test_reference_arm_decode_and_fp8():
+    out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--workload", "decode",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=ROOT,
+                         check=True)
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["config"]["Nk"] == 32768 and line["e2e"]["h2d_bytes_per_step"] == 0
+    out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--workload", "fp8",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=120, cwd=ROOT,
+                         check=True)
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["impl"] == "reference" and "unavailable" in line
