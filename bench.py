@@ -1108,7 +1108,7 @@ def run_fp8(args, world: int, rank: int):
                          "peak": mixed, "unit": "TFLOP/s", "frac": achieved / mixed, "traffic": None,
                          "peak_source": f"derived from the {peak_src} cuBLAS bf16 burst peak: Q.K^T at 2x (nominal "
                                         "e4m3:bf16), P.V at 1x"},
-            "quantiser": {"kernel": "quant_tma_kernel<128, rotate>", "bound": "hbm", "bytes": qbytes,
+            "quantiser": {"kernel": "quant_tensor_kernel<128, rotate>", "bound": "hbm", "bytes": qbytes,
                           "achieved_gbs": qbytes / (comp[0] * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                           "frac": qbytes / (comp[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "gpu_launches": step.launches_per_step * args.steps,

@@ -174,8 +174,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                  void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace fa_hadamard_quant and fa_hadamard_quant_multi need (the amax
- * words and a grid-barrier counter, padded). */
+/* Bytes of device workspace fa_hadamard_quant and fa_hadamard_quant_multi need (an amax
+ * word and a grid-barrier counter per tensor, padded). */
 #define FA_QUANT_WORKSPACE_BYTES 256
 
 /*
@@ -285,15 +285,15 @@ fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, in
  * no device allocator (a plugin inside an application that manages all device
  * memory itself), or code that must not trigger the implicit device-wide
  * synchronisation an allocation can cause. This entry point needs no workspace:
- * the scratch (one 4-byte amax word per tensor) is a 256-byte array inside the
- * library, allocated when the library is loaded and held by every device that
- * loads it until the process exits. Results are identical to calling
- * fa_hadamard_quant once per tensor.
+ * the scratch (one 4-byte amax word per tensor and 8 grid-barrier counters) is
+ * a 288-byte array inside the library, allocated when the library is loaded and
+ * held by every device that loads it until the process exits. Results are
+ * identical to calling fa_hadamard_quant once per tensor.
  *
  * xs, outs   host arrays of `ntensors` device pointers: bf16 inputs [rows][d] and
  *            e4m3 outputs [rows][d], each 16-byte aligned (may be NULL if rows = 0).
  * descales   device, ntensors fp32 (descale of tensor i at descales[i]).
- * ntensors   1..64; more is rejected with FA_ERR_INVALID_ARG (the array holds 64 words).
+ * ntensors   1..64; more is rejected with FA_ERR_INVALID_ARG (the array holds 64 amax words).
  * rows, d, rotate, signs: as for fa_hadamard_quant, shared by all tensors.
  * The first call on a device looks up the array's device address (a one-time
  * set-up per device, with that device current); make that first call before any

@@ -92,11 +92,6 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const 
       "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until the bulk operations of this thread have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Wait until the bulk operations of this thread have completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -107,14 +102,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
                    smem_u32(smem_dst)),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
-}
-
-// Bounded wait used only while tearing down after an abort.
-__device__ __forceinline__ void mbar_drain_bwd(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return;
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait_sleep(bar, parity, 20000u))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
 template <int D, bool CAUSAL>
@@ -222,9 +209,9 @@ __global__ void __launch_bounds__(384, 1)
       ++issued;
     }
     // every load this thread issued lands before the CTA can exit
-    mbar_drain_bwd(bar_kv, 0);
+    mbar_drain(bar_kv, 0);
     for (int i = issued - C::NST; i < issued; ++i)
-      if (i >= 0) mbar_drain_bwd(&bar_full[i % C::NST], (i / C::NST) & 1);
+      if (i >= 0) mbar_drain(&bar_full[i % C::NST], (i / C::NST) & 1);
   } else if (warp == C::MMA_WARP && lane == 0) {
     // ---------------------------------------------------------- MMA issuer --
     constexpr uint32_t idesc_kq = idesc_make(1u, 128, 128, false);            // A, B K-major
@@ -292,7 +279,7 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) mma_commit(bar_done);
     // TMEM is freed below only after every issued MMA has finished
     mma_commit(bar_drain);
-    mbar_drain_bwd(bar_drain, 0);
+    mbar_drain(bar_drain, 0);
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
     const int g = static_cast<int>(warp >> 2);  // query columns 64g .. 64g + 63

@@ -30,11 +30,16 @@
 //    the O rescale (a TMEM read-modify-write) is rare. The final O / l and the
 //    LSE use the same reference, so the result is exact, not approximated;
 //  * the QK product can take e4m3 Q and K (the FP8 path with Hadamard-rotated
-//    inputs: section "Inovações técnicas", 3); P and V stay bf16.
+//    inputs: section "Inovações técnicas", 3); P and V stay bf16. Under QROT the
+//    kernel rotates and quantises its own bf16 query tiles: the MMA warp
+//    multiplies each tile by the signed Hadamard operand (hadamard.cuh) into
+//    the tile's S columns, and the tile's softmax warpgroup turns the product
+//    into e4m3 codes in place of the bf16 tile.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include "hadamard.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -46,9 +51,10 @@ namespace fa {
 #define FA_REG_OTHER 88
 #endif
 
-// QROT: Q arrives in bf16 and each query tile is rotated and quantised to e4m3
-// (one scale per tile) by its softmax warpgroup in shared memory, in place,
-// before its first Q Kᵀ; K is e4m3 with one scale per 128-key tile.
+// QROT: Q arrives in bf16 and each query tile is rotated (on the tensor core,
+// into its S columns) and quantised to e4m3 (one scale per tile, by its softmax
+// warpgroup, in place in shared memory) before its first Q Kᵀ; K is e4m3 with
+// one scale per 128-key tile.
 template <int D, int NQ, bool QK_FP8, bool QROT = false>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per tile (TMEM lanes)
@@ -67,7 +73,8 @@ struct FwdCfg {
   static constexpr int SLOT = V_TILE;  // a ring slot holds one K or one V tile
   static constexpr int RING_BUDGET = 200 * 1024 - NQ * Q_TILE;
   static constexpr int NSLOT = (RING_BUDGET / SLOT) > 6 ? 6 : (RING_BUDGET / SLOT);
-  static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + NSLOT * SLOT;
+  static constexpr int ROT_OP = QROT ? HadCfg<D>::HMAT : 0;  // the rotation operand (QROT)
+  static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + ROT_OP + NSLOT * SLOT;
   static constexpr int SOFTMAX_WARPS = 4 * NQ;
   static constexpr int MMA_WARP = SOFTMAX_WARPS;
   static constexpr int TMA_WARP = SOFTMAX_WARPS + 1;
@@ -134,15 +141,6 @@ struct FwdParams {
 struct FwdItem {
   int bh, sp, q0, kt0, n_kv0, n_kv1, n_kv;
 };
-
-// Bounded wait used only while tearing down after an abort: ignores the abort
-// flag and records nothing.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return;
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait_sleep(bar, parity, 20000u))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
 
 #ifndef FA_MMA_WAIT_SLEEP_NS
 #define FA_MMA_WAIT_SLEEP_NS 0
@@ -244,90 +242,6 @@ __device__ __forceinline__ float row_max_tmem(uint32_t tS, uint32_t* s, int kbas
     }
   }
   return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
-}
-
-// In-kernel rotate-and-quantise of one query tile (QROT). Thread r of the
-// tile's warpgroup owns row r: it reads the row's 128 bf16 values from the
-// tile as the TMA left it (two 64-element columns, 128-byte swizzle), applies
-// the signs and the 7 butterfly stages of H_128 in registers (index bits 0, 1,
-// ... in increasing order with the same operations as the standalone
-// quantisers, so the rotated values are the same bits), then the warpgroup
-// takes the tile's amax through `red` and named barrier `bar_id`; the codes
-// e4m3(x' / sqrt(128) * 448 / amax) go to the row's first 128 bytes in the
-// swizzled K-major layout of an e4m3 operand. Every thread has read its row
-// before the barrier, so the in-place writes (row r's codes over the first
-// half of row r's bf16 values) never meet a read. Rows past the end of the
-// sequence hold zeros (TMA fill) and do not change the amax. Returns the
-// tile's descale amax / 448 (1 when the tile is zero): "FlashAttention-3 (PT)",
-// section "Inovações técnicas", subsection 3, steps 1-3, one scale per block of
-// 128 rows.
-__device__ __forceinline__ float qrot_tile(uint8_t* tile, int r, const float* signs, bool rotate, float* red,
-                                           uint32_t wq, uint32_t lane, uint32_t bar_id) {
-  constexpr float inv_sqrt_d = 0.08838834764831845f;  // 1 / sqrt(128)
-  uint64_t w[64];  // w[i] = elements 2i, 2i+1 of the row
-#pragma unroll
-  for (int c = 0; c < 2; ++c)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint4 u = *reinterpret_cast<const uint4*>(tile + c * (128 * 128) + r * 128 + ((j ^ (r & 7)) << 4));
-      w[32 * c + 4 * j + 0] = f2_pack(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
-      w[32 * c + 4 * j + 1] = f2_pack(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-      w[32 * c + 4 * j + 2] = f2_pack(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
-      w[32 * c + 4 * j + 3] = f2_pack(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
-    }
-  if (rotate) {
-    if (signs != nullptr) {
-#pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float4 s4 = __ldg(reinterpret_cast<const float4*>(signs + 2 * i));
-        w[i] = f2_mul(w[i], f2_pack(s4.x, s4.y));
-        w[i + 1] = f2_mul(w[i + 1], f2_pack(s4.z, s4.w));
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {  // index bit 0: inside each pair
-      float a, b;
-      f2_unpack(w[i], a, b);
-      w[i] = f2_pack(a + b, a - b);
-    }
-#pragma unroll
-    for (int h = 1; h < 64; h <<= 1)  // index bits 1 .. 6: pair i with pair i + h
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if ((i & h) == 0) {
-          const uint64_t a = w[i], b = w[i + h];
-          w[i] = f2_add(a, b);
-          w[i + h] = f2_sub(a, b);
-        }
-  }
-  float m = 0.f;
-#pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    float a, b;
-    f2_unpack(w[i], a, b);
-    m = fmax3(m, fabsf(a), fabsf(b));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[wq] = m;
-  named_barrier_sync(bar_id, 128);
-  float amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  if (rotate) amax *= inv_sqrt_d;  // fp32 rounding is monotonic: max fl(|v| c) = fl(c max |v|)
-  const float sc = amax > 0.f ? 448.0f / amax : 1.0f;
-  const uint64_t sc2 = f2_pack(sc, sc), isd = f2_pack(inv_sqrt_d, inv_sqrt_d);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {  // 16 codes (elements 16j .. 16j+15) per 16-byte chunk
-    uint32_t q[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float a0, b0, a1, b1;
-      f2_unpack(f2_mul(rotate ? f2_mul(w[8 * j + 2 * k], isd) : w[8 * j + 2 * k], sc2), a0, b0);
-      f2_unpack(f2_mul(rotate ? f2_mul(w[8 * j + 2 * k + 1], isd) : w[8 * j + 2 * k + 1], sc2), a1, b1);
-      q[k] = static_cast<uint32_t>(pack_e4m3x2(a0, b0)) | (static_cast<uint32_t>(pack_e4m3x2(a1, b1)) << 16);
-    }
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
-  }
-  return amax > 0.f ? amax / 448.0f : 1.0f;
 }
 
 // Softmax warps of a DEC CTA (see attn_fwd_kernel): warp w, lane r holds query
@@ -542,15 +456,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   static_assert(!DEC || C::NSLOT * C::SLOT >= 3 * 32 * D * 4, "decode merge buffer lives in the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                      // NQ tiles
-  uint8_t* sRing = smem + NQ * C::Q_TILE;  // NSLOT slots
+  uint8_t* sQ = smem;                                // NQ tiles
+  uint8_t* sRot = smem + NQ * C::Q_TILE;             // QROT: the rotation operand
+  uint8_t* sRing = smem + NQ * C::Q_TILE + C::ROT_OP;  // NSLOT slots
 
   __shared__ __align__(8) uint64_t bar_full[C::NSLOT], bar_empty[C::NSLOT];
   // bar_qfree: the S MMAs that read the current item's Q tiles are done (the
   // producer may load the next item's Q)
   __shared__ __align__(8) uint64_t bar_q, bar_qfree, bar_drain, bar_s[NQ], bar_p[NQ], bar_o[NQ];
-  // QROT: query tile t is in e4m3 (its warpgroup has converted it)
-  __shared__ __align__(8) uint64_t bar_qready[NQ];
+  // QROT: bar_rot[t]: the product of query tile t and the rotation operand is
+  // in its S columns (and the bf16 tile has been read); bar_qready[t]: query
+  // tile t is in e4m3 (its warpgroup has converted it)
+  // bar_qamax[t]: the four warps of tile t's warpgroup have posted their maxima
+  __shared__ __align__(8) uint64_t bar_rot[NQ], bar_qready[NQ], bar_qamax[NQ];
   __shared__ float qrot_red[NQ][4];  // per-warp maxima of each tile
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -606,9 +524,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], 4);  // one arrival per softmax warp of the tile
       mbar_init(&bar_o[t], 1);
+      mbar_init(&bar_rot[t], 1);
       mbar_init(&bar_qready[t], 4);
+      mbar_init(&bar_qamax[t], 4);
     }
     fence_mbar_init();
+  }
+  if constexpr (QROT) {
+    if (p.qrot_rotate)
+      build_rotation_operand<D, true>(sRot, p.qrot_signs);
+    else
+      build_rotation_operand<D, false>(sRot, nullptr);
+    fence_proxy_async_shared();  // the tensor core reads the operand through the async proxy
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(&tmem_slot, C::TMEM_COLS);
@@ -686,7 +613,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const FwdItem w = item_at(it);
       const int n_kv = w.n_kv;
       auto n_kv_at = [&](int t) { return t == 0 ? w.n_kv0 : w.n_kv1; };
-      if constexpr (!QROT) ok = mbar_wait(&bar_q, iter & 1, &abort_flag, st, 20);
+      ok = mbar_wait(&bar_q, iter & 1, &abort_flag, st, 20);
+      if constexpr (QROT) {
+        // Each query tile times the rotation operand, into the tile's S
+        // columns: the previous item's last P V of the tile, which read P
+        // there, was issued before (the tensor core runs them in order).
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < NQ; ++t) {
+            issue_rotation<D>(tbase + C::S_COL(t), qaddr + t * C::Q_TILE, smem_u32(sRot));
+            mma_commit(&bar_rot[t]);
+          }
+        }
+      }
       for (int j = 0; j <= n_kv && ok; ++j) {
         const int kpos = pos + 2 * j, vpos = pos + 2 * j - 1;
         const int kslot = kpos % C::NSLOT, vslot = (vpos + C::NSLOT) % C::NSLOT;
@@ -776,14 +715,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float s_q = p.scale_log2;
     const float* dkb = nullptr;
     if constexpr (QROT) {
-      // this warpgroup's Q tile, bf16 from the TMA, to e4m3 in place
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_q, round & 1, &abort_flag, st, 35));
+      // this warpgroup's Q tile: the rotated rows from tensor memory, to e4m3
+      // codes in place of the bf16 tile (which the product has finished reading)
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&bar_rot[t], round & 1, &abort_flag, st, 35));
+      float m = 0.f;
+      if (got) {
+        tc_fence_after();
+        m = p.qrot_rotate ? row_absmax<D, true>(tS) : row_absmax<D, false>(tS);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      // The tile's amax from the four warps' maxima. An mbarrier, not a named
+      // barrier: a warp that has left after an abort leaves the others a
+      // bounded wait, not a hang.
+      if (lane == 0) {
+        qrot_red[t][warp & 3u] = m;
+        mbar_arrive(&bar_qamax[t]);  // release: the maximum is visible to the waiters
+      }
+      ok = got && __all_sync(0xffffffffu, mbar_wait(&bar_qamax[t], round & 1, &abort_flag, st, 36));
       if (!ok) break;
-      const float dq = qrot_tile(sQ + t * C::Q_TILE, r, p.qrot_rotate ? p.qrot_signs : nullptr, p.qrot_rotate != 0,
-                                 qrot_red[t], warp & 3u, lane, 2 + t);
-      fence_proxy_async_shared();  // the tensor core reads the codes through the async proxy
+      float amax = fmaxf(fmaxf(qrot_red[t][0], qrot_red[t][1]), fmaxf(qrot_red[t][2], qrot_red[t][3]));
+      if (p.qrot_rotate) amax *= HadCfg<D>::INV_SQRT_D;  // fp32 rounding is monotonic: max fl(|v| c) = fl(c max |v|)
+      const float qsc = amax > 0.f ? 448.0f / amax : 1.0f;
+      const float dq = amax > 0.f ? amax / 448.0f : 1.0f;
+      // Rows past the end of the sequence hold zeros (TMA fill): they do not
+      // change the amax, and their codes are never used.
+      uint8_t* qrow_codes = sQ + t * C::Q_TILE + r * 128;
+      auto put = [&](int j, const uint4& v) {  // 16 codes, at their swizzled place
+        *reinterpret_cast<uint4*>(qrow_codes + ((j ^ (r & 7)) << 4)) = v;
+      };
+      if (p.qrot_rotate)
+        row_codes<D, true>(tS, qsc, put);
+      else
+        row_codes<D, false>(tS, qsc, put);
+      // the tensor core reads the codes through the async proxy, and the S
+      // product overwrites the columns just read
+      fence_proxy_async_shared();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_qready[t]);
+      // qrot_red[t] is written again only after the next item's bar_rot wait,
+      // which follows this item's S products, which follow every warp's
+      // bar_qready arrival, which follows its reads of qrot_red[t]
       if (p.dq_out != nullptr && r == 0 && q0 + t * C::BM < p.Nq)
         p.dq_out[static_cast<size_t>(bh) * p.nbq + (q0 + t * C::BM) / C::BM] = dq;
       s_q *= dq;

@@ -222,6 +222,19 @@ size_t part_bytes(int B, int H, int Nq, int d, int n_split) {
   return o + static_cast<size_t>(n_split) * B * H * Nq * sizeof(float);
 }
 
+// L2 cache bytes of the current device (looked up once per device).
+double device_l2_bytes() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 126.0 * (1 << 20);
+  if (cached[dev] == 0) {
+    int l2 = 0;
+    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 < 1) return 126.0 * (1 << 20);
+    cached[dev] = l2;
+  }
+  return static_cast<double>(cached[dev]);
+}
+
 int device_sms() {
   static int cached[64] = {};
   int dev = 0;
@@ -294,108 +307,85 @@ size_t plan_bytes(const Plan& pl, int B, int H, int Nq, int d) {
 // tensor of bf16 rows would not fit in a GPU's memory anyway).
 constexpr int64_t kQuantMaxRows = (static_cast<int64_t>(1) << 31) - 4096;
 
-template <int D>
-fa_status launch_quant(const void* x, void* out, float* descale_out, int64_t rows, int rotate, const float* signs,
-                       unsigned int* amax, cudaStream_t stream) {
-  using QC = fa::QuantCfg<D>;
-  if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
-  const int64_t steps = (rows + QC::ROWS_PER_STEP - 1) / QC::ROWS_PER_STEP;  // warp-steps of work
-  const int64_t warps_per_block = fa::kQuantThreads / 32;
-  int64_t blocks = (steps + warps_per_block - 1) / warps_per_block;
-  int sms = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident blocks of 256 threads per SM
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  uint8_t* ob = static_cast<uint8_t*>(out);
-  if (rotate) {
-    fa::quant_amax_kernel<D, true><<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, rows, signs, amax);
-    fa::quant_apply_kernel<D, true>
-        <<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, ob, rows, signs, amax, descale_out);
-  } else {
-    fa::quant_amax_kernel<D, false><<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, rows, nullptr, amax);
-    fa::quant_apply_kernel<D, false>
-        <<<static_cast<unsigned>(blocks), fa::kQuantThreads, 0, stream>>>(xb, ob, rows, nullptr, amax, descale_out);
-  }
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-// Both quantisation passes in one cooperative launch (quant_tma_kernel) for
-// the tensors of `b`: the workspace holds their amax words and the grid
-// barrier's counter, zeroed here. One CTA per SM (up to one per row block), all
-// co-resident.
+// Both quantisation passes in one cooperative launch (quant_tensor_kernel) for
+// the tensors of `b`: amax_words[0 .. n-1] and counters[0 .. n-1] (the grid
+// barriers' arrivals) are zeroed here. One CTA per SM (up to one per 128-row
+// tile), all co-resident.
 template <int D>
 fa_status launch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int rotate,
-                             const float* signs, unsigned int* ws, cudaStream_t stream) {
-  using TC = fa::TmaQuantCfg<D>;
-  if (cudaMemsetAsync(ws, 0, (b.n + 1) * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+                             const float* signs, unsigned int* amax_words, unsigned int* counters,
+                             cudaStream_t stream) {
+  using RC = fa::RotQuantCfg<D>;
+  if (counters == amax_words + b.n) {  // one contiguous scratch (the workspace entry points)
+    if (cudaMemsetAsync(amax_words, 0, 2 * b.n * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  } else {
+    if (cudaMemsetAsync(amax_words, 0, b.n * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemsetAsync(counters, 0, b.n * sizeof(unsigned int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  }
   if (rows == 0) {  // nothing to read: every descale is 1
     fa::fill_f32_kernel<<<1, 32, 0, stream>>>(descale_out, b.n, 1.0f);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
   }
-  auto kernel = rotate ? fa::quant_tma_kernel<D, true> : fa::quant_tma_kernel<D, false>;
+  auto kernel = rotate ? fa::quant_tensor_kernel<D, true> : fa::quant_tensor_kernel<D, false>;
   static unsigned long long smem_set[2] = {0, 0};
-  if (!set_smem_once(kernel, TC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
-  // Co-resident CTAs per SM, looked up once per device (host time in front of
-  // a ~20 us kernel).
-  static int cached_per_sm[2][64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return FA_ERR_UNSUPPORTED;
-  int& per_sm = cached_per_sm[rotate ? 1 : 0][dev];
-  if (per_sm == 0 &&
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, TC::THREADS, TC::SMEM) != cudaSuccess)
-    return FA_ERR_CUDA;
-  if (per_sm < 1) return FA_ERR_CUDA;
-  const int64_t nblk = (rows + TC::RB - 1) / TC::RB;
-  int64_t blocks = static_cast<int64_t>(per_sm) * device_sms();
-  if (blocks > nblk) blocks = nblk;
+  if (!set_smem_once(kernel, RC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
+  const int64_t ntile = (rows + RC::BM - 1) / RC::BM;
+  int64_t blocks = device_sms();  // one CTA per SM: the kernel holds all of an SM's tensor memory
+  if (blocks > ntile) blocks = ntile;
   fa::QuantMaps qm;
   std::memset(&qm, 0, sizeof(qm));
   for (int t = 0; t < b.n; ++t) {
     if (!fa::make_tmap_2d(&qm.x[t], b.x[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(rows), 64,
-                          TC::BOX_ROWS))
+                          RC::BM))
       return FA_ERR_CUDA;
-    qm.out[t] = b.out[t];
+    if (!fa::make_tmap_2d(&qm.y[t], b.out[t], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, static_cast<uint64_t>(rows),
+                          RC::CROW, 32, fa::codes_swizzle<D>()))
+      return FA_ERR_CUDA;
   }
   qm.n = b.n;
   int rows_i = static_cast<int>(rows);
-  void* args[] = {&qm, &rows_i, &signs, &ws, &descale_out};
+  // The next tensor's pass 1 runs ahead of this tensor's pass 2: all of it
+  // when two tensors fit in two thirds of L2 (pass 2 still finds its tensor
+  // there), else the first few tiles of each CTA, to cover the grid barrier.
+  const double two_tensors = 2.0 * static_cast<double>(rows) * D * 2;
+  int lead = two_tensors <= device_l2_bytes() * 2.0 / 3.0 ? 0x7fffffff : 4;
+  void* args[] = {&qm, &rows_i, &lead, &signs, &amax_words, &counters, &descale_out};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(static_cast<unsigned>(blocks)),
-                                  dim3(TC::THREADS), args, TC::SMEM, stream) != cudaSuccess)
+                                  dim3(RC::THREADS + 32), args, RC::SMEM, stream) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }
 
-// One scale per 128-row block of a head (quant_block_tma_kernel): one pass,
-// persistent CTAs (one per SM) over the stages of RB rows of each head.
+// One scale per 128-row block of a head (quant_block_kernel): one pass,
+// persistent CTAs (one per SM) over the tiles of each head.
 template <int D>
 fa_status launch_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int rotate,
                               const float* signs, cudaStream_t stream) {
-  using TC = fa::TmaQuantCfg<D>;
-  auto kernel = rotate ? fa::quant_block_tma_kernel<D, true> : fa::quant_block_tma_kernel<D, false>;
+  using RC = fa::RotQuantCfg<D>;
+  auto kernel = rotate ? fa::quant_block_kernel<D, true> : fa::quant_block_kernel<D, false>;
   static unsigned long long smem_set[2] = {0, 0};
-  if (!set_smem_once(kernel, TC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
-  CUtensorMap tm;
+  if (!set_smem_once(kernel, RC::SMEM, &smem_set[rotate ? 1 : 0])) return FA_ERR_CUDA;
+  CUtensorMap tm, tmy;
   if (!fa::make_tmap_3d(&tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(N),
-                        static_cast<uint64_t>(BH), 64, TC::BOX_ROWS))
+                        static_cast<uint64_t>(BH), 64, RC::BM))
     return FA_ERR_CUDA;
-  const long long units = static_cast<long long>(BH) * ((N + TC::RB - 1) / TC::RB);
+  if (!fa::make_tmap_3d(&tmy, out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, static_cast<uint64_t>(N),
+                        static_cast<uint64_t>(BH), RC::CROW, 32, fa::codes_swizzle<D>()))
+    return FA_ERR_CUDA;
+  const long long units = static_cast<long long>(BH) * ((N + RC::BM - 1) / RC::BM);
   long long grid = device_sms();
   if (grid > units) grid = units;
-  kernel<<<static_cast<unsigned>(grid), TC::THREADS, TC::SMEM, stream>>>(tm, static_cast<uint8_t*>(out), BH, N,
-                                                                          signs, descales);
+  kernel<<<static_cast<unsigned>(grid), RC::THREADS, RC::SMEM, stream>>>(tm, tmy, BH, N, signs, descales);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status dispatch_quant_fused(const fa::QuantBatch& b, float* descale_out, int64_t rows, int d, int rotate,
-                               const float* signs, unsigned int* ws, cudaStream_t s) {
+                               const float* signs, unsigned int* amax_words, unsigned int* counters,
+                               cudaStream_t s) {
   switch (d) {
-    case 64: return launch_quant_fused<64>(b, descale_out, rows, rotate, signs, ws, s);
-    case 128: return launch_quant_fused<128>(b, descale_out, rows, rotate, signs, ws, s);
-    default: return launch_quant_fused<256>(b, descale_out, rows, rotate, signs, ws, s);
+    case 64: return launch_quant_fused<64>(b, descale_out, rows, rotate, signs, amax_words, counters, s);
+    case 128: return launch_quant_fused<128>(b, descale_out, rows, rotate, signs, amax_words, counters, s);
+    default: return launch_quant_fused<256>(b, descale_out, rows, rotate, signs, amax_words, counters, s);
   }
 }
 
@@ -630,8 +620,8 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
   b.x[0] = static_cast<const __nv_bfloat16*>(x);
   b.out[0] = static_cast<uint8_t*>(out);
   b.n = 1;
-  return dispatch_quant_fused(b, descale_out, rows, d, rotate, sg, static_cast<unsigned int*>(workspace),
-                              static_cast<cudaStream_t>(stream));
+  unsigned int* ws = static_cast<unsigned int*>(workspace);  // word 0: amax, word 1: barrier counter (n = 1)
+  return dispatch_quant_fused(b, descale_out, rows, d, rotate, sg, ws, ws + 1, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, float* descales, int ntensors,
@@ -652,8 +642,9 @@ fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, floa
     b.out[i] = static_cast<uint8_t*>(outs[i]);
   }
   b.n = ntensors;
-  return dispatch_quant_fused(b, descales, rows, d, rotate, rotate ? signs : nullptr,
-                              static_cast<unsigned int*>(workspace), static_cast<cudaStream_t>(stream));
+  unsigned int* ws = static_cast<unsigned int*>(workspace);  // words 0 .. n-1: amax, n .. 2n-1: barrier counters
+  return dispatch_quant_fused(b, descales, rows, d, rotate, rotate ? signs : nullptr, ws, ws + ntensors,
+                              static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, int BH, int N, int d, int rotate,
@@ -679,17 +670,17 @@ fa_status fa_hadamard_quant_blocks(const void* x, void* out, float* descales, in
 // ---------------------------------------------------------------------------
 // Allocation-free quantisation (fa_hadamard_quant_noalloc).
 //
-// The scratch of the quantiser (one amax word per tensor) lives in this
-// file-scope device array instead of a caller workspace. Every device that
+// The scratch of the quantiser (one amax word per tensor, then one grid
+// barrier counter per tensor of a launch) lives in this file-scope device array
+// instead of a caller workspace. Every device that
 // loads the library holds it until the process exits. In host code the name
 // g_noalloc_scratch is only a host-side stand-in, never a device address: the
 // kernels get the address cudaGetSymbolAddress returns, looked up once per
 // device with that device current.
 namespace {
 
-constexpr int kNoallocScratchBytes = 256;
-constexpr int kNoallocMaxTensors = kNoallocScratchBytes / static_cast<int>(sizeof(unsigned int));  // 64
-static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoallocMaxTensors];
+constexpr int kNoallocMaxTensors = 64;
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoallocMaxTensors + fa::kQuantBatch];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
@@ -717,8 +708,8 @@ extern "C" {
 fa_status fa_hadamard_quant_noalloc(const void* const* xs, void* const* outs, float* descales, int ntensors,
                                     int64_t rows, int d, int rotate, const float* signs, void* stream) {
   if (xs == nullptr || outs == nullptr || descales == nullptr) return FA_ERR_INVALID_ARG;
-  if (ntensors < 1 || ntensors > kNoallocMaxTensors) return FA_ERR_INVALID_ARG;  // scratch holds 64 words
-  if (rows < 0 || rows > (static_cast<int64_t>(1) << 40) || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (ntensors < 1 || ntensors > kNoallocMaxTensors) return FA_ERR_INVALID_ARG;  // scratch holds 64 amax words
+  if (rows < 0 || rows > kQuantMaxRows || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (!aligned(descales, 4)) return FA_ERR_ALIGNMENT;
   if (signs != nullptr && !aligned(signs, 16)) return FA_ERR_ALIGNMENT;
@@ -731,15 +722,19 @@ fa_status fa_hadamard_quant_noalloc(const void* const* xs, void* const* outs, fl
   if (sst != FA_OK) return sst;
   const float* sg = rotate ? signs : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  for (int i = 0; i < ntensors; ++i) {
-    // Word i of the array is tensor i's amax; launch_quant zeroes it first on
-    // this stream, so what an earlier call left there does not matter.
-    fa_status r;
-    switch (d) {
-      case 64: r = launch_quant<64>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
-      case 128: r = launch_quant<128>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
-      default: r = launch_quant<256>(xs[i], outs[i], descales + i, rows, rotate, sg, scratch + i, s); break;
+  // Up to kQuantBatch tensors per launch; word i of the array is tensor i's
+  // amax and the last kQuantBatch words the launch's barrier counters, all
+  // zeroed by the launch on this stream, so what an earlier call left there
+  // does not matter.
+  for (int i0 = 0; i0 < ntensors; i0 += fa::kQuantBatch) {
+    fa::QuantBatch b = {};
+    b.n = ntensors - i0 < fa::kQuantBatch ? ntensors - i0 : fa::kQuantBatch;
+    for (int i = 0; i < b.n; ++i) {
+      b.x[i] = static_cast<const __nv_bfloat16*>(xs[i0 + i]);
+      b.out[i] = static_cast<uint8_t*>(outs[i0 + i]);
     }
+    const fa_status r = dispatch_quant_fused(b, descales + i0, rows, d, rotate, sg, scratch + i0,
+                                             scratch + kNoallocMaxTensors, s);
     if (r != FA_OK) return r;
   }
   return FA_OK;

@@ -39,3 +39,20 @@ def record(case: str, **values) -> None:
     if path:
         with open(path, "a") as f:
             f.write(json.dumps({"case": case, **{k: float(v) for k, v in values.items()}}) + "\n")
+
+
+def rotation_error_bound(x: np.ndarray, rotate: bool) -> np.ndarray:
+    """Bound on |x'_kernel - x'_exact| for each element of x' = x D H_d / sqrt(d)
+    (rows of x along the last axis, fp64), as the kernels compute it: each value
+    of x D H_d is a tensor-core sum of d exact products +-x_k in fp32, in an
+    order and with a rounding (nearest or towards zero) the hardware does not
+    document. Each of its d - 1 additions errs by at most one fp32 unit (2^-23)
+    of a partial sum bounded by sum_k |x_k|, so the error is below
+    d 2^-23 sum_k |x_k| (at d = 256 this also covers the one fp32 addition of
+    the last butterfly stage); then / sqrt(d). Without rotation the kernels
+    reproduce x exactly (a product with the identity): bound 0."""
+    if not rotate:
+        return np.zeros_like(x)
+    d = x.shape[-1]
+    l1 = np.abs(x).sum(axis=-1, keepdims=True)
+    return np.broadcast_to(d * 2.0**-23 * l1 / np.sqrt(d), x.shape)

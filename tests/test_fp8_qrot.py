@@ -6,11 +6,12 @@ section "Inovações técnicas", subsection 3, steps 1-3, one scale per block of
 
 * Bit for bit the same query-block descales as quantising Q first with
   fa_hadamard_quant_blocks and running the FA_E4M3_BLOCK attention (the
-  in-kernel rotation takes the same butterfly stages in the same order, so the
-  codes are the same), and, where both run two query tiles per CTA (N > 128),
-  bit for bit the same O and LSE. For N <= 128 the FA_E4M3_BLOCK launch takes
-  one query tile per CTA, which sums in another order, so O and LSE are
-  compared there within the bf16 tolerance.
+  in-kernel rotation is the same tensor-core product with the same operand,
+  followed by the same amax and rounding steps, so the codes are the same),
+  and, where both run two query tiles per CTA (N > 128), bit for bit the same
+  O and LSE. For N <= 128 the FA_E4M3_BLOCK launch takes one query tile per
+  CTA, which sums in another order, so O and LSE are compared there within
+  the bf16 tolerance.
 * The query-block descales against the oracle's per-block quantiser, and the
   output against oracle attention on the oracle's dequantised Q and K.
 * The relative RMSE at the FP8 workload's shape against exact attention.
