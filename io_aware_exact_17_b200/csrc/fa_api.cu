@@ -446,9 +446,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH, N,
       Npad);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  auto kernel = fa::attn_bwd_kernel<D, CAUSAL>;
+  // d = 128: the two softmax warpgroups ping-pong over half steps of 64 queries
+  auto kernel = D == 128 ? fa::attn_bwd_pp_kernel<CAUSAL> : fa::attn_bwd_kernel<D, CAUSAL>;
+  const int smem_bytes = D == 128 ? fa::BwdPpCfg::SMEM_BYTES : C::SMEM_BYTES;
   static unsigned long long smem_done = 0;
-  if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
+  if (!set_smem_once(kernel, smem_bytes, &smem_done)) return FA_ERR_CUDA;
   fa::BwdParams p;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -460,7 +462,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.n_t = Npad / 128;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, C::SMEM_BYTES, stream>>>(
+  kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, smem_bytes, stream>>>(
       tmQ, tmK, tmV, tmdO, tmdQ, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const long long n4 = static_cast<long long>(BH) * N * D / 4;

@@ -133,26 +133,27 @@ __device__ __forceinline__ void row_chunks(uint32_t tb, int c0, uint32_t (&v)[NC
   for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
     for (int b = 0; b < NBLK; ++b) tmem_wait_ld_dep32(v[cc][b]);  // the first waits for all; each ties its registers
-  if (!ROT) return;
+  if constexpr (ROT && NBLK > 1) {
 #pragma unroll
-  for (int cc = 0; cc < NC; ++cc)
+    for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
-    for (int h = 1; h < NBLK; h <<= 1)
+      for (int h = 1; h < NBLK; h <<= 1)
 #pragma unroll
-      for (int b = 0; b < NBLK; ++b)
-        if ((b & h) == 0)
+        for (int b = 0; b < NBLK; ++b)
+          if ((b & h) == 0)
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const uint64_t x = f2_pack(__uint_as_float(v[cc][b][j]), __uint_as_float(v[cc][b][j + 1]));
-            const uint64_t y = f2_pack(__uint_as_float(v[cc][b + h][j]), __uint_as_float(v[cc][b + h][j + 1]));
-            float s0, s1, d0, d1;
-            f2_unpack(f2_add(x, y), s0, s1);
-            f2_unpack(f2_sub(x, y), d0, d1);
-            v[cc][b][j] = __float_as_uint(s0);
-            v[cc][b][j + 1] = __float_as_uint(s1);
-            v[cc][b + h][j] = __float_as_uint(d0);
-            v[cc][b + h][j + 1] = __float_as_uint(d1);
-          }
+            for (int j = 0; j < 32; j += 2) {
+              const uint64_t x = f2_pack(__uint_as_float(v[cc][b][j]), __uint_as_float(v[cc][b][j + 1]));
+              const uint64_t y = f2_pack(__uint_as_float(v[cc][b + h][j]), __uint_as_float(v[cc][b + h][j + 1]));
+              float s0, s1, d0, d1;
+              f2_unpack(f2_add(x, y), s0, s1);
+              f2_unpack(f2_sub(x, y), d0, d1);
+              v[cc][b][j] = __float_as_uint(s0);
+              v[cc][b][j + 1] = __float_as_uint(s1);
+              v[cc][b + h][j] = __float_as_uint(d0);
+              v[cc][b + h][j + 1] = __float_as_uint(d1);
+            }
+  }
 }
 
 // max |x'| over the thread's row of a product in tensor memory (tb: the warp's
