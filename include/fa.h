@@ -93,10 +93,16 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  *         blocks of ceil(ceil(Nk/128)/n_split) key tiles of 128 keys (the last ones
  *         may be empty); 0 = automatic: with fewer query blocks (of 128 or 256
  *         rows) than SMs, fa_fwd_splitkv_splits(B, H, Nq, Nk, d) blocks for every
- *         query block, else no split.
+ *         query block; else, without causal masking, when the last round of
+ *         query blocks over the SMs (one CTA per SM) is at most half full and a
+ *         head has at least 4 key tiles, each block of that round as 2-4 pieces
+ *         over disjoint key tiles, merged by their LSEs inside the kernel (the
+ *         result does not depend on the order the pieces finish in); else no
+ *         split.
  * workspace  device, >= fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split)
  *         bytes, 256-byte aligned, owned by the caller (may be NULL if that is 0);
- *         overwritten. Calls that overlap on the GPU must not share it.
+ *         overwritten; its contents before the call do not matter. Calls that
+ *         overlap on the GPU must not share it.
  * Errors: FA_ERR_INVALID_ARG (also: workspace missing or too small),
  *         FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
  */

@@ -75,6 +75,20 @@ struct FwdCfg {
   static constexpr int NSLOT = (RING_BUDGET / SLOT) > 6 ? 6 : (RING_BUDGET / SLOT);
   static constexpr int ROT_OP = QROT ? HadCfg<D>::HMAT : 0;  // the rotation operand (QROT)
   static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + ROT_OP + NSLOT * SLOT;
+  // O staging (direct-mode epilogue): OST_COLS columns of a query tile's O as
+  // bf16, 64-column boxes of 128 rows with the 128-byte swizzle, written to
+  // global memory by TMA stores; D / OST_COLS rounds per tile. For the bf16
+  // kernels, where it fits beside the rest, without causal masking
+  // (fwd_ostage). (Measured on B200: +4% at N = 512, neutral at N >= 4096 for
+  // non-causal bf16; 1-2% slower for causal launches and for the e4m3-QK kernel
+  // at B=2, H=16, N=8192, which keep their per-row stores.)
+  static constexpr int OST_COLS = D < 128 ? D : 128;
+  static constexpr int OST_ROUNDS = D / OST_COLS;
+  static constexpr int OST_BOXES = OST_COLS / 64;
+  static constexpr bool OST_FITS = !QK_FP8 && SMEM_BYTES + BM * OST_COLS * 2 <= 225 * 1024;
+  static constexpr int OST_BYTES = OST_FITS ? BM * OST_COLS * 2 : 0;
+  // dynamic shared memory of a launch (direct: O goes through the staging buffer)
+  static constexpr int smem_bytes(bool direct) { return SMEM_BYTES + (direct ? OST_BYTES : 0); }
   static constexpr int SOFTMAX_WARPS = 4 * NQ;
   static constexpr int MMA_WARP = SOFTMAX_WARPS;
   static constexpr int TMA_WARP = SOFTMAX_WARPS + 1;
@@ -100,6 +114,12 @@ struct FwdCfg {
   // Two co-resident CTAs must not both want all 512 TMEM columns.
   static_assert(SMEM_BYTES > 114 * 1024 || TMEM_COLS <= 256, "TMEM of co-resident CTAs");
 };
+
+// Whether a forward kernel writes O through the staging buffer (FwdCfg::OST_*).
+template <typename C, bool CAUSAL, bool PARTIAL, bool DEC>
+__host__ __device__ constexpr bool fwd_ostage() {
+  return C::OST_FITS && !CAUSAL && !PARTIAL && !DEC;
+}
 
 struct FwdParams {
   __nv_bfloat16* o;          // [BH][Nq][D]; null in partial mode
@@ -134,12 +154,38 @@ struct FwdParams {
   // r * gridDim.x + c in even rounds r, r * gridDim.x + gridDim.x - 1 - c in odd
   // ones, which balances work that decreases with i
   int snake;
+  // Tail split (direct mode, non-causal, persistent): query blocks n_full ..
+  // (units - 1), the blocks of a mostly empty last round, are computed as
+  // tail_split pieces of tail_tiles key tiles each, as items n_full + k with
+  // k = (block - n_full) * tail_split + piece, so that the round's CTAs share
+  // them. Each warp of a piece writes its rows' O (fp32, normalised over the
+  // piece's keys; [D/4][128][4] per piece and tile, so a warp's stores are
+  // contiguous) and base-2 LSE to tail_o / tail_lse, then takes a ticket on its
+  // group's word of tail_cnt (bits 8-63: tail_tag, a 56-bit value new for every
+  // launch, so a word left by an aborted launch, or never written, counts as
+  // zero; bits 0-7: pieces done). The warp whose ticket completes the group sets
+  // the word back to zero, merges the pieces by their LSEs, in piece order
+  // whichever piece it is, and writes O and the LSE; no warp waits for another.
+  // n_full = number of query blocks (tail_split = 0) when there is no tail split.
+  int n_full;
+  int tail_split, tail_tiles;
+  unsigned long long tail_tag;
+  float* tail_o;
+  float* tail_lse;
+  unsigned long long* tail_cnt;
 };
+
+// Tail-split workspace of one (query tile, piece): the piece's normalised O,
+// then (separately) its LSE per row.
+template <int D>
+__host__ __device__ constexpr size_t tail_o_floats() { return static_cast<size_t>(128) * D; }
+constexpr int kTailMaxSplit = 4;
 
 // One work item of a CTA: head, key split, first query row, first key tile and
 // the key tiles its query tiles step through.
 struct FwdItem {
   int bh, sp, q0, kt0, n_kv0, n_kv1, n_kv;
+  int tail;  // tail-split query block index (its pieces' group), -1 if the item is whole
 };
 
 #ifndef FA_MMA_WAIT_SLEEP_NS
@@ -149,6 +195,13 @@ struct FwdItem {
 // on the critical path, but a polling warp also takes issue slots from the two
 // softmax warps on its sub-partition.
 constexpr uint32_t kMmaWaitSleepNs = FA_MMA_WAIT_SLEEP_NS;
+
+// Longest item (in key tiles) whose Q buffer is released right after its last
+// S product rather than after its last P V product (non-causal launches).
+// Measured on B200 (interleaved A/B): the early release gains 2-7% at N =
+// 512-2048; on longer items it gained nothing, and on causal launches (whose
+// snake order ends with short items) it cost 2-4%.
+constexpr int kEarlyQMaxTiles = 24;
 
 // Exponentials of one 32-key chunk of a row of S: p = 2^(x*s - m), packed to
 // bf16 pairs into pk[0..15]; accumulates the fp32 weights, with ROUND also the
@@ -434,6 +487,183 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
     p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = lse;
 }
 
+// Epilogue of a tail-split piece for one warp's 32 query rows (see FwdParams):
+// the piece's O (TMEM, weights relative to m_ref, summing to l_round) and LSE
+// go to the workspace, the warp takes a ticket, and the warp whose ticket
+// completes its group merges every piece by its LSE (the same combination as
+// the blocks of a split: O = sum_k 2^(lse_k - L) O_k, L = log2 sum_k 2^lse_k)
+// into the bf16 output and the natural-log LSE. The merge takes the pieces in
+// index order, its own normalised O recomputed with the rounding it was stored
+// with, so the result does not depend on which piece finished last. The CAS
+// loop is not a wait: each failed attempt means another piece's ticket went in,
+// so it ends within tail_split attempts; the bound only guards the status path.
+template <int D, int NQ>
+__device__ __forceinline__ void tail_piece_epilogue(const FwdParams& p, const FwdItem& w, int t, uint32_t warp_in_tile,
+                                                 uint32_t lane, uint32_t tO, int r, int qrow, float m_ref,
+                                                 float l_exact, float l_round, DevStatus* st) {
+  const int ns = p.tail_split;
+  const size_t grp = static_cast<size_t>(w.tail) * NQ + t;  // (tail block, query tile)
+  float* const o_base = p.tail_o + grp * ns * tail_o_floats<D>();
+  float* const l_base = p.tail_lse + grp * ns * 128;
+  const float inv_l = 1.0f / l_round;
+  const float lse2 = m_ref + __log2f(l_exact);  // base 2
+  float4* const mine = reinterpret_cast<float4*>(o_base + w.sp * tail_o_floats<D>());
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t ov[32];
+    tmem_ld32(tO + c0, ov);
+    tmem_wait_ld_dep32(ov);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      mine[(c0 / 4 + i) * 128 + r] = make_float4(
+          __fmul_rn(__uint_as_float(ov[4 * i]), inv_l), __fmul_rn(__uint_as_float(ov[4 * i + 1]), inv_l),
+          __fmul_rn(__uint_as_float(ov[4 * i + 2]), inv_l), __fmul_rn(__uint_as_float(ov[4 * i + 3]), inv_l));
+  }
+  l_base[w.sp * 128 + r] = lse2;
+  __threadfence();  // this lane's results before the ticket (release side)
+  __syncwarp();
+  unsigned int done = 0;
+  if (lane == 0) {
+    unsigned long long* cnt = p.tail_cnt + grp * 4 + warp_in_tile;
+    unsigned long long cur = atomicAdd(cnt, 0ull);
+    for (int a = 0; a < 64 && done == 0; ++a) {
+      const unsigned long long base = (cur >> 8) == p.tail_tag ? cur : (p.tail_tag << 8);
+      const unsigned long long got = atomicCAS(cnt, cur, base + 1ull);
+      if (got == cur) done = static_cast<unsigned int>((base + 1ull) & 0xffull);
+      cur = got;
+    }
+    if (done == 0 && atomicCAS(&st->code, 0u, 5u /*FA_ERR_TIMEOUT*/) == 0u) {
+      st->site = 45;
+      st->block = blockIdx.x;
+    }
+  }
+  done = __shfl_sync(0xffffffffu, done, 0);
+  if (done != static_cast<unsigned int>(ns)) return;  // warp-uniform
+  // Every piece has its ticket: the word goes back to zero, so that the next
+  // launch starts from zero even with this launch's tag (a replayed CUDA graph
+  // launches with the parameters it was captured with).
+  if (lane == 0) atomicExch(p.tail_cnt + grp * 4 + warp_in_tile, 0ull);
+  __threadfence();  // acquire side: the other pieces' results, read through L2 below
+  float lk[kTailMaxSplit], wk[kTailMaxSplit];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kTailMaxSplit; ++k) {
+    lk[k] = k < ns ? (k == w.sp ? lse2 : __ldcg(l_base + k * 128 + r)) : -INFINITY;
+    mx = fmaxf(mx, lk[k]);
+  }
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kTailMaxSplit; ++k) sum += k < ns ? exp2f(lk[k] - mx) : 0.f;
+  const float L = mx + log2f(sum);
+#pragma unroll
+  for (int k = 0; k < kTailMaxSplit; ++k) wk[k] = k < ns ? exp2f(lk[k] - L) : 0.f;
+  const bool in_range = qrow < p.Nq;
+  __nv_bfloat16* orow = p.o + (static_cast<size_t>(w.bh) * p.Nq + (in_range ? qrow : 0)) * D;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t ov[32];
+    tmem_ld32(tO + c0, ov);
+    tmem_wait_ld_dep32(ov);
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kTailMaxSplit; ++k) {
+      if (k >= ns) continue;
+      const float4* src = reinterpret_cast<const float4*>(o_base + k * tail_o_floats<D>());
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 v;
+        if (k == w.sp) {
+          v = make_float4(__fmul_rn(__uint_as_float(ov[4 * i]), inv_l), __fmul_rn(__uint_as_float(ov[4 * i + 1]), inv_l),
+                          __fmul_rn(__uint_as_float(ov[4 * i + 2]), inv_l),
+                          __fmul_rn(__uint_as_float(ov[4 * i + 3]), inv_l));
+        } else {
+          v = __ldcg(src + (c0 / 4 + i) * 128 + r);
+        }
+        acc[4 * i] = __fmaf_rn(wk[k], v.x, acc[4 * i]);
+        acc[4 * i + 1] = __fmaf_rn(wk[k], v.y, acc[4 * i + 1]);
+        acc[4 * i + 2] = __fmaf_rn(wk[k], v.z, acc[4 * i + 2]);
+        acc[4 * i + 3] = __fmaf_rn(wk[k], v.w, acc[4 * i + 3]);
+      }
+    }
+    if (in_range) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                            pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]), pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+    }
+  }
+  if (in_range && p.lse != nullptr)
+    p.lse[static_cast<size_t>(w.bh) * p.Nq + qrow] = L * 0.69314718055994530942f;
+}
+
+// Direct-mode epilogue of one warp's 32 rows of query tile t through the
+// staging buffer (FwdCfg::OST_*): O / l in bf16 into 64-column boxes of 128 rows
+// (128-byte swizzle), written by TMA stores that one thread of the tile issues
+// (whole rows at once, rows past Nq clipped), then the LSE. The tiles take turns
+// on the buffer (use u = (round * NQ + t) * OST_ROUNDS + part waits for the
+// stores of use u - 1 to have read it); a tile with no rows takes its turn
+// without writing, so the turns stay in step. Kept out of line: the softmax
+// loop's registers and code are not shared with it. Returns ok.
+template <int D, int NQ, typename C>
+__device__ __noinline__ bool staged_o_epilogue(const CUtensorMap* tmO, uint8_t* sOst, uint64_t* bar_ost,
+                                               uint64_t* bar_ofree, volatile int* abort_flag, DevStatus* st,
+                                               float* lse, int Nq, uint32_t tO, int r, uint32_t lane, uint32_t warp,
+                                               int t, int round, bool has, bool ok, float l_round, float l_exact,
+                                               float m_ref, int q0, int bh, int qrow) {
+  const bool issuer = (warp & 3u) == 0 && lane == 0;
+  const float inv_l = has ? 1.0f / l_round : 0.f;
+  if (ok && has) tc_fence_after();
+#pragma unroll 1
+  for (int part = 0; part < C::OST_ROUNDS && ok; ++part) {
+    const int u = (round * NQ + t) * C::OST_ROUNDS + part;  // the buffer's use
+    if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_ofree, (u - 1) & 1, abort_flag, st, 46));
+    if (!ok) break;
+    if (has) {
+#pragma unroll 1
+      for (int cc = 0; cc < C::OST_COLS; cc += 32) {
+        uint32_t ov[32];
+        tmem_ld32(tO + part * C::OST_COLS + cc, ov);
+        tmem_wait_ld_dep32(ov);
+        uint32_t q[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          q[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        // row r of the 64-column box holding these columns; 16-byte chunk c of
+        // a row sits at c ^ (r mod 8) (the 128-byte swizzle)
+        uint8_t* brow = sOst + (cc / 64) * (C::BM * 128) + r * 128;
+        const int c0 = (cc % 64) / 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(brow + (((c0 + i) ^ (r & 7)) << 4)) =
+              make_uint4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]);
+      }
+      fence_proxy_async_shared();  // the TMA store reads the buffer through the async proxy
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar_ost[t]);
+    if (issuer) {
+      ok = mbar_wait(&bar_ost[t], (round * C::OST_ROUNDS + part) & 1, abort_flag, st, 47 + t);
+      if (ok) {
+        if (has) {
+#pragma unroll
+          for (int b = 0; b < C::OST_BOXES; ++b)
+            tma_store_3d(tmO, sOst + b * (C::BM * 128), part * C::OST_COLS + 64 * b, q0 + t * C::BM, bh);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        mbar_arrive(bar_ofree);
+      }
+    }
+    ok = __all_sync(0xffffffffu, ok);
+  }
+  if (ok && has && qrow < Nq && lse != nullptr)
+    lse[static_cast<size_t>(bh) * Nq + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
+  return ok;
+}
+
 // PARTIAL: the CTA's keys are one block of a split (p.n_split blocks) and it
 // writes fp32 partial results (o_part, lse_part) instead of O and LSE.
 //
@@ -449,16 +679,23 @@ __device__ __forceinline__ void decode_softmax(const P& p, uint32_t tbase, uint3
 template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC, bool QROT = false>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, QK_FP8, QROT>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const FwdParams p) {
   using C = FwdCfg<D, NQ, QK_FP8, QROT>;
   static_assert(!DEC || NQ == 1, "the decode layout uses one query tile");
   static_assert(!QROT || (!PARTIAL && !DEC && NQ == 2), "in-kernel Q quantisation: square launches only");
   static_assert(!DEC || C::NSLOT * C::SLOT >= 3 * 32 * D * 4, "decode merge buffer lives in the ring");
+  // kernels that may take a tail split (the host sets it up only for these)
+  constexpr bool TAIL = !PARTIAL && !DEC && !CAUSAL && !QROT;
+  // direct-mode O through the staging buffer and TMA stores (tmO: O as
+  // [BH][Nq][D] bf16, 64 x 128 boxes, 128-byte swizzle); non-causal only
+  constexpr bool OSTAGE = fwd_ostage<C, CAUSAL, PARTIAL, DEC>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                // NQ tiles
   uint8_t* sRot = smem + NQ * C::Q_TILE;             // QROT: the rotation operand
   uint8_t* sRing = smem + NQ * C::Q_TILE + C::ROT_OP;  // NSLOT slots
+  uint8_t* sOst = sRing + C::NSLOT * C::SLOT;          // OSTAGE: O staging
 
   __shared__ __align__(8) uint64_t bar_full[C::NSLOT], bar_empty[C::NSLOT];
   // bar_qfree: the S MMAs that read the current item's Q tiles are done (the
@@ -469,6 +706,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // tile t is in e4m3 (its warpgroup has converted it)
   // bar_qamax[t]: the four warps of tile t's warpgroup have posted their maxima
   __shared__ __align__(8) uint64_t bar_rot[NQ], bar_qready[NQ], bar_qamax[NQ];
+  // OSTAGE: bar_ost[t]: the four warps of tile t have written their rows of the
+  // staging buffer; bar_ofree: the TMA stores of the buffer's last use have read
+  // it (the tiles use it in turn: use u = (round * NQ + t) * OST_ROUNDS + part)
+  __shared__ __align__(8) uint64_t bar_ost[NQ], bar_ofree;
   __shared__ float qrot_red[NQ][4];  // per-warp maxima of each tile
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -490,20 +731,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   auto item_at = [&](int it) {
     FwdItem w;
     const int n_split = PARTIAL ? p.n_split : 1;
-    const int unit = PARTIAL ? it / n_split : it;  // query block
+    int unit = PARTIAL ? it / n_split : it;  // query block
     w.sp = PARTIAL ? it % n_split : 0;
+    w.tail = -1;
+    int span = PARTIAL ? p.split_tiles : 0;  // key tiles of a split block (0: all)
+    if constexpr (TAIL) {
+      if (it >= p.n_full) {
+        const int k = it - p.n_full;
+        w.tail = k / p.tail_split;
+        w.sp = k - w.tail * p.tail_split;
+        unit = p.n_full + w.tail;
+        span = p.tail_tiles;
+      }
+    }
     w.bh = p.snake ? unit % p.BH : unit / p.n_qb;
     int qb = p.snake ? unit / p.BH : unit % p.n_qb;
     if (CAUSAL) qb = p.n_qb - 1 - qb;
     w.q0 = qb * NQ * C::BM;
-    w.kt0 = PARTIAL ? w.sp * p.split_tiles : 0;
+    w.kt0 = w.sp * span;
     auto n_kv_of = [&](int t) {
       const int row0 = w.q0 + t * C::BM;
       if (row0 >= p.Nq) return 0;
       const int end = CAUSAL ? min(p.Nk, min(p.Nq, row0 + C::BM) + p.causal_off) : p.Nk;  // keys [0, end)
       const int tiles = (end + C::BN - 1) / C::BN;
-      if (!PARTIAL) return tiles;
-      return max(0, min(tiles, w.kt0 + p.split_tiles) - w.kt0);
+      if (span == 0) return tiles;
+      return max(0, min(tiles, w.kt0 + span) - w.kt0);
     };
     w.n_kv0 = n_kv_of(0);
     w.n_kv1 = NQ > 1 ? n_kv_of(NQ - 1) : w.n_kv0;
@@ -520,7 +772,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(&bar_q, 1);
     mbar_init(&bar_qfree, 1);
     mbar_init(&bar_drain, 1);
+    mbar_init(&bar_ofree, 1);
     for (int t = 0; t < NQ; ++t) {
+      mbar_init(&bar_ost[t], 4);
       mbar_init(&bar_s[t], 1);
       mbar_init(&bar_p[t], 4);  // one arrival per softmax warp of the tile
       mbar_init(&bar_o[t], 1);
@@ -626,12 +880,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      for (int j = 0; j <= n_kv && ok; ++j) {
+      // Step j of the item: P V of key tile j - 1 (j > 0), then S of key tile j
+      // (j < n_kv), for each query tile. Returns false on an abort.
+      auto issue_step = [&](int j) -> bool {
+        bool ok = true;
         const int kpos = pos + 2 * j, vpos = pos + 2 * j - 1;
         const int kslot = kpos % C::NSLOT, vslot = (vpos + C::NSLOT) % C::NSLOT;
         if (j < n_kv) ok = mbar_wait(&bar_full[kslot], (kpos / C::NSLOT) & 1, &abort_flag, st, 21);
         if (ok && j > 0) ok = mbar_wait(&bar_full[vslot], (vpos / C::NSLOT) & 1, &abort_flag, st, 22);
-        if (!ok) break;
+        if (!ok) return false;
         tc_fence_after();
         for (int t = 0; t < NQ && ok; ++t) {
           const int n_kv_t = n_kv_at(t);
@@ -676,12 +933,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mma_commit(&bar_s[t]);
           }
         }
-        if (!ok) break;
+        if (!ok) return false;
         if (j > 0) mma_commit(&bar_empty[vslot]);
         if (j < n_kv) mma_commit(&bar_empty[kslot]);
-      }
+        return true;
+      };
+      for (int j = 0; j < n_kv && ok; ++j) ok = issue_step(j);
+      // bar_qfree: done when this item's S MMAs (the readers of sQ) are. For a
+      // short item it is committed before the last P V products, so that the
+      // next item's Q load overlaps them.
+      const bool early_q = !CAUSAL && n_kv > 0 && n_kv <= kEarlyQMaxTiles;
+      if (ok && early_q) mma_commit(&bar_qfree);
+      if (ok) ok = issue_step(n_kv);
       if (!ok) break;
-      mma_commit(&bar_qfree);  // done when this item's S MMAs (readers of sQ) are
+      if (!early_q) mma_commit(&bar_qfree);
       pos += 2 * n_kv;
       }  // items
       // Drain: TMEM is freed below only after every issued MMA has finished.
@@ -876,6 +1141,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (in_range)
           p.lse_part[prow] = empty ? -INFINITY : (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
       }
+    } else if (TAIL && w.tail >= 0) {
+      if (ok && n_kv_t > 0) {
+        tc_fence_after();
+        tail_piece_epilogue<D, NQ>(p, w, t, warp & 3u, lane, tO, r, qrow, m_ref, l_exact, l_round, st);
+      }
+    } else if (OSTAGE) {
+      ok = staged_o_epilogue<D, NQ, C>(&tmO, sOst, bar_ost, &bar_ofree, &abort_flag, st, p.lse, p.Nq, tO, r, lane,
+                                        warp, t, round, n_kv_t > 0, ok, l_round, l_exact, m_ref, q0, bh, qrow);
     } else if (ok && n_kv_t > 0) {
       tc_fence_after();
       const float inv_l = 1.0f / l_round;
@@ -899,6 +1172,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = (m_ref + __log2f(l_exact)) * 0.69314718055994530942f;
     }
     }  // items
+    // the O stores this thread issued complete before the CTA exits
+    if constexpr (OSTAGE) {
+      if ((warp & 3u) == 0 && lane == 0) bulk_wait_all();
+    }
     }  // not DEC
   }
 

@@ -2,11 +2,14 @@
 // maps, and the launches of the attention and quantisation kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <random>
 
 #include "../../include/fa.h"
 #include "attn_bwd.cuh"
@@ -54,6 +57,13 @@ struct FwdArgs {
   int qrot_rotate = 0;
   const float* qrot_signs = nullptr;
   float* dq_out = nullptr;
+  // tail split of a direct, non-causal persistent launch (FwdParams): 0 = none
+  int tail_split = 0;
+  int tail_tiles = 0;
+  long long n_full = 0;
+  float* tail_o = nullptr;
+  float* tail_lse = nullptr;
+  unsigned long long* tail_cnt = nullptr;
 };
 
 constexpr int kKeyTile = 128;  // keys per K/V tile (FwdCfg::BN)
@@ -77,6 +87,27 @@ constexpr bool kPersistent = FA_PERSISTENT != 0;
 #define FA_PERSIST_CAUSAL 1
 #endif
 constexpr bool kPersistCausal = FA_PERSIST_CAUSAL != 0;
+#ifndef FA_TAIL_SPLIT
+#define FA_TAIL_SPLIT 1
+#endif
+constexpr bool kTailSplit = FA_TAIL_SPLIT != 0;
+
+// A new 56-bit tail-split tag for every launch that takes one: a per-process
+// random start plus a launch count, never 0 (the tag of a zeroed word), so that a
+// ticket word left by another launch, or never written, matches it only by a
+// 2^-56 chance.
+unsigned long long next_tail_tag() {
+  static std::atomic<unsigned long long> count{0};
+  static const unsigned long long start = [] {
+    std::random_device rd;
+    return (static_cast<unsigned long long>(rd()) << 32) ^ rd() ^
+           static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count());
+  }();
+  for (;;) {
+    const unsigned long long t = (start + count.fetch_add(1ull)) & ((1ull << 56) - 1ull);
+    if (t != 0ull) return t;
+  }
+}
 
 template <int D, int NQ, bool CAUSAL, bool QK_FP8, bool PARTIAL, bool DEC, bool QROT = false>
 fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
@@ -90,9 +121,18 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   if (!q_ok || !fa::make_tmap_3d(&tmK, a.k, qk_type, C::EQK, D, a.Nk, BH, 128 / C::EQK, C::BN) ||
       !fa::make_tmap_3d(&tmV, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nk, BH, 64, C::BN))
     return FA_ERR_CUDA;
+  // direct-mode O goes through shared memory and TMA stores where the staging
+  // buffer fits (FwdCfg::OST_*); the map is unused otherwise
+  constexpr bool kOStage = fa::fwd_ostage<C, CAUSAL, PARTIAL, DEC>();
+  CUtensorMap tmO = tmV;
+  if constexpr (kOStage) {
+    if (!fa::make_tmap_3d(&tmO, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.Nq, BH, 64, C::BM))
+      return FA_ERR_CUDA;
+  }
+  constexpr int kSmem = C::smem_bytes(kOStage);
   auto kernel = fa::attn_fwd_kernel<D, NQ, CAUSAL, QK_FP8, PARTIAL, DEC, QROT>;
   static unsigned long long smem_done = 0;
-  if (!set_smem_once(kernel, C::SMEM_BYTES, &smem_done)) return FA_ERR_CUDA;
+  if (!set_smem_once(kernel, kSmem, &smem_done)) return FA_ERR_CUDA;
   if constexpr (C::SPLIT_REGS) {
     // The kernel moves registers between warpgroups with setmaxnreg; that only
     // completes if the block was launched with the register count the split was
@@ -136,8 +176,30 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   p.split_tiles = (key_tiles(a.Nk) + a.n_split - 1) / a.n_split;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const long long units = static_cast<long long>(p.n_qb) * BH;
-  const long long items = units * (PARTIAL ? a.n_split : 1);
+  long long items = units * (PARTIAL ? a.n_split : 1);
   if (items < 1) return FA_OK;
+  p.n_full = static_cast<int>(units);
+  p.tail_split = 0;
+  p.tail_tiles = 0;
+  p.tail_tag = 0;
+  p.tail_o = nullptr;
+  p.tail_lse = nullptr;
+  p.tail_cnt = nullptr;
+  constexpr bool kTailKernel = !PARTIAL && !DEC && !CAUSAL && !QROT;
+  if (kTailKernel && a.tail_split >= 2) {
+    if (a.tail_split > fa::kTailMaxSplit || a.n_full < 0 || a.n_full >= units || a.tail_o == nullptr ||
+        a.tail_lse == nullptr || a.tail_cnt == nullptr)
+      return FA_ERR_INVALID_ARG;
+    p.n_full = static_cast<int>(a.n_full);
+    p.tail_split = a.tail_split;
+    p.tail_tiles = a.tail_tiles;
+    p.tail_tag = next_tail_tag();
+    p.tail_o = a.tail_o;
+    p.tail_lse = a.tail_lse;
+    p.tail_cnt = a.tail_cnt;
+    items = a.n_full + (units - a.n_full) * a.tail_split;
+    if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  }
   p.n_items = static_cast<int>(items);
   // Persistent: at most one CTA per SM, each looping over work items, so the
   // next item's Q load and first S MMA overlap the current item's last steps and
@@ -154,7 +216,7 @@ fa_status launch_fwd(const FwdArgs& a, cudaStream_t stream) {
     const long long sms = device_sms();
     if (grid > sms) grid = sms;
   }
-  kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  kernel<<<static_cast<unsigned>(grid), C::THREADS, kSmem, stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -277,29 +339,72 @@ int auto_splits(int B, int H, int Nq, int Nk, int d) {
 }
 
 // The automatic schedule of fa_fwd_splitkv (n_split = 0): with fewer query
-// blocks than SMs, every block's keys are split (auto_splits) and merged; else one
-// CTA per query block. (Measured on B200 and dropped: splitting only the blocks
-// of a mostly empty last wave, either by keys with the merge in the kernel or as
-// one-tile CTAs, was slower than leaving that wave as it is: the split CTAs' fp32
-// partial stores and merge, or the one-tile CTAs' unhidden softmax, cost as much
-// as the wave they save.)
+// blocks than SMs, every block's keys are split (auto_splits) and merged by a
+// second launch; else one persistent CTA per SM over the query blocks, with a
+// tail split: without causal masking, when the launch's last round is at most
+// half full, the keys of that round's query blocks are split into tail_split
+// pieces (as many as the round's idle CTAs allow, at most four), merged by the
+// kernel itself (FwdParams). Measured on B200 at B=4, H=16, N=2048, d=128
+// (68 of 512 blocks in the last round, two pieces each): +3-6%. (An earlier
+// form, with one row per thread in the pieces' fp32 stores and one CTA per
+// work item, was slower than no split.)
 struct Plan {
   int n_split = 1;
   int nq = 1;
   long long units = 0;
+  int tail_split = 0;
+  int tail_tiles = 0;
+  long long n_full = 0;
 };
 
+// Fewest key tiles per query block for a tail split to pay for its merge.
+constexpr int kTailMinTiles = 4;
+
 Plan plan_fwd(int B, int H, int Nq, int Nk, int d, bool causal) {
-  (void)causal;
   Plan pl;
   pl.nq = nq_for(d, Nq);
   pl.units = static_cast<long long>(B) * H * ((Nq + pl.nq * 128 - 1) / (pl.nq * 128));
   const int sms = device_sms();
-  if (pl.units < sms) pl.n_split = pick_splits(pl.units, key_tiles(Nk), sms);
+  if (pl.units < sms) {
+    pl.n_split = pick_splits(pl.units, key_tiles(Nk), sms);
+  } else if (kTailSplit && kPersistent && !causal && !(pl.nq == 1 && Nq <= kDecodeMaxQ)) {
+    const long long full = pl.units / sms * sms, tail = pl.units - full;
+    const int kt = key_tiles(Nk);
+    if (tail > 0 && 2 * tail <= sms && kt >= kTailMinTiles) {
+      long long ns = sms / tail;
+      if (ns > fa::kTailMaxSplit) ns = fa::kTailMaxSplit;
+      if (ns > kt) ns = kt;
+      const int span = static_cast<int>((kt + ns - 1) / ns);
+      ns = (kt + span - 1) / span;  // no empty piece
+      if (ns >= 2) {
+        pl.tail_split = static_cast<int>(ns);
+        pl.tail_tiles = span;
+        pl.n_full = full;
+      }
+    }
+  }
   return pl;
 }
 
+// Tail-split workspace: the pieces' O, their LSEs, the ticket words; each part
+// 256-byte aligned.
+struct TailLayout {
+  size_t o = 0, lse = 0, cnt = 0, bytes = 0;
+};
+TailLayout tail_layout(const Plan& pl, int d) {
+  TailLayout t;
+  if (pl.tail_split < 2) return t;
+  const size_t groups = static_cast<size_t>(pl.units - pl.n_full) * pl.nq;  // (tail block, query tile)
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  t.o = 0;
+  t.lse = up(groups * pl.tail_split * 128 * d * sizeof(float));
+  t.cnt = t.lse + up(groups * pl.tail_split * 128 * sizeof(float));
+  t.bytes = t.cnt + up(groups * 4 * sizeof(unsigned long long));
+  return t;
+}
+
 size_t plan_bytes(const Plan& pl, int B, int H, int Nq, int d) {
+  if (pl.tail_split >= 2) return tail_layout(pl, d).bytes;
   return pl.n_split <= 1 ? 0 : part_bytes(B, H, Nq, d, pl.n_split);
 }
 
@@ -542,6 +647,18 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (n_split == 1) {
     FwdArgs a{q, k, v, o, lse, nullptr, nullptr, B, H, Nq, Nk, d, causal != 0, scale, qk_dtype, descale_qk, 1};
+    if (pl.tail_split >= 2) {
+      const TailLayout tl = tail_layout(pl, d);
+      if (workspace == nullptr || workspace_bytes < tl.bytes) return FA_ERR_INVALID_ARG;
+      if (!aligned(workspace, 256)) return FA_ERR_ALIGNMENT;
+      char* ws = static_cast<char*>(workspace);
+      a.tail_split = pl.tail_split;
+      a.tail_tiles = pl.tail_tiles;
+      a.n_full = pl.n_full;
+      a.tail_o = reinterpret_cast<float*>(ws + tl.o);
+      a.tail_lse = reinterpret_cast<float*>(ws + tl.lse);
+      a.tail_cnt = reinterpret_cast<unsigned long long*>(ws + tl.cnt);
+    }
     return dispatch_fwd(a, s);
   }
   if (workspace == nullptr || workspace_bytes < part_bytes(B, H, Nq, d, n_split)) return FA_ERR_INVALID_ARG;

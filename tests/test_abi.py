@@ -113,6 +113,53 @@ def test_splitkv_argument_errors(lib):
     assert lib.fa_fwd_splitkv_workspace_bytes(0, 1, 1, 300, 128, 2) == 0
 
 
+def _sms():
+    import torch
+    return torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+
+
+def _tail_plan(B, H, N, d, sms):
+    """The automatic schedule's tail split, restated: without causal masking, a
+    persistent launch whose last round is at most half full splits that round's
+    query blocks into min(4, sms // tail, key tiles) pieces of equal key-tile
+    spans (no empty piece). Returns (pieces, tail blocks, query tiles per block)."""
+    nq = 2 if (d <= 128 and N > 128) else 1
+    units = B * H * -(-N // (128 * nq))
+    tiles = -(-N // 128)
+    tail = units % sms
+    if units < sms or tail == 0 or 2 * tail > sms or tiles < 4 or (nq == 1 and N <= 32):
+        return 0, 0, nq
+    ns = min(4, sms // tail, tiles)
+    span = -(-tiles // ns)
+    ns = -(-tiles // span)
+    return (ns if ns >= 2 else 0), tail, nq
+
+
+def test_tail_split_workspace(lib):
+    # B=4, H=16, N=2048, d=128: 512 two-tile query blocks on 148 SMs leave 68 for
+    # a last round: two pieces of 8 key tiles each
+    sms = _sms()
+    for (B, H, N, d) in [(4, 16, 2048, 128), (1, 19, 2048, 128), (2, 20, 1000, 64), (2, 13, 700, 256),
+                         (1, 16, 16384, 128), (8, 16, 2048, 128)]:
+        ns, tail, nq = _tail_plan(B, H, N, d, sms)
+        up = lambda x: (x + 255) // 256 * 256
+        groups = tail * nq
+        want = up(groups * ns * 128 * d * 4) + up(groups * ns * 128 * 4) + up(groups * 4 * 8) if ns else 0
+        if ns == 0 and B * H * -(-N // (128 * nq)) < sms:
+            continue  # a key split instead
+        assert lib.fa_fwd_splitkv_workspace_bytes(B, H, N, N, d, 0) == want, (B, H, N, d)
+    if sms == 148:
+        assert _tail_plan(4, 16, 2048, 128, sms)[:2] == (2, 68)
+        assert _tail_plan(2, 13, 700, 256, sms)[:2] == (3, 8)
+        need = lib.fa_fwd_splitkv_workspace_bytes(4, 16, 2048, 2048, 128, 0)
+        assert need == 17969408
+        # the automatic schedule then needs the workspace, 256-byte aligned
+        big = dict(B=4, H=16, Nq=2048, Nk=2048, ns=0)
+        assert _skv(lib, **big) == binding.FA_ERR_INVALID_ARG
+        assert _skv(lib, ws=A, wsb=need - 1, **big) == binding.FA_ERR_INVALID_ARG
+        assert _skv(lib, ws=A + 16, wsb=need, **big) == binding.FA_ERR_ALIGNMENT
+
+
 def test_partial_and_merge_argument_errors(lib):
     part = lambda **kw: lib.fa_fwd_partial(kw.get("q", A), A, A, kw.get("op", A), kw.get("lp", A), 1, 1, 4, 64, 128,
                                            kw.get("causal", 0), 0.1, 0, None, kw.get("ns", 1), None)
