@@ -126,7 +126,10 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmdK,
+                    const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
+  (void)tmdK;  // dK and dV by per-row stores here (the d = 128 kernel stages them)
+  (void)tmdV;
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0u) {
@@ -521,7 +524,7 @@ struct BwdPpCfg {
   static constexpr int OFF_STAGE = OFF_DS + DS_TILE;
   static constexpr int OFF_LD = OFF_STAGE + NST * STAGE;
   static constexpr int OFF_BAR = OFF_LD + NST * LD_BYTES;
-  static constexpr int N_BARS = 1 + 2 * NST + 2 * 5 + 2;
+  static constexpr int N_BARS = 1 + 2 * NST + 2 * 5 + 2 + 2;
   static constexpr int SMEM_BYTES = OFF_BAR + 8 * N_BARS + 16;
   static constexpr int THREADS = 384;
   static constexpr int MMA_WARP = 8;
@@ -538,7 +541,8 @@ template <bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmdK,
+                       const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using C = BwdPpCfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -567,6 +571,7 @@ __global__ void __launch_bounds__(384, 1)
   auto bar_dqfree = [&](int h) { return hb + 5 * h + 4; };  // dQᵀ_h read out
   uint64_t* bar_done = hb + 10;                         // dK, dV complete
   uint64_t* bar_drain = hb + 11;
+  auto bar_epi = [&](int h) { return hb + 12 + h; };    // warpgroup h's dK, dV rows staged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -594,6 +599,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_epi(0), 4);
+    mbar_init(bar_epi(1), 4);
     fence_mbar_init();
   }
   if (warp == C::MMA_WARP) {
@@ -895,12 +902,20 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (ok && n_steps > 0) ok = dq_out(n_steps - 1);
     // ------------------------------------------------------------ epilogue --
+    // dV and scale dK in bf16 through shared memory: once every MMA has
+    // completed (bar_done), the K and V tiles are free, and warpgroup h stages
+    // its 64 columns of dV (in sK) and dK (in sV) for all 128 key rows, as
+    // 64-column boxes with the 128-byte swizzle (row r's 16-byte chunk c at c ^
+    // (r mod 8)); one thread of the warpgroup stores both boxes with the TMA
+    // (rows past N clipped).
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, st, 63));
     if (ok) {
       tc_fence_after();
-      const size_t orow = (static_cast<size_t>(bh) * p.N + (kr < p.N ? kr : 0)) * D;
+      uint8_t* dv_row = sK + h * C::CHUNK + r * 128;
+      uint8_t* dk_row = sV + h * C::CHUNK + r * 128;
 #pragma unroll
-      for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
+      for (int cc = 0; cc < D / 2; cc += 32) {
+        const int c0 = h * (D / 2) + cc;
         uint32_t v[32], k[32];
         tmem_ld32(row_addr + C::DV_COL + c0, v);
         tmem_ld32(row_addr + C::DK_COL + c0, k);
@@ -912,18 +927,26 @@ __global__ void __launch_bounds__(384, 1)
           pv2[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
           pk2[e] = pack_bf16x2(__uint_as_float(k[2 * e]) * p.scale, __uint_as_float(k[2 * e + 1]) * p.scale);
         }
-        if (kr < p.N) {
-          uint4* dv4 = reinterpret_cast<uint4*>(p.dv + orow + c0);
-          uint4* dk4 = reinterpret_cast<uint4*>(p.dk + orow + c0);
+        const int cb = cc / 8;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            dv4[u] = make_uint4(pv2[4 * u], pv2[4 * u + 1], pv2[4 * u + 2], pv2[4 * u + 3]);
-            dk4[u] = make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
-          }
+        for (int u = 0; u < 4; ++u) {
+          const int off = ((cb + u) ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(dv_row + off) = make_uint4(pv2[4 * u], pv2[4 * u + 1], pv2[4 * u + 2], pv2[4 * u + 3]);
+          *reinterpret_cast<uint4*>(dk_row + off) = make_uint4(pk2[4 * u], pk2[4 * u + 1], pk2[4 * u + 2], pk2[4 * u + 3]);
+        }
+      }
+      fence_proxy_async_shared();  // the TMA store reads the boxes through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_epi(h));
+      if ((warp & 3u) == 0 && lane == 0) {
+        if (mbar_wait(bar_epi(h), 0, abort_flag, st, 66 + h)) {
+          tma_store_3d(&tmdV, sK + h * C::CHUNK, h * (D / 2), kt * C::BK, bh);
+          tma_store_3d(&tmdK, sV + h * C::CHUNK, h * (D / 2), kt * C::BK, bh);
+          bulk_commit();
         }
       }
     }
-    if (lane == 0) bulk_wait_all();  // the dQ reductions have completed before the CTA exits
+    if (lane == 0) bulk_wait_all();  // the dQ reductions and dK, dV stores have completed before the CTA exits
   }
 
   tc_fence_before();

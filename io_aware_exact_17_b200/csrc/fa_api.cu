@@ -546,6 +546,10 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     return FA_ERR_CUDA;
   // the fp32 dQ accumulator, reduced into in tiles of 32 rows x 32 columns
   if (!fa::make_tmap_3d(&tmdQ, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, 32, 32)) return FA_ERR_CUDA;
+  // dK and dV, stored in 64-column boxes of 128 key rows (d = 128 kernel)
+  CUtensorMap tmdK, tmdV;
+  if (!fa::make_tmap_3d(&tmdK, dk, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmdV, dv, bf, 2, D, N, BH, 64, 128))
+    return FA_ERR_CUDA;
   const long long rows = static_cast<long long>(BH) * Npad;
   fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH, N,
@@ -568,7 +572,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, smem_bytes, stream>>>(
-      tmQ, tmK, tmV, tmdO, tmdQ, p);
+      tmQ, tmK, tmV, tmdO, tmdQ, tmdK, tmdV, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const long long n4 = static_cast<long long>(BH) * N * D / 4;
   const long long cap = static_cast<long long>(device_sms()) * 8;
