@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   DevStatus* st = &g_fa_status;
+  if (threadIdx.x == 0) launch_dependents();  // the dQ conversion may be scheduled (it waits for this grid)
 
   if (warp == C::TMA_WARP && lane == 0) {
     // ------------------------------------------------------------ producer --
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_load_3d(sK + c * C::CHUNK, &tmK, bar_kv, c * 64, kt * C::BK, bh);
       tma_load_3d(sV + c * C::CHUNK, &tmV, bar_kv, c * 64, kt * C::BK, bh);
     }
+    grid_dependency_wait();  // the prologue's -LSE, D (and zeroed dQ accumulator) from here on
     const float* nlse2h = p.nlse2 + static_cast<size_t>(bh) * p.Npad;
     const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
     bool ok = true;
@@ -303,6 +305,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_drain(bar_drain, 0);
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
+    grid_dependency_wait();  // they reduce into the accumulator the prologue zeroed
     const int g = static_cast<int>(warp >> 2);  // query columns 64g .. 64g + 63
     const uint32_t lane_base = (warp & 3u) * 32u;
     const int r = static_cast<int>(lane_base + lane);  // key row (Sᵀ lane); query row for dQ
@@ -612,6 +615,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   DevStatus* st = &g_fa_status;
+  if (threadIdx.x == 0) launch_dependents();  // the dQ conversion may be scheduled (it waits for this grid)
 
   if (warp == C::TMA_WARP && lane == 0) {
     // ------------------------------------------------------------ producer --
@@ -627,6 +631,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_load_3d_hint(sK + c * C::CHUNK, &tmK, bar_kv, c * 64, kt * C::BK, bh, pol_once);
       tma_load_3d_hint(sV + c * C::CHUNK, &tmV, bar_kv, c * 64, kt * C::BK, bh, pol_once);
     }
+    grid_dependency_wait();  // the prologue's -LSE, D (and zeroed dQ accumulator) from here on
     const float* nlse2h = p.nlse2 + static_cast<size_t>(bh) * p.Npad;
     const float* dvh = p.dvec + static_cast<size_t>(bh) * p.Npad;
     bool ok = true;
@@ -753,6 +758,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_drain(bar_drain, 0);
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax --
+    grid_dependency_wait();  // they reduce into the accumulator the prologue zeroed
     const int h = static_cast<int>(warp >> 2);  // this warpgroup's half: queries 64 h .. 64 h + 63 of a step
     const uint32_t lane_base = (warp & 3u) * 32u;
     const int r = static_cast<int>(lane_base + lane);  // key row (Sᵀ lane); d index for dQᵀ
@@ -958,52 +964,53 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // Prologue: per padded query row, D_i = dO_i · O_i and -LSE_i log2(e) (-inf
-// and 0 past N), and zero row i of the dQ accumulator. One warp per row.
+// and 0 past N), and zero row i of the dQ accumulator. D / 8 lanes per row,
+// 16 bytes of O and of dO each; warps stride over the rows.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
                                                             const float* __restrict__ lse, float* nlse2, float* dvec,
                                                             float* dq_acc, int BH, int N, int Npad) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  launch_dependents();  // the main kernel may set up and load K, V (it waits for this grid before the rest)
+  constexpr int LPR = D / 8;     // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp per pass
+  const long long rows = static_cast<long long>(BH) * Npad;
   const uint32_t lane = lane_id();
-  if (row >= static_cast<long long>(BH) * Npad) return;
-  const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
-  if (i >= N) {
-    if (lane == 0) {
-      nlse2[row] = -INFINITY;
-      dvec[row] = 0.f;
-    }
-    return;
-  }
-  constexpr int PER = D / 32;  // elements per lane: 2 or 4
-  const size_t off = (static_cast<size_t>(bh) * N + i) * D + lane * PER;
-  float acc = 0.f;
-  if constexpr (PER == 4) {
-    const uint2 a = *reinterpret_cast<const uint2*>(o + off);
-    const uint2 b = *reinterpret_cast<const uint2*>(dout + off);
-    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-    const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
-    const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
-    acc = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
-    *reinterpret_cast<float4*>(dq_acc + off) = make_float4(0.f, 0.f, 0.f, 0.f);
-  } else {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + off));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + off));
-    acc = a.x * b.x + a.y * b.y;
-    *reinterpret_cast<float2*>(dq_acc + off) = make_float2(0.f, 0.f);
-  }
+  const int sub = static_cast<int>(lane) / LPR, l = static_cast<int>(lane) % LPR;
+  const long long stride = static_cast<long long>(gridDim.x) * 8 * RPW;
+  for (long long r0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * RPW; r0 < rows; r0 += stride) {
+    const long long row = r0 + sub;
+    const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
+    const bool valid = row < rows && i < N;
+    float acc = 0.f;
+    if (valid) {
+      const size_t off = (static_cast<size_t>(bh) * N + i) * D + l * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
-    nlse2[row] = lse[static_cast<size_t>(bh) * N + i] * -1.4426950408889634f;
-    dvec[row] = acc;
+      for (int e = 0; e < 4; ++e) {
+        const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[e]));
+        const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[e]));
+        acc += af.x * bf.x + af.y * bf.y;
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int s = LPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (row < rows && l == 0) {
+      nlse2[row] = valid ? lse[static_cast<size_t>(bh) * N + i] * -1.4426950408889634f : -INFINITY;
+      dvec[row] = valid ? acc : 0.f;
+    }
   }
 }
 
 // Epilogue: dQ = scale * accumulator, rounded to bf16. n4 groups of 4 elements.
 __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq,
                                                           long long n4, float scale) {
+  grid_dependency_wait();  // the main kernel's reductions are complete
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 a = acc[i];

@@ -551,10 +551,23 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   if (!fa::make_tmap_3d(&tmdK, dk, bf, 2, D, N, BH, 64, 128) || !fa::make_tmap_3d(&tmdV, dv, bf, 2, D, N, BH, 64, 128))
     return FA_ERR_CUDA;
   const long long rows = static_cast<long long>(BH) * Npad;
-  fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH, N,
-      Npad);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  {
+    const long long per_block = 8LL * (32 / (D / 8));  // rows one pass of a block covers
+    long long blocks = (rows + per_block - 1) / per_block;
+    const long long cap = static_cast<long long>(device_sms()) * 16;
+    if (blocks > cap) blocks = cap;
+    fa::attn_bwd_prep_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2, dvec, dq_acc, BH,
+        N, Npad);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // The main kernel and the dQ conversion are launched with programmatic
+  // stream serialisation: each may start (set up, load K and V) while the
+  // kernel before it finishes, and waits for it (griddepcontrol.wait) before
+  // reading what it wrote.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   // d = 128: the two softmax warpgroups ping-pong over half steps of 64 queries
   auto kernel = D == 128 ? fa::attn_bwd_pp_kernel<CAUSAL> : fa::attn_bwd_kernel<D, CAUSAL>;
   const int smem_bytes = D == 128 ? fa::BwdPpCfg::SMEM_BYTES : C::SMEM_BYTES;
@@ -571,15 +584,30 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   p.n_t = Npad / 128;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  kernel<<<static_cast<unsigned>(static_cast<long long>(BH) * p.n_t), C::THREADS, smem_bytes, stream>>>(
-      tmQ, tmK, tmV, tmdO, tmdQ, tmdK, tmdV, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(BH) * p.n_t));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, tmQ, tmK, tmV, tmdO, tmdQ, tmdK, tmdV, p) != cudaSuccess) return FA_ERR_CUDA;
+  }
   const long long n4 = static_cast<long long>(BH) * N * D / 4;
   const long long cap = static_cast<long long>(device_sms()) * 8;
   const long long blocks = (n4 + 255) / 256 < cap ? (n4 + 255) / 256 : cap;
-  fa::attn_bwd_dq_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
-                                                                             static_cast<uint2*>(dq), n4, scale);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::attn_bwd_dq_kernel, reinterpret_cast<const float4*>(dq_acc), static_cast<uint2*>(dq),
+                         n4, scale) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 extern "C" {

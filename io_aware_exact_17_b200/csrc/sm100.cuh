@@ -189,6 +189,15 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
 
 // Order this thread's generic-proxy shared-memory accesses before later
 // async-proxy accesses (TMA, tensor core) that are ordered after it.
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialisation may start while the kernel before it on the stream is still
+// running: grid_dependency_wait() returns once that kernel has completed and its
+// memory writes are visible (at once for a kernel launched without the
+// attribute), and launch_dependents() lets the next such kernel start once every
+// CTA of this one has issued it or exited.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
