@@ -896,7 +896,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // The single issuer polls: its wake-up is on the critical path.
             const uint32_t ph = (t == 0 ? pc0 : pc1) & 1u;
             if (t == 0) ++pc0; else ++pc1;
-            ok = mbar_wait(&bar_p[t], ph, &abort_flag, st, 23, kMmaWaitSleepNs);
+            // bf16 at d = 128: spin (the wake-up is on the chain; +0.2-2% on
+            // B200); e4m3 and d = 64 / 256: the blocking wait (the spin
+            // measured 0.5-1% slower or even there)
+            ok = (QK_FP8 || D != 128) ? mbar_wait(&bar_p[t], ph, &abort_flag, st, 23, kMmaWaitSleepNs)
+                                      : mbar_wait_spin(&bar_p[t], ph, &abort_flag, st, 23);
             if (!ok) break;
             tc_fence_after();
             // O_t += P_t V_{j-1}: A = P_t from TMEM (bf16 pairs), B = V tile (MN-major).

@@ -90,6 +90,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // try_wait with a suspend-time hint: a thread whose phase is not complete sleeps
 // in hardware (issuing nothing) until the phase completes or hint_ns pass, so
 // waiting warps leave the issue slots to the warps sharing their SM sub-partition.
+// Non-blocking test of a phase (returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
@@ -108,6 +120,29 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // `sleep_ns` is the suspend-time hint of each poll: 0 polls without sleeping
 // (lowest wake-up latency), larger values leave more issue slots to the warps
 // sharing the sub-partition.
+// mbar_wait by spinning on test_wait: the waiting thread is never suspended,
+// so it resumes as soon as the phase completes, at the cost of issue slots on
+// its sub-partition. Bounded like mbar_wait (the abort flag and the time limit
+// are checked every 64 tests).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               DevStatus* st, uint32_t site) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((n & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        if (st != nullptr && atomicCAS(&st->code, 0u, 5u /*FA_ERR_TIMEOUT*/) == 0u) {
+          st->site = site;
+          st->block = blockIdx.x;
+        }
+        return false;
+      }
+    }
+  }
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           DevStatus* st, uint32_t site, uint32_t sleep_ns = 20000u) {
   if (mbar_try_wait(bar, parity)) return true;
