@@ -783,6 +783,14 @@ def extras(peaks: dict, reps: int) -> dict:
 
         ms_s = time_call(fused_step, reps, flush)
         res["step_quant_k_plus_attn_q_in_kernel"] = {"ms": ms_s, "tflops": fl / (ms_s * 1e-3) / 1e12}
+        # V's codes with one scale per tensor, transposed per head (an amax pass
+        # and a quantise pass; algorithmic bytes: 2 read + 1 written per element)
+        vbytes = v.numel() * 3
+        v8t = torch.empty((v.shape[0], v.shape[1], v.shape[3], v.shape[2]), dtype=torch.uint8, device=v.device)
+        dv = torch.empty(1, dtype=torch.float32, device=v.device)
+        ms_v = time_call(lambda: fa.quant_v_transposed(v, out=v8t, descale=dv), reps, flush)
+        res["quant_v_transposed"] = {"ms": ms_v, "gbs": vbytes / (ms_v * 1e-3) / 1e9,
+                                     "frac": vbytes / (ms_v * 1e-3) / 1e9 / hbm, "bytes": vbytes, "bound": "hbm"}
         return res
 
     guarded(f"fp8_b{FP8_CFG['B']}h{FP8_CFG['H']}n{FP8_CFG['N']}d{FP8_CFG['d']}", fp8)

@@ -244,6 +244,30 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
                             const float* signs, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_quant_v_transposed — V's e4m3 codes with one scale per tensor, written with
+ * the keys along the contiguous dimension.
+ *
+ * Defined by: "FlashAttention-3 (PT)", section "Inovações técnicas", subsection 3
+ * (FP8 operands quantised with a scale; only Q and K are rotated). The pages give
+ * neither V's scale granularity nor its layout; this entry takes one scale per
+ * tensor and no rotation:
+ *   amax = max |v| over the tensor;  descale_out[0] = amax / 448 (1 if amax = 0);
+ *   out_t[bh][c][n] = e4m3(fl(v[bh][n][c] * fl(448 / amax)))  (RNE, saturating),
+ * the same codes fa_hadamard_quant gives with rotate = 0, transposed per head.
+ *
+ * v          device bf16 [BH][N][d] (B and H folded), 16-byte aligned.
+ * out_t      device e4m3 codes [BH][d][N], 16-byte aligned.
+ * descale_out device fp32, 1 value.
+ * BH in 1..65535, N >= 1, d in {64, 128, 256}; BH * N rows at most 2^31 - 4096.
+ * workspace  device, >= FA_QUANT_WORKSPACE_BYTES, 16-byte aligned (the amax word;
+ *            zeroed here). Calls that overlap on the GPU must not share it.
+ * Two launches on `stream` (the amax, then the codes).
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA.
+ */
+fa_status fa_quant_v_transposed(const void* v, void* out_t, float* descale_out, int BH, int N, int d,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_hadamard_quant_multi — fa_hadamard_quant for up to 8 tensors of one shape
  * (for example Q and K) in one launch, each with its own scale: the same codes
  * and descales as one call per tensor, with one grid-wide barrier in place of one
@@ -322,9 +346,9 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block);
 
-/* ABI version of this header: 5 (1, plus the split-key, partial and merge calls in 2,
+/* ABI version of this header: 6 (1, plus the split-key, partial and merge calls in 2,
  * plus per-block e4m3 scales in 3, plus the backward pass in 4, plus
- * fa_fwd_fp8_qrot in 5). */
+ * fa_fwd_fp8_qrot in 5, plus fa_quant_v_transposed in 6). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     hadamard_quant,
     hadamard_quant_blocks,
     hadamard_quant_multi,
+    quant_v_transposed,
     library_path,
     load_library,
     lse_merge,
@@ -27,4 +28,4 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = ["fwd", "fwd_fp8_qrot", "bwd", "bwd_workspace_bytes", "fwd_splitkv", "fwd_partial", "lse_merge", "splitkv_splits", "hadamard_quant",
-           "hadamard_quant_blocks", "hadamard_quant_multi", "device_status", "load_library", "library_path", "FaError"]
+           "hadamard_quant_blocks", "hadamard_quant_multi", "quant_v_transposed", "device_status", "load_library", "library_path", "FaError"]

@@ -80,6 +80,8 @@ def load_library():
         lib.fa_bwd.restype = i
         lib.fa_fwd_fp8_qrot.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, i, vp, vp, vp]
         lib.fa_fwd_fp8_qrot.restype = i
+        lib.fa_quant_v_transposed.argtypes = [vp, vp, vp, i, i, i, vp, sz, vp]
+        lib.fa_quant_v_transposed.restype = i
         _lib = lib
         return lib
 
@@ -478,6 +480,34 @@ def hadamard_quant(x, rotate: bool = True, signs=None, out=None, descale=None, w
                                    _ptr(signs) if (rotate and signs is not None) else None, _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(x.device))
     _check(rc, "fa_hadamard_quant")
+    return out, descale
+
+
+def quant_v_transposed(v, out=None, descale=None, workspace=None):
+    """V's e4m3 codes with one scale per tensor and no rotation, transposed per
+    head, through ``fa_quant_v_transposed``: ``v`` bf16 ``[B, H, N, d]``.
+    Returns ``(codes, descale)``: uint8 codes ``[B, H, d, N]`` (``codes[b, h, c,
+    n]`` is v[b, h, n, c]'s code) and a CUDA fp32 tensor of one element, ``amax /
+    448``."""
+    _require_cuda(v)
+    lib = load_library()
+    if v.dtype != torch.bfloat16 or v.dim() != 4:
+        raise FaError("v must be bf16 [B, H, N, d]")
+    v = v.contiguous()
+    B, H, N, d = v.shape
+    if out is None:
+        out = torch.empty((B, H, d, N), dtype=torch.uint8, device=v.device)
+    if descale is None:
+        descale = torch.empty(1, dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = _workspace(v.device)
+    _tensor_arg(out, "out", v.device, E4M3_DTYPES, (B, H, d, N))
+    _tensor_arg(descale, "descale", v.device, (torch.float32,), min_bytes=4)
+    _tensor_arg(workspace, "workspace", v.device, min_bytes=QUANT_WORKSPACE_BYTES)
+    with torch.cuda.device(v.device):
+        rc = lib.fa_quant_v_transposed(_ptr(v), _ptr(out), _ptr(descale), B * H, N, d, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(v.device))
+    _check(rc, "fa_quant_v_transposed")
     return out, descale
 
 

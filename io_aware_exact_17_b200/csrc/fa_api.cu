@@ -13,6 +13,7 @@
 
 #include "../../include/fa.h"
 #include "attn_bwd.cuh"
+#include "quant_t.cuh"
 #include "attn_fwd.cuh"
 #include "merge.cuh"
 #include "quant.cuh"
@@ -775,6 +776,36 @@ fa_status fa_hadamard_quant(const void* x, void* out, float* descale_out, int64_
   return dispatch_quant_fused(b, descale_out, rows, d, rotate, sg, ws, ws + 1, static_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_quant_v_transposed(const void* v, void* out_t, float* descale_out, int BH, int N, int d,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (v == nullptr || out_t == nullptr || descale_out == nullptr || workspace == nullptr) return FA_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1 || BH > 65535) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < FA_QUANT_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(BH) * N > kQuantMaxRows) return FA_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(out_t, 16) || !aligned(workspace, 16) || !aligned(descale_out, 4))
+    return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* amax_word = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s) != cudaSuccess) return FA_ERR_CUDA;
+  const int64_t n16 = static_cast<int64_t>(BH) * N * d / 8;
+  long long blocks = (n16 + 4095) / 4096;  // 4 chunks of 16 bytes per thread and step
+  const long long cap = static_cast<long long>(device_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  fa::quant_t_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<const uint4*>(v), n16, amax_word);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((N + fa::kQuantTPos - 1) / fa::kQuantTPos), static_cast<unsigned>(BH));
+  const auto* x = static_cast<const __nv_bfloat16*>(v);
+  auto* o = static_cast<uint8_t*>(out_t);
+  switch (d) {
+    case 64: fa::quant_t_kernel<64><<<grid, 256, 0, s>>>(x, o, N, amax_word, descale_out); break;
+    case 128: fa::quant_t_kernel<128><<<grid, 256, 0, s>>>(x, o, N, amax_word, descale_out); break;
+    default: fa::quant_t_kernel<256><<<grid, 256, 0, s>>>(x, o, N, amax_word, descale_out); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_hadamard_quant_multi(const void* const* xs, void* const* outs, float* descales, int ntensors,
                                   int64_t rows, int d, int rotate, const float* signs, void* workspace,
                                   size_t workspace_bytes, void* stream) {
@@ -915,7 +946,7 @@ fa_status fa_device_status(int* code, unsigned int* site, unsigned int* block) {
   return FA_OK;
 }
 
-int fa_abi_version(void) { return 5; }
+int fa_abi_version(void) { return 6; }
 
 #ifdef FA_TEST_HOOKS
 // Test build only (not declared in include/, not in the product library): arm

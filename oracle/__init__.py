@@ -338,6 +338,29 @@ def quantize_per_tensor(x, rotate_qk: bool, signs=None, return_scaled: bool = Fa
     return codes, descale
 
 
+def quantize_v_transposed(v, return_scaled: bool = False):
+    """V's e4m3 codes with one scale per tensor, laid out ``[B, H, d, N]``.
+
+    "FlashAttention-3 (PT)", section "Inovações técnicas", subsection 3
+    quantises the FP8 operands with a scale and rotates only Q and K; the pages
+    give neither V's scale granularity nor its layout. Reading: no rotation, one
+    scale per tensor (amax over all of V, descale = amax / 448, 1 if amax = 0,
+    codes = e4m3_encode(v * 448 / amax)), and the codes of head (b, h) stored
+    with the keys along the last dimension: out[b, h, c, n] = code(v[b, h, n, c]).
+    Returns ``(codes, descale)`` and, with ``return_scaled``, the unrounded scaled
+    values in the same transposed layout.
+    """
+    vf = _as_f64(v)
+    amax = float(np.max(np.abs(vf))) if vf.size else 0.0
+    scaled = np.zeros_like(vf) if amax == 0.0 else vf * (E4M3_MAX / amax)
+    descale = 1.0 if amax == 0.0 else amax / E4M3_MAX
+    scaled_t = np.ascontiguousarray(np.swapaxes(scaled, -1, -2))
+    codes = e4m3_encode(scaled_t)
+    if return_scaled:
+        return codes, descale, scaled_t
+    return codes, descale
+
+
 def quantize_per_block(x, rotate_qk: bool, signs=None, block_rows: int = 128):
     """Rotate (optionally) then quantise ``x`` ``[B, H, N, d]`` to e4m3 with one
     scale per block of ``block_rows`` rows of each head (the last block of a head

@@ -30,8 +30,8 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
     assert {"fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_splits", "fa_fwd_partial",
             "fa_lse_merge"} <= set(names)
-    assert {"fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8_qrot"} <= set(names)
-    assert lib.fa_abi_version() == 5
+    assert {"fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8_qrot", "fa_quant_v_transposed"} <= set(names)
+    assert lib.fa_abi_version() == 6
 
 
 def test_status_strings(lib):
@@ -158,6 +158,23 @@ def test_tail_split_workspace(lib):
         assert _skv(lib, **big) == binding.FA_ERR_INVALID_ARG
         assert _skv(lib, ws=A, wsb=need - 1, **big) == binding.FA_ERR_INVALID_ARG
         assert _skv(lib, ws=A + 16, wsb=need, **big) == binding.FA_ERR_ALIGNMENT
+
+
+def test_v_transposed_quant_argument_errors(lib):
+    def q(v=A, o=A, ds=A, BH=2, N=100, d=128, ws=A, wsb=256):
+        return lib.fa_quant_v_transposed(v, o, ds, BH, N, d, ws, wsb, None)
+    assert q(v=None) == binding.FA_ERR_INVALID_ARG
+    assert q(o=None) == binding.FA_ERR_INVALID_ARG
+    assert q(ds=None) == binding.FA_ERR_INVALID_ARG
+    assert q(ws=None) == binding.FA_ERR_INVALID_ARG
+    assert q(BH=0) == binding.FA_ERR_INVALID_ARG
+    assert q(BH=65536) == binding.FA_ERR_INVALID_ARG
+    assert q(N=0) == binding.FA_ERR_INVALID_ARG
+    assert q(wsb=255) == binding.FA_ERR_INVALID_ARG
+    assert q(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert q(v=MIS) == binding.FA_ERR_ALIGNMENT
+    assert q(o=MIS) == binding.FA_ERR_ALIGNMENT
+    assert q(ds=A + 2) == binding.FA_ERR_ALIGNMENT
 
 
 def test_partial_and_merge_argument_errors(lib):
